@@ -1,0 +1,610 @@
+// Persistent, warp-specialised tcgen05 GEMM for every contraction of the MoE
+// layer: one main loop (TMA / cp.async gather -> shared-memory ring ->
+// tcgen05.mma into a double-buffered TMEM accumulator) and one epilogue per
+// kernel kind.
+//
+// Kernel kinds (rows r of the expert-major, 128-padded row space; e = expert):
+//   UP   H_r = X[tok_r] W1[e]  (gather on A); epilogue stores H and SwiGLU(H)
+//   DOWN Y_r = A_r W2[e]
+//   DH   dA'_r = dO[tok_r] W2[e]^T (gather on A); epilogue reloads H, forms
+//        dS partials, dSwiGLU -> dH, and A_hat = s_r * A_r
+//   DXT  dX~_r = dH_r W1[e]^T
+//   DW1  dW1[e] = X[tok]^T dH   (K runs over the rows of expert e; gather on A)
+//   DW2  dW2[e] = A_hat^T dO[tok] (K runs over the rows of expert e; gather on B)
+//   RTR  router logits X Wr with Wr split into three bf16 parts (hi+mid+lo)
+//   DWR  router weight gradient X^T dz, dz split into two bf16 parts, split-K
+//
+// Sources: page "SonicMoE：突破细粒度MoE硬件效率瓶颈，实现高稀疏性下的极致训练加速"
+// (implementation paragraph: grouped GEMMs with modular fusion, eight kernels);
+// page "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE", section
+// "第二，IO 感知的算子融合" (gather fused into the GEMM, SwiGLU in the
+// epilogue, dH kernel overlapping IO with MMA) and section "软件抽象层 QuACK"
+// (every MoE GEMM = shared main loop + per-kernel epilogue).
+//
+// Roles: warp 0 lane 0 issues TMA loads; warp 1 allocates TMEM and issues the
+// MMAs (one thread); warps 2-5 run the epilogue (one accumulator row each);
+// warps 6-9 (gather kinds only) stream gathered rows with cp.async into the
+// same 128-byte-swizzled layout TMA would produce.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace moe {
+
+enum GemmKind : int { G_UP = 0, G_DOWN, G_DH, G_DXT, G_DW1, G_DW2, G_RTR, G_DWR };
+
+struct GemmParams {
+  CUtensorMap tmA;  // TMA map of A (kinds whose A is not gathered)
+  CUtensorMap tmB;  // TMA map of B (kinds whose B is not gathered)
+  DevStatus st;
+  const int* offsets;      // [E+1] 128-aligned segment starts
+  const int* counts;       // [E]
+  const int* tile_expert;  // [R_max/128]
+  const int* row_tok;      // [R_max]  token of each row, -1 for padding
+  const float* row_gate;   // [R_max]
+  const __nv_bfloat16* gsrc;  // gathered operand source [T, gld]
+  int gld;
+  int T, d, n, E, Epad;
+  int num_n_tiles;
+  int num_m_tiles;   // non-grouped-M kinds
+  int ksplit;        // DWR
+  int ksplit_rows;   // DWR, multiple of 64
+  __nv_bfloat16* out0;
+  __nv_bfloat16* out1;
+  const __nv_bfloat16* hin;
+  float* outf;
+  const float* bias;
+};
+
+template <int KIND>
+struct KindTraits {
+  static constexpr bool kGroupedM = (KIND == G_UP || KIND == G_DOWN || KIND == G_DH || KIND == G_DXT);
+  static constexpr bool kGroupedK = (KIND == G_DW1 || KIND == G_DW2);
+  static constexpr bool kAGather = (KIND == G_UP || KIND == G_DH || KIND == G_DW1);
+  static constexpr bool kBGather = (KIND == G_DW2);
+  static constexpr bool kGather = kAGather || kBGather;
+  static constexpr bool kAMN = (KIND == G_DW1 || KIND == G_DW2 || KIND == G_DWR);
+  static constexpr bool kBMN = !(KIND == G_DH || KIND == G_DXT);
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
+constexpr int kStageBudget = 200 * 1024;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStagesRaw = kStageBudget / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // accumulator buffers start at power-of-two column offsets
+  static constexpr int kAccStride = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);
+  static constexpr int kTmemCols = 2 * kAccStride;
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;  // barriers + alignment slack
+};
+
+struct TileInfo {
+  int e, mt, nt, m0, n0, krow0, nkb, split;
+};
+
+template <int KIND, int BN>
+__device__ __forceinline__ int gemm_num_tiles(const GemmParams& p) {
+  using KT = KindTraits<KIND>;
+  if constexpr (KT::kGroupedM) {
+    return (__ldg(p.offsets + p.E) / kBM) * p.num_n_tiles;
+  } else if constexpr (KT::kGroupedK) {
+    return p.E * p.num_m_tiles * p.num_n_tiles;
+  } else if constexpr (KIND == G_DWR) {
+    return p.num_m_tiles * p.num_n_tiles * p.ksplit;
+  } else {
+    return p.num_m_tiles * p.num_n_tiles;
+  }
+}
+
+template <int KIND, int BN>
+__device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
+  using KT = KindTraits<KIND>;
+  TileInfo t;
+  t.split = 0;
+  t.krow0 = 0;
+  if constexpr (KT::kGroupedM) {
+    t.mt = tile / p.num_n_tiles;
+    t.nt = tile - t.mt * p.num_n_tiles;
+    t.e = __ldg(p.tile_expert + t.mt);
+    t.m0 = t.mt * kBM;
+    if constexpr (KIND == G_UP) t.n0 = t.nt * (BN / 2);
+    else t.n0 = t.nt * BN;
+    const int K = (KIND == G_UP || KIND == G_DH) ? p.d : (KIND == G_DOWN ? p.n : 2 * p.n);
+    t.nkb = K / kBK;
+  } else if constexpr (KT::kGroupedK) {
+    const int per_e = p.num_m_tiles * p.num_n_tiles;
+    t.e = tile / per_e;
+    const int rem = tile - t.e * per_e;
+    t.mt = rem / p.num_n_tiles;
+    t.nt = rem - t.mt * p.num_n_tiles;
+    t.m0 = t.mt * kBM;
+    t.n0 = t.nt * BN;
+    t.krow0 = __ldg(p.offsets + t.e);
+    t.nkb = (__ldg(p.counts + t.e) + kBK - 1) / kBK;
+  } else if constexpr (KIND == G_DWR) {
+    const int per_s = p.num_m_tiles * p.num_n_tiles;
+    t.split = tile / per_s;
+    const int rem = tile - t.split * per_s;
+    t.mt = rem / p.num_n_tiles;
+    t.nt = rem - t.mt * p.num_n_tiles;
+    t.e = 0;
+    t.m0 = t.mt * kBM;
+    t.n0 = t.nt * BN;
+    t.krow0 = t.split * p.ksplit_rows;
+    int rows = p.T - t.krow0;
+    if (rows > p.ksplit_rows) rows = p.ksplit_rows;
+    t.nkb = rows > 0 ? (rows + kBK - 1) / kBK : 0;
+  } else {  // G_RTR
+    t.mt = tile / p.num_n_tiles;
+    t.nt = tile - t.mt * p.num_n_tiles;
+    t.e = 0;
+    t.m0 = t.mt * kBM;
+    t.n0 = t.nt * BN;
+    t.nkb = p.d / kBK;
+  }
+  return t;
+}
+
+// Byte offset of 16-byte chunk `c` of 128-byte line `i` in a 128B-swizzled tile.
+__device__ __forceinline__ uint32_t sw128(int line, int chunk) {
+  return (uint32_t)(line * 128 + ((chunk ^ (line & 7)) << 4));
+}
+
+// ----------------------------------------------------------------- producer
+template <int KIND, int BN>
+__device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t, int kb, uint32_t a_s,
+                                          uint32_t b_s, uint32_t bar) {
+  const void* tA = &p.tmA;
+  const void* tB = &p.tmB;
+  const int k0 = kb * kBK;
+  if constexpr (KIND == G_UP) {
+    constexpr int nb = BN / 64, half = nb / 2;
+    mbar_arrive_expect_tx(bar, nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) {
+      const int col = (j < half) ? (t.n0 + 64 * j) : (p.n + t.n0 + 64 * (j - half));
+      tma_load_2d(b_s + j * kBoxBytes, tB, bar, col, t.e * p.d + k0);
+    }
+  } else if constexpr (KIND == G_DOWN) {
+    constexpr int nb = BN / 64;
+    mbar_arrive_expect_tx(bar, kABytes + nb * kBoxBytes);
+    tma_load_2d(a_s, tA, bar, k0, t.m0);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.e * p.n + k0);
+  } else if constexpr (KIND == G_DH) {
+    mbar_arrive_expect_tx(bar, BN * 128);
+    tma_load_2d(b_s, tB, bar, k0, t.e * p.n + t.n0);
+  } else if constexpr (KIND == G_DXT) {
+    mbar_arrive_expect_tx(bar, kABytes + BN * 128);
+    tma_load_2d(a_s, tA, bar, k0, t.m0);
+    tma_load_2d(b_s, tB, bar, k0, t.e * p.d + t.n0);
+  } else if constexpr (KIND == G_DW1) {
+    constexpr int nb = BN / 64;
+    mbar_arrive_expect_tx(bar, nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.krow0 + k0);
+  } else if constexpr (KIND == G_DW2) {
+    mbar_arrive_expect_tx(bar, 2 * kBoxBytes);
+    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar, t.m0 + 64 * h, t.krow0 + k0);
+  } else if constexpr (KIND == G_RTR) {
+    constexpr int nb = BN / 64;
+    mbar_arrive_expect_tx(bar, kABytes + nb * kBoxBytes);
+    tma_load_2d(a_s, tA, bar, k0, t.m0);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, k0);
+  } else {  // G_DWR
+    constexpr int nb = BN / 64;
+    mbar_arrive_expect_tx(bar, 2 * kBoxBytes + nb * kBoxBytes);
+    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar, t.m0 + 64 * h, t.krow0 + k0);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.krow0 + k0);
+  }
+}
+
+// ----------------------------------------------------------------- epilogue helpers
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d4[q] = w;
+  }
+}
+__device__ __forceinline__ void load_row32_bf16(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w = s4[q];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      v[8 * q + 2 * i] = f.x;
+      v[8 * q + 2 * i + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void zero32(float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = 0.f;
+}
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+// ----------------------------------------------------------------- kernel
+template <int KIND, int BN>
+__global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using KT = KindTraits<KIND>;
+  using SH = GemmShape<BN>;
+  constexpr int S = SH::kStages;
+  constexpr int kLag = S - 1;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(BN, KT::kAMN, KT::kBMN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SH::kBarOffset);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
+  uint64_t* acc_empty = bars + 2 * S + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1 + (KT::kGather ? 128 : 0));
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if constexpr (!(KIND == G_UP || KIND == G_DH || KIND == G_DW1)) tma_prefetch_desc(&p.tmA);
+    if constexpr (!KT::kBGather) tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), SH::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = gemm_num_tiles<KIND, BN>(p);
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_s = base + s * SH::kStageBytes;
+          issue_tma<KIND, BN>(p, t, kb, a_s, a_s + kABytes, smem_u32(&full[s]));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    int it = 0, tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if (t.nkb == 0) continue;
+      const int b = tcount & 1;
+      const int use = tcount >> 1;
+      if (!mbar_wait(smem_u32(&acc_empty[b]), (use & 1) ^ 1, abort_flag, p.st, KIND * 16 + 2)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(b * SH::kAccStride);
+      for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+        const int s = it % S;
+        if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_s = base + s * SH::kStageBytes;
+          const uint32_t b_s = a_s + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = KT::kAMN ? smem_desc_sw128(a_s + kk * 2048, kBoxBytes, 1024)
+                                         : smem_desc_sw128(a_s + kk * 32, 16, 1024);
+            const uint64_t bd = KT::kBMN ? smem_desc_sw128(b_s + kk * 2048, kBoxBytes, 1024)
+                                         : smem_desc_sw128(b_s + kk * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&empty[s]));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(smem_u32(&acc_full[b]));
+      __syncwarp();
+      ++tcount;
+    }
+  } else if (warp < 6) {
+    // ---------------- epilogue: one accumulator row per thread
+    const int q = warp & 3;
+    const int rloc = q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if constexpr (KT::kGroupedK) {
+        if (t.nkb == 0) {  // expert without tokens: its weight gradient is zero
+          const int M = (KIND == G_DW1) ? p.d : p.n;
+          const int N = (KIND == G_DW1) ? 2 * p.n : p.d;
+          const int m = t.m0 + rloc;
+          if (m < M) {
+            float z[32];
+            zero32(z);
+            for (int c = 0; c < BN; c += 32) store_row32_bf16(p.out0 + ((size_t)t.e * M + m) * N + t.n0 + c, z);
+          }
+          continue;
+        }
+      } else if constexpr (KIND == G_DWR) {
+        if (t.nkb == 0) {
+          const int m = t.m0 + rloc;
+          if (m < p.d) {
+            float* dst = p.outf + ((size_t)t.split * p.d + m) * p.Epad + t.nt * 64;
+            for (int c = 0; c < 64; ++c) dst[c] = 0.f;
+          }
+          continue;
+        }
+      }
+      const int b = tcount & 1;
+      const int use = tcount >> 1;
+      if (!mbar_wait(smem_u32(&acc_full[b]), use & 1, abort_flag, p.st, KIND * 16 + 4)) break;
+      tc_fence_after();
+      const uint32_t tacc = lane_addr + (uint32_t)(b * SH::kAccStride);
+
+      if constexpr (KIND == G_UP) {
+        constexpr int BNh = BN / 2;
+        const int r = t.m0 + rloc;
+        __nv_bfloat16* Hrow = p.out0 + (size_t)r * (2 * p.n);
+        __nv_bfloat16* Arow = p.out1 + (size_t)r * p.n;
+#pragma unroll 1
+        for (int c = 0; c < BNh; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tacc + c, g);
+          tmem_ld32(tacc + BNh + c, u);
+          tc_wait_ld();
+          float gv[32], uv[32], av[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            gv[i] = bf16_round(__uint_as_float(g[i]));
+            uv[i] = bf16_round(__uint_as_float(u[i]));
+            av[i] = gv[i] * sigmoidf_(gv[i]) * uv[i];
+          }
+          store_row32_bf16(Hrow + t.n0 + c, gv);
+          store_row32_bf16(Hrow + p.n + t.n0 + c, uv);
+          store_row32_bf16(Arow + t.n0 + c, av);
+        }
+      } else if constexpr (KIND == G_DOWN || KIND == G_DXT) {
+        const int r = t.m0 + rloc;
+        __nv_bfloat16* row = p.out0 + (size_t)r * p.d + t.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(tacc + c, a);
+          tc_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+          store_row32_bf16(row + c, v);
+        }
+      } else if constexpr (KIND == G_DH) {
+        const int r = t.m0 + rloc;
+        const float s = __ldg(p.row_gate + r);
+        const __nv_bfloat16* Hrow = p.hin + (size_t)r * (2 * p.n);
+        __nv_bfloat16* dHrow = p.out0 + (size_t)r * (2 * p.n);
+        __nv_bfloat16* Ahrow = p.out1 + (size_t)r * p.n;
+        float dsum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(tacc + c, a);
+          float gv[32], uv[32];
+          load_row32_bf16(Hrow + t.n0 + c, gv);
+          load_row32_bf16(Hrow + p.n + t.n0 + c, uv);
+          tc_wait_ld();
+          float dg[32], du[32], ah[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float dap = __uint_as_float(a[i]);
+            const float g = gv[i], u = uv[i];
+            const float sg = sigmoidf_(g);
+            const float silu = g * sg;
+            const float A = silu * u;
+            dsum = fmaf(dap, A, dsum);
+            const float dA = s * dap;
+            dg[i] = dA * u * sg * (1.0f + g * (1.0f - sg));
+            du[i] = dA * silu;
+            ah[i] = s * A;
+          }
+          store_row32_bf16(dHrow + t.n0 + c, dg);
+          store_row32_bf16(dHrow + p.n + t.n0 + c, du);
+          store_row32_bf16(Ahrow + t.n0 + c, ah);
+        }
+        p.outf[(size_t)r * p.num_n_tiles + t.nt] = dsum;
+      } else if constexpr (KT::kGroupedK) {
+        const int M = (KIND == G_DW1) ? p.d : p.n;
+        const int N = (KIND == G_DW1) ? 2 * p.n : p.d;
+        const int m = t.m0 + rloc;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(tacc + c, a);
+          tc_wait_ld();
+          if (m < M) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+            store_row32_bf16(p.out0 + ((size_t)t.e * M + m) * N + t.n0 + c, v);
+          }
+        }
+      } else if constexpr (KIND == G_RTR) {
+        const int trow = t.m0 + rloc;
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t hi[32], mid[32], lo[32];
+          tmem_ld32(tacc + c, hi);
+          tmem_ld32(tacc + 64 + c, mid);
+          tmem_ld32(tacc + 128 + c, lo);
+          tc_wait_ld();
+          if (trow < p.T) {
+            float* dst = p.outf + (size_t)trow * p.E;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int e = t.nt * 64 + c + i;
+              if (e < p.E) {
+                float z = __uint_as_float(hi[i]) + __uint_as_float(mid[i]) + __uint_as_float(lo[i]);
+                if (p.bias) z += __ldg(p.bias + e);
+                dst[e] = z;
+              }
+            }
+          }
+        }
+      } else {  // G_DWR
+        const int m = t.m0 + rloc;
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t hi[32], lo[32];
+          tmem_ld32(tacc + c, hi);
+          tmem_ld32(tacc + 64 + c, lo);
+          tc_wait_ld();
+          if (m < p.d) {
+            float* dst = p.outf + ((size_t)t.split * p.d + m) * p.Epad + t.nt * 64 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 v = make_float4(__uint_as_float(hi[i]) + __uint_as_float(lo[i]),
+                                     __uint_as_float(hi[i + 1]) + __uint_as_float(lo[i + 1]),
+                                     __uint_as_float(hi[i + 2]) + __uint_as_float(lo[i + 2]),
+                                     __uint_as_float(hi[i + 3]) + __uint_as_float(lo[i + 3]));
+              *reinterpret_cast<float4*>(dst + i) = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[b]));
+      ++tcount;
+    }
+  } else if constexpr (KT::kGather) {
+    // ---------------- gather producers (warps 6-9): cp.async rows into the swizzled ring
+    const int gt = threadIdx.x - 192;  // 0..127
+    const int chunk = gt & 7;
+    const int line0 = gt >> 3;         // 0..15
+    int it = 0;
+    int pending = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if constexpr (KIND == G_UP || KIND == G_DH) {
+        // A tile = 128 gathered rows x 64 columns; this thread: lines line0 + 16 j
+        const __nv_bfloat16* src[8];
+        uint32_t nbytes[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int tok = __ldg(p.row_tok + t.m0 + line0 + 16 * j);
+          src[j] = p.gsrc + (size_t)(tok < 0 ? 0 : tok) * p.gld + chunk * 8;
+          nbytes[j] = tok < 0 ? 0u : 16u;
+        }
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 5)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_s = base + s * SH::kStageBytes;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) cp_async_16(a_s + sw128(line0 + 16 * j, chunk), src[j] + kb * kBK, nbytes[j]);
+          cp_async_commit();
+          if (pending == kLag) {
+            cp_async_wait<kLag>();
+            fence_proxy_async_smem();
+            mbar_arrive(smem_u32(&full[(it - kLag) % S]));
+          } else {
+            ++pending;
+          }
+        }
+      } else {
+        // MN-major gathered operand: 64 K-rows (tokens) per k-block
+        constexpr int nbox = (KIND == G_DW1) ? 2 : BN / 64;
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst0 = base + s * SH::kStageBytes + (KIND == G_DW1 ? 0 : kABytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = line0 + 16 * j;
+            const int tok = __ldg(p.row_tok + t.krow0 + kb * kBK + i);
+#pragma unroll
+            for (int bx = 0; bx < nbox; ++bx) {
+              const int col = (KIND == G_DW1 ? t.m0 : t.n0) + 64 * bx + chunk * 8;
+              const bool valid = tok >= 0 && (KIND != G_DW1 || col < p.d);
+              const __nv_bfloat16* src = p.gsrc + (valid ? ((size_t)tok * p.gld + col) : 0);
+              cp_async_16(dst0 + bx * kBoxBytes + sw128(i, chunk), src, valid ? 16u : 0u);
+            }
+          }
+          cp_async_commit();
+          if (pending == kLag) {
+            cp_async_wait<kLag>();
+            fence_proxy_async_smem();
+            mbar_arrive(smem_u32(&full[(it - kLag) % S]));
+          } else {
+            ++pending;
+          }
+        }
+      }
+    }
+    // drain: the last `pending` k-blocks are complete after wait_group 0
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (ok) {
+      for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&full[(it - k) % S]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, SH::kTmemCols);
+  }
+}
+
+}  // namespace moe

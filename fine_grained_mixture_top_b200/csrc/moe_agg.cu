@@ -1,0 +1,232 @@
+// Bandwidth-bound kernels: expert aggregation (forward O and backward dX) and
+// the router backward (dS reduction, softmax-over-selected-logits Jacobian).
+//
+// Sources: page "SonicMoE：突破细粒度MoE硬件效率瓶颈，实现高稀疏性下的极致训练加速",
+// implementation paragraph (expert aggregation kernel O in the forward, dX
+// aggregation in the backward; the layer is grouped GEMMs plus aggregation)
+// and algorithm paragraph (router gradient without cached activations).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+__device__ __forceinline__ void acc8(float (&acc)[8], uint4 v, float g) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    acc[2 * i] = fmaf(g, f.x, acc[2 * i]);
+    acc[2 * i + 1] = fmaf(g, f.y, acc[2 * i + 1]);
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  return o;
+}
+
+// O[t, 8c .. 8c+8) = sum_p gate_p * Y[row_p, 8c .. 8c+8)   (fp32 accumulate)
+__global__ void __launch_bounds__(256) aggregate_fwd_kernel(int T, int d8, const int* __restrict__ tok_ptr,
+                                                            const int* __restrict__ pair_row,
+                                                            const float* __restrict__ pair_gate,
+                                                            const uint4* __restrict__ Y, uint4* __restrict__ O) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)T * d8) return;
+  const int t = (int)(idx / d8), c = (int)(idx - (int64_t)t * d8);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const int p0 = __ldg(tok_ptr + t), p1 = __ldg(tok_ptr + t + 1);
+  int p = p0;
+  for (; p + 4 <= p1; p += 4) {
+    uint4 v[4];
+    float g[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[j] = __ldg(Y + (size_t)__ldg(pair_row + p + j) * d8 + c);
+      g[j] = __ldg(pair_gate + p + j);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc8(acc, v[j], g[j]);
+  }
+  for (; p < p1; ++p) acc8(acc, __ldg(Y + (size_t)__ldg(pair_row + p) * d8 + c), __ldg(pair_gate + p));
+  O[idx] = pack8(acc);
+}
+
+cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pair_row, const float* pair_gate,
+                                 const __nv_bfloat16* Y, __nv_bfloat16* O, cudaStream_t s) {
+  const int d8 = d / 8;
+  const int64_t n = (int64_t)T * d8;
+  aggregate_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      T, d8, tok_ptr, pair_row, pair_gate, reinterpret_cast<const uint4*>(Y), reinterpret_cast<uint4*>(O));
+  return cudaGetLastError();
+}
+
+// One warp per token.  dS_p = sum of the dH kernel's per-N-tile partials of
+// row(p); dz_p = s_p (dS_p - sum_j s_j dS_j).  Writes dz per pair (fp32) and
+// the token's dense dz row split into bf16 hi + lo parts for the tensor-core
+// dWr = X^T dz GEMM (layout: group g of 64 experts at columns [128 g, 128 g +
+// 128): hi parts then lo parts).
+__global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad, int nts,
+                                                         const int* __restrict__ tok_ptr,
+                                                         const int* __restrict__ pair_row,
+                                                         const int* __restrict__ pair_expert,
+                                                         const float* __restrict__ pair_gate,
+                                                         const float* __restrict__ dS_part, float* __restrict__ dz_pair,
+                                                         __nv_bfloat16* __restrict__ dz_split) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
+  float inner = 0.f;
+  for (int p = p0 + lane; p < p1; p += 32) {
+    const float* part = dS_part + (size_t)pair_row[p] * nts;
+    float ds = 0.f;
+    for (int j = 0; j < nts; ++j) ds += part[j];
+    dz_pair[p] = ds;  // dS for now
+    inner += pair_gate[p] * ds;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) inner += __shfl_xor_sync(0xffffffffu, inner, o);
+  __syncwarp();
+  __nv_bfloat16* row = dz_split + (size_t)t * 2 * Epad;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+  for (int c = lane; c < 2 * Epad; c += 32) row[c] = zero;
+  __syncwarp();
+  for (int p = p0 + lane; p < p1; p += 32) {
+    const float dz = pair_gate[p] * (dz_pair[p] - inner);
+    dz_pair[p] = dz;
+    const int e = pair_expert[p];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(dz);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(dz - __bfloat162float(hi));
+    const int col = (e >> 6) * 128 + (e & 63);
+    row[col] = hi;
+    row[col + 64] = lo;
+  }
+}
+
+cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
+                              const int* pair_expert, const float* pair_gate, const float* dS_part,
+                              float* dz_pair, __nv_bfloat16* dz_split, cudaStream_t s) {
+  router_bwd_kernel<<<(T + 7) / 8, 256, 0, s>>>(T, E, Epad, nts, tok_ptr, pair_row, pair_expert, pair_gate,
+                                                dS_part, dz_pair, dz_split);
+  return cudaGetLastError();
+}
+
+// WrT[e, i] = Wr[i, e]
+__global__ void transpose_kernel(const float* __restrict__ in, float* __restrict__ out, int rows, int cols) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+cudaError_t launch_transpose_wr(int d, int E, const float* Wr, float* WrT, cudaStream_t s) {
+  dim3 grid((E + 31) / 32, (d + 31) / 32), block(32, 8);
+  transpose_kernel<<<grid, block, 0, s>>>(Wr, WrT, d, E);
+  return cudaGetLastError();
+}
+
+// dWr[i, e] = sum over K splits of the split-K partials
+__global__ void dwr_reduce_kernel(int d, int E, int Epad, int splits, const float* __restrict__ part,
+                                  float* __restrict__ dWr) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)d * E) return;
+  const int i = (int)(idx / E), e = (int)(idx - (int64_t)i * E);
+  float s = 0.f;
+  for (int k = 0; k < splits; ++k) s += part[((size_t)k * d + i) * Epad + e];
+  dWr[idx] = s;
+}
+
+cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s) {
+  const int64_t n = (int64_t)d * E;
+  dwr_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d, E, Epad, splits, part, dWr);
+  return cudaGetLastError();
+}
+
+// dX[t, 8c .. 8c+8) = sum_p dX~[row_p, ...] (+ sum_p dz_p WrT[e_p, ...])
+__global__ void __launch_bounds__(256) aggregate_bwd_kernel(int T, int d8, const int* __restrict__ tok_ptr,
+                                                            const int* __restrict__ pair_row,
+                                                            const int* __restrict__ pair_expert,
+                                                            const uint4* __restrict__ dXt,
+                                                            const float* __restrict__ dz_pair,
+                                                            const float4* __restrict__ WrT, int router_grad,
+                                                            uint4* __restrict__ dX) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)T * d8) return;
+  const int t = (int)(idx / d8), c = (int)(idx - (int64_t)t * d8);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const int p0 = __ldg(tok_ptr + t), p1 = __ldg(tok_ptr + t + 1);
+  int p = p0;
+  for (; p + 4 <= p1; p += 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = __ldg(dXt + (size_t)__ldg(pair_row + p + j) * d8 + c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc8(acc, v[j], 1.0f);
+  }
+  for (; p < p1; ++p) acc8(acc, __ldg(dXt + (size_t)__ldg(pair_row + p) * d8 + c), 1.0f);
+  if (router_grad) {
+    for (p = p0; p < p1; ++p) {
+      const float dz = __ldg(dz_pair + p);
+      const float4* w = WrT + ((size_t)__ldg(pair_expert + p) * d8 + c) * 2;
+      const float4 a = __ldg(w), b = __ldg(w + 1);
+      acc[0] = fmaf(dz, a.x, acc[0]);
+      acc[1] = fmaf(dz, a.y, acc[1]);
+      acc[2] = fmaf(dz, a.z, acc[2]);
+      acc[3] = fmaf(dz, a.w, acc[3]);
+      acc[4] = fmaf(dz, b.x, acc[4]);
+      acc[5] = fmaf(dz, b.y, acc[5]);
+      acc[6] = fmaf(dz, b.z, acc[6]);
+      acc[7] = fmaf(dz, b.w, acc[7]);
+    }
+  }
+  dX[idx] = pack8(acc);
+}
+
+cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const int* pair_expert,
+                                 const __nv_bfloat16* dXt, const float* dz_pair, const float* WrT, int router_grad,
+                                 __nv_bfloat16* dX, cudaStream_t s) {
+  const int d8 = d / 8;
+  const int64_t n = (int64_t)T * d8;
+  aggregate_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      T, d8, tok_ptr, pair_row, pair_expert, reinterpret_cast<const uint4*>(dXt), dz_pair,
+      reinterpret_cast<const float4*>(WrT), router_grad, reinterpret_cast<uint4*>(dX));
+  return cudaGetLastError();
+}
+
+// Failure-detection self test: one thread waits on an mbarrier that nothing
+// will ever complete, through the same bounded wait the GEMM kernels use, and
+// must come back with ST_TIMEOUT recorded in the status word.
+__global__ void wait_selftest_kernel(int* out, DevStatus st) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, st, 999);
+    out[0] = ok ? 1 : 0;
+    mbar_arrive(smem_u32(&bar));  // complete the phase so the barrier is left consistent
+  }
+}
+
+cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(flag, st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,520 @@
+// C-ABI layer (include/moe.h): argument checks, workspace carving, TMA
+// descriptor encoding and the launch order of the layer's kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+using namespace moe;
+
+namespace {
+
+// ----------------------------------------------------------------- status word
+__device__ int g_status_word[2];  // [0] first error code, [1] where it happened
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+long long g_spin_limit = 1ll << 31;
+std::mutex g_mu;
+
+bool device_state(int* dev_out, int** status_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return false;
+    g_status_ptr[dev] = static_cast<int*>(p);
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    g_num_sms[dev] = sms;
+  }
+  *dev_out = dev;
+  *status_out = g_status_ptr[dev];
+  *sms_out = g_num_sms[dev];
+  return true;
+}
+
+// ----------------------------------------------------------------- TMA encoding
+using EncodeFn = decltype(&cuTensorMapEncodeTiled);
+EncodeFn g_encode = nullptr;
+
+bool get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return false;
+  g_encode = reinterpret_cast<EncodeFn>(fn);
+  return true;
+}
+
+// 2-D bf16 row-major tensor [rows, cols], box [box_rows, box_cols], 128B swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+               uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- shapes
+struct Plan {
+  int64_t T;
+  int d, E, n, K, Epad, Ew, nchunks;
+  int64_t P_max, R_max;
+  int bn_up, bn_down, bn_dh, bn_dxt, bn_dw1, bn_dw2;
+  int nts;  // N tiles of the dH kernel (dS partials per row)
+  int ksplit, ksplit_rows;
+};
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
+  if (!dims || !opts) return MOE_ERR_INVALID_ARG;
+  if (opts->round_mode < 0 || opts->round_mode > 2 || (opts->router_grad != 0 && opts->router_grad != 1))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t T = dims->T;
+  const int d = dims->d, E = dims->E, n = dims->n, K = dims->K;
+  if (T < 1 || d < 128 || n < 64 || E < 1 || K < 1) return MOE_ERR_UNSUPPORTED;
+  if (d % 128 != 0 || n % 64 != 0 || K > 32 || K > E || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)std::max(K, E) >= (int64_t(1) << 31) - 4096 * 1024) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)d * 2 * n * E >= (int64_t(1) << 40)) return MOE_ERR_UNSUPPORTED;
+  Plan p;
+  p.T = T;
+  p.d = d;
+  p.E = E;
+  p.n = n;
+  p.K = K;
+  p.Epad = (int)cdiv(E, 64) * 64;
+  p.Ew = (int)cdiv(E, 32);
+  p.nchunks = (int)cdiv(T, kChunk);
+  p.P_max = T * K;
+  if (opts->round_mode != 0) p.P_max = std::min<int64_t>(T * E, T * K + (int64_t)(kTile - 1) * E);
+  p.R_max = cdiv(p.P_max + (int64_t)(kTile - 1) * E, kTile) * kTile;
+  p.bn_up = (n % 128 == 0) ? 256 : 128;
+  p.bn_down = (d % 256 == 0) ? 256 : 128;
+  p.bn_dh = (n % 256 == 0) ? 256 : ((n % 128 == 0) ? 128 : 64);
+  p.bn_dxt = p.bn_down;
+  p.bn_dw1 = ((2 * n) % 256 == 0) ? 256 : 128;
+  p.bn_dw2 = p.bn_down;
+  p.nts = n / p.bn_dh;
+  // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
+  const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
+  int64_t ks = std::max<int64_t>(1, cdiv(296, mn_tiles));
+  ks = std::min<int64_t>(ks, cdiv(T, 64));
+  p.ksplit_rows = (int)(cdiv(cdiv(T, ks), 64) * 64);
+  p.ksplit = (int)cdiv(T, p.ksplit_rows);
+  *pl = p;
+  return MOE_OK;
+}
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* r = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off = align256(off + count * sizeof(T));
+    return r;
+  }
+};
+
+struct RouteWs {
+  __nv_bfloat16* Wr_split;
+  float* logits;
+  int* hist;
+  int* local_rank;
+  uint32_t* member;
+  uint32_t* final_;
+  int* cnt;
+};
+size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
+  Carve c{static_cast<char*>(ws)};
+  w->Wr_split = c.take<__nv_bfloat16>((size_t)p.d * 3 * p.Epad);
+  w->logits = c.take<float>((size_t)p.T * p.E);
+  w->hist = c.take<int>((size_t)p.nchunks * p.E);
+  w->local_rank = c.take<int>((size_t)p.P_max);
+  w->member = c.take<uint32_t>((size_t)p.T * p.Ew);
+  w->final_ = c.take<uint32_t>((size_t)p.T * p.Ew);
+  w->cnt = c.take<int>((size_t)p.T);
+  return c.off;
+}
+
+struct FwdWs {
+  __nv_bfloat16* A;
+  __nv_bfloat16* Y;
+};
+size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
+  Carve c{static_cast<char*>(ws)};
+  w->A = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
+  w->Y = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
+  return c.off;
+}
+
+struct BwdWs {
+  __nv_bfloat16 *dH, *Ahat, *dXt, *dz_split;
+  float *dS_part, *dz_pair, *WrT, *dWr_part;
+};
+size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
+  Carve c{static_cast<char*>(ws)};
+  w->dH = c.take<__nv_bfloat16>((size_t)p.R_max * 2 * p.n);
+  w->Ahat = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
+  w->dXt = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
+  w->dS_part = c.take<float>((size_t)p.R_max * p.nts);
+  w->dz_split = c.take<__nv_bfloat16>((size_t)p.T * 2 * p.Epad);
+  w->dz_pair = c.take<float>((size_t)p.P_max);
+  w->WrT = c.take<float>((size_t)p.E * p.d);
+  w->dWr_part = c.take<float>((size_t)p.ksplit * p.d * p.Epad);
+  return c.off;
+}
+
+inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bool routing_ok(const moe_routing* rt, const Plan& p, bool need_probs) {
+  if (!rt) return false;
+  const void* req[] = {rt->topk_idx, rt->topk_gate, rt->tok_ptr, rt->pair_expert, rt->pair_gate, rt->pair_row,
+                       rt->counts, rt->offsets, rt->row_tok, rt->row_gate, rt->tile_expert};
+  for (const void* q : req)
+    if (!q || !aligned16(q)) return false;
+  if (need_probs && (!rt->probs || !aligned16(rt->probs))) return false;
+  if (rt->logits && !aligned16(rt->logits)) return false;
+  return rt->P_max >= p.P_max && rt->R_max >= p.R_max;
+}
+
+RouteArgs route_args(const Plan& p, const moe_routing* rt, const RouteWs& w) {
+  RouteArgs a;
+  a.T = (int)p.T;
+  a.d = p.d;
+  a.E = p.E;
+  a.K = p.K;
+  a.Epad = p.Epad;
+  a.Wr = nullptr;
+  a.Wr_split = w.Wr_split;
+  a.logits = rt->logits ? rt->logits : w.logits;
+  a.probs = rt->probs;
+  a.topk_idx = rt->topk_idx;
+  a.topk_gate = rt->topk_gate;
+  a.tok_ptr = rt->tok_ptr;
+  a.pair_expert = rt->pair_expert;
+  a.pair_gate = rt->pair_gate;
+  a.pair_row = rt->pair_row;
+  a.counts = rt->counts;
+  a.offsets = rt->offsets;
+  a.row_tok = rt->row_tok;
+  a.row_gate = rt->row_gate;
+  a.tile_expert = rt->tile_expert;
+  a.hist = w.hist;
+  a.local_rank = w.local_rank;
+  a.nchunks = p.nchunks;
+  a.st = DevStatus{nullptr, g_spin_limit};
+  return a;
+}
+
+GemmParams base_params(const Plan& p, const moe_routing* rt, int* status) {
+  GemmParams g;
+  std::memset(&g, 0, sizeof(g));
+  g.st = DevStatus{status, g_spin_limit};
+  g.offsets = rt ? rt->offsets : nullptr;
+  g.counts = rt ? rt->counts : nullptr;
+  g.tile_expert = rt ? rt->tile_expert : nullptr;
+  g.row_tok = rt ? rt->row_tok : nullptr;
+  g.row_gate = rt ? rt->row_gate : nullptr;
+  g.T = (int)p.T;
+  g.d = p.d;
+  g.n = p.n;
+  g.E = p.E;
+  g.Epad = p.Epad;
+  return g;
+}
+
+inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, sms)); }
+
+#define MOE_TRY_CUDA(x)                         \
+  do {                                          \
+    if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+#define MOE_TRY_MAP(x)                                 \
+  do {                                                 \
+    if (!(x)) return MOE_ERR_INVALID_ARG;              \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  RouteWs rw;
+  FwdWs fw;
+  BwdWs bw;
+  out->P_max = p.P_max;
+  out->R_max = p.R_max;
+  out->route_ws = carve_route(p, nullptr, &rw);
+  out->fwd_ws = carve_fwd(p, nullptr, &fw);
+  out->bwd_ws = carve_bwd(p, nullptr, &bw);
+  out->h_elems = p.R_max * 2 * p.n;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr, const float* bias,
+                     const moe_routing* rt, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!X || !Wr || !aligned16(X) || !aligned16(Wr) || (bias && !aligned16(bias)) || !routing_ok(rt, p, true))
+    return MOE_ERR_INVALID_ARG;
+  RouteWs w;
+  if (!ws || ws_bytes < carve_route(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_route(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  RouteArgs a = route_args(p, rt, w);
+  a.Wr = Wr;
+  a.st.word = status;
+  MOE_TRY_CUDA(launch_split_wr(a, st));
+
+  GemmParams g = base_params(p, rt, status);
+  MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
+  MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
+  g.num_m_tiles = (int)cdiv(p.T, 128);
+  g.num_n_tiles = p.Epad / 64;
+  g.outf = const_cast<float*>(a.logits);
+  g.bias = bias;
+  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+
+  MOE_TRY_CUDA(launch_softmax_topk(a, st));
+  MOE_TRY_CUDA(launch_permute(a, st));
+  return MOE_OK;
+}
+
+moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
+                           size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (opts->round_mode == 0) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, p, true)) return MOE_ERR_INVALID_ARG;
+  RouteWs w;
+  if (!ws || ws_bytes < carve_route(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_route(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  RouteArgs a = route_args(p, rt, w);
+  a.st.word = status;
+  RoundArgs r;
+  r.T = (int)p.T;
+  r.E = p.E;
+  r.mode = opts->round_mode;
+  r.seed = (unsigned long long)opts->seed;
+  r.probs = rt->probs;
+  r.member = w.member;
+  r.final_ = w.final_;
+  r.cnt = w.cnt;
+  r.Ew = p.Ew;
+  MOE_TRY_CUDA(launch_token_round(a, r, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1, const void* W2,
+                       const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  const void* ptrs[] = {X, W1, W2, O, H};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  FwdWs w;
+  if (!ws || ws_bytes < carve_fwd(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_fwd(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t mtiles = p.R_max / kTile;
+
+  // up-projection: H = X[tok] W1[e], A = SwiGLU(H)
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 64));
+    g.gsrc = static_cast<const __nv_bfloat16*>(X);
+    g.gld = p.d;
+    g.num_n_tiles = p.n / (p.bn_up / 2);
+    g.out0 = static_cast<__nv_bfloat16*>(H);
+    g.out1 = w.A;
+    MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  // down-projection: Y = A W2[e]
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmA, w.A, (uint64_t)p.R_max, (uint64_t)p.n, 64, 128));
+    MOE_TRY_MAP(make_tmap(&g.tmB, W2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 64));
+    g.num_n_tiles = p.d / p.bn_down;
+    g.out0 = w.Y;
+    MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  MOE_TRY_CUDA(launch_aggregate_fwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_gate, w.Y,
+                                    static_cast<__nv_bfloat16*>(O), st));
+  return MOE_OK;
+}
+
+moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X, const float* Wr,
+                        const void* W1, const void* W2, const moe_routing* rt, const void* H, void* dX, void* dW1,
+                        void* dW2, float* dWr, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  const void* ptrs[] = {dO, X, W1, W2, H, dX, dW1, dW2};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  const bool rg = opts->router_grad != 0;
+  if (rg && (!Wr || !dWr || !aligned16(Wr) || !aligned16(dWr))) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  BwdWs w;
+  if (!ws || ws_bytes < carve_bwd(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_bwd(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t mtiles = p.R_max / kTile;
+  const __nv_bfloat16* dOb = static_cast<const __nv_bfloat16*>(dO);
+  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+
+  // dH kernel: dA' = dO[tok] W2[e]^T; epilogue: H -> A, dS partials, dSwiGLU, A_hat
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmB, W2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, (uint32_t)p.bn_dh));
+    g.gsrc = dOb;
+    g.gld = p.d;
+    g.num_n_tiles = p.nts;
+    g.hin = static_cast<const __nv_bfloat16*>(H);
+    g.out0 = w.dH;
+    g.out1 = w.Ahat;
+    g.outf = w.dS_part;
+    MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  // dW2[e] = A_hat^T dO[tok]
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmA, w.Ahat, (uint64_t)p.R_max, (uint64_t)p.n, 64, 64));
+    g.gsrc = dOb;
+    g.gld = p.d;
+    g.num_m_tiles = (int)cdiv(p.n, 128);
+    g.num_n_tiles = p.d / p.bn_dw2;
+    g.out0 = static_cast<__nv_bfloat16*>(dW2);
+    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, g,
+                             grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+  }
+  // dX~ = dH W1[e]^T
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmA, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n, 64, 128));
+    MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
+    g.num_n_tiles = p.d / p.bn_dxt;
+    g.out0 = w.dXt;
+    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  // dW1[e] = X[tok]^T dH
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmB, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n, 64, 64));
+    g.gsrc = Xb;
+    g.gld = p.d;
+    g.num_m_tiles = (int)cdiv(p.d, 128);
+    g.num_n_tiles = 2 * p.n / p.bn_dw1;
+    g.out0 = static_cast<__nv_bfloat16*>(dW1);
+    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, g,
+                             grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+  }
+  if (rg) {
+    MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nts, rt->tok_ptr, rt->pair_row, rt->pair_expert,
+                                   rt->pair_gate, w.dS_part, w.dz_pair, w.dz_split, st));
+    MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 64));
+    MOE_TRY_MAP(make_tmap(&g.tmB, w.dz_split, (uint64_t)p.T, (uint64_t)2 * p.Epad, 64, 64));
+    g.num_m_tiles = (int)cdiv(p.d, 128);
+    g.num_n_tiles = p.Epad / 64;
+    g.ksplit = p.ksplit;
+    g.ksplit_rows = p.ksplit_rows;
+    g.outf = w.dWr_part;
+    MOE_TRY_CUDA(launch_gemm(G_DWR, 128, g,
+                             grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st));
+    MOE_TRY_CUDA(launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st));
+  }
+  MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_expert, w.dXt, w.dz_pair,
+                                    w.WrT, rg ? 1 : 0, static_cast<__nv_bfloat16*>(dX), st));
+  return MOE_OK;
+}
+
+moe_status moe_get_status(void* stream, int32_t* where) {
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero[2] = {0, 0};
+  if (cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+  if (where) *where = h[1];
+  return static_cast<moe_status>(h[0]);
+}
+
+moe_status moe_set_spin_limit(int64_t cycles) {
+  if (cycles < 1000) return MOE_ERR_INVALID_ARG;
+  g_spin_limit = cycles;
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream) {
+  if (!waited_ok) return MOE_ERR_INVALID_ARG;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  if (launch_wait_selftest(waited_ok, DevStatus{status, g_spin_limit}, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_CHECK: return "device consistency check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

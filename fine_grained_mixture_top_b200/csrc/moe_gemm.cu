@@ -1,0 +1,60 @@
+// Instantiations and launcher of the tcgen05 grouped GEMM (see gemm.cuh).
+#include <cuda_runtime.h>
+
+#include "gemm.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+template <int KIND, int BN>
+static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream) {
+  using KT = KindTraits<KIND>;
+  constexpr int smem = GemmShape<BN>::kSmemBytes;
+  constexpr int threads = KT::kGather ? 320 : 192;
+  auto fn = moe_gemm_kernel<KIND, BN>;
+  static int configured_dev = -1;  // per-process; the library serves one device at a time
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured_dev = dev;
+  }
+  if (grid <= 0) return cudaSuccess;
+  fn<<<grid, threads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(int kind, int bn, const GemmParams& p, int grid, cudaStream_t s) {
+#define MOE_CASE(K, B) \
+  if (kind == K && bn == B) return launch_one<K, B>(p, grid, s);
+  MOE_CASE(G_UP, 128)
+  MOE_CASE(G_UP, 256)
+  MOE_CASE(G_DOWN, 128)
+  MOE_CASE(G_DOWN, 256)
+  MOE_CASE(G_DH, 64)
+  MOE_CASE(G_DH, 128)
+  MOE_CASE(G_DH, 256)
+  MOE_CASE(G_DXT, 128)
+  MOE_CASE(G_DXT, 256)
+  MOE_CASE(G_DW1, 128)
+  MOE_CASE(G_DW1, 256)
+  MOE_CASE(G_DW2, 128)
+  MOE_CASE(G_DW2, 256)
+  MOE_CASE(G_RTR, 192)
+  MOE_CASE(G_DWR, 128)
+#undef MOE_CASE
+  return cudaErrorInvalidValue;
+}
+
+int gemm_smem_bytes(int bn) {
+  switch (bn) {
+    case 64: return GemmShape<64>::kSmemBytes;
+    case 128: return GemmShape<128>::kSmemBytes;
+    case 192: return GemmShape<192>::kSmemBytes;
+    case 256: return GemmShape<256>::kSmemBytes;
+  }
+  return 0;
+}
+
+}  // namespace moe

@@ -1,0 +1,68 @@
+// Internal launch interface between the C-ABI layer (moe_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int kTile = 128;        // rows per expert tile (segments are padded to it)
+constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation
+
+cudaError_t launch_gemm(int kind, int bn, const GemmParams& p, int grid, cudaStream_t s);
+int gemm_smem_bytes(int bn);
+
+// ---- routing (moe_route.cu)
+struct RouteArgs {
+  int T, d, E, K, Epad;
+  const float* Wr;
+  __nv_bfloat16* Wr_split;  // [d, 3*Epad]
+  const float* logits;      // [T, E]
+  float* probs;             // [T, E]
+  int* topk_idx;            // [T, K]
+  float* topk_gate;         // [T, K]
+  int* tok_ptr;             // [T+1]
+  int* pair_expert;         // [P_max]
+  float* pair_gate;         // [P_max]
+  int* pair_row;            // [P_max]
+  int* counts;              // [E]
+  int* offsets;             // [E+1]
+  int* row_tok;             // [R_max]
+  float* row_gate;          // [R_max]
+  int* tile_expert;         // [R_max/128]
+  int* hist;                // [nchunks, E]
+  int* local_rank;          // [P_max]
+  int nchunks;
+  DevStatus st;
+};
+cudaError_t launch_split_wr(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_softmax_topk(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s);  // rank + scan + scatter
+
+struct RoundArgs {
+  int T, E, mode;
+  unsigned long long seed;
+  const float* probs;
+  uint32_t* member;   // [T, Ew]
+  uint32_t* final_;   // [T, Ew]
+  int* cnt;           // [T]
+  int Ew;
+};
+cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStream_t s);
+
+// ---- aggregation and router backward (moe_agg.cu)
+cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pair_row, const float* pair_gate,
+                                 const __nv_bfloat16* Y, __nv_bfloat16* O, cudaStream_t s);
+cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
+                              const int* pair_expert, const float* pair_gate, const float* dS_part,
+                              float* dz_pair, __nv_bfloat16* dz_split, cudaStream_t s);
+cudaError_t launch_transpose_wr(int d, int E, const float* Wr, float* WrT, cudaStream_t s);
+cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s);
+cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const int* pair_expert,
+                                 const __nv_bfloat16* dXt, const float* dz_pair, const float* WrT, int router_grad,
+                                 __nv_bfloat16* dX, cudaStream_t s);
+cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
+
+}  // namespace moe

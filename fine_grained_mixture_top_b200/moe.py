@@ -1,0 +1,226 @@
+"""Python binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; torch supplies the
+device memory and the stream.  There is no fallback: if the shared library is
+missing the import of this module's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+c_void_p = ctypes.c_void_p
+c_int32 = ctypes.c_int32
+c_int64 = ctypes.c_int64
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
+    MOE_ERR_DEVICE_CHECK = range(7)
+
+
+class MoeDims(ctypes.Structure):
+    _fields_ = [("T", c_int64), ("d", c_int32), ("E", c_int32), ("n", c_int32), ("K", c_int32)]
+
+
+class MoeOpts(ctypes.Structure):
+    _fields_ = [("round_mode", c_int32), ("router_grad", c_int32), ("seed", ctypes.c_uint64)]
+
+
+_ROUTING_PTRS = ["logits", "probs", "topk_idx", "topk_gate", "tok_ptr", "pair_expert", "pair_gate", "pair_row",
+                 "counts", "offsets", "row_tok", "row_gate", "tile_expert"]
+
+
+class MoeRouting(ctypes.Structure):
+    _fields_ = [(name, c_void_p) for name in _ROUTING_PTRS] + [("P_max", c_int64), ("R_max", c_int64)]
+
+
+class MoeSizes(ctypes.Structure):
+    _fields_ = [("P_max", c_int64), ("R_max", c_int64), ("route_ws", ctypes.c_size_t),
+                ("fwd_ws", ctypes.c_size_t), ("bwd_ws", ctypes.c_size_t), ("h_elems", c_int64)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_str(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by fine_grained_mixture_top_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so is not built ({LIB_PATH}); run python -m "
+                               "fine_grained_mixture_top_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        L.moe_query_sizes.argtypes = [P(MoeDims), P(MoeOpts), P(MoeSizes)]
+        L.moe_route.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
+                                ctypes.c_size_t, c_void_p]
+        L.moe_token_round.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, ctypes.c_size_t, c_void_p]
+        L.moe_forward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
+                                  c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
+        L.moe_backward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   ctypes.c_size_t, c_void_p]
+        L.moe_get_status.argtypes = [c_void_p, P(c_int32)]
+        L.moe_set_spin_limit.argtypes = [c_int64]
+        L.moe_selftest_wait_timeout.argtypes = [c_void_p, c_void_p]
+        L.moe_status_str.argtypes = [c_int32]
+        L.moe_status_str.restype = ctypes.c_char_p
+        for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
+                  "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout"):
+            getattr(L, f).restype = c_int32
+        _lib = L
+    return _lib
+
+
+def status_str(code: int) -> str:
+    return lib().moe_status_str(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != MOE_OK:
+        raise MoEError(code, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def dims_of(T, d, E, n, K) -> MoeDims:
+    return MoeDims(int(T), int(d), int(E), int(n), int(K))
+
+
+def opts_of(round_mode=0, router_grad=1, seed=0) -> MoeOpts:
+    return MoeOpts(int(round_mode), int(router_grad), int(seed))
+
+
+def query_sizes(dims: MoeDims, opts: MoeOpts) -> MoeSizes:
+    s = MoeSizes()
+    _check(lib().moe_query_sizes(ctypes.byref(dims), ctypes.byref(opts), ctypes.byref(s)), "moe_query_sizes")
+    return s
+
+
+@dataclass
+class Routing:
+    """Device buffers of a moe_routing, allocated with torch."""
+    tensors: dict
+    struct: MoeRouting
+
+    def __getitem__(self, k):
+        return self.tensors[k]
+
+    @classmethod
+    def allocate(cls, dims: MoeDims, sizes: MoeSizes, device="cuda", with_logits: bool = True) -> "Routing":
+        import torch
+        T, E, K = dims.T, dims.E, dims.K
+        P, R = sizes.P_max, sizes.R_max
+        i32, f32 = torch.int32, torch.float32
+        shapes = {"logits": ((T, E), f32), "probs": ((T, E), f32), "topk_idx": ((T, K), i32),
+                  "topk_gate": ((T, K), f32), "tok_ptr": ((T + 1,), i32), "pair_expert": ((P,), i32),
+                  "pair_gate": ((P,), f32), "pair_row": ((P,), i32), "counts": ((E,), i32),
+                  "offsets": ((E + 1,), i32), "row_tok": ((R,), i32), "row_gate": ((R,), f32),
+                  "tile_expert": ((R // 128,), i32)}
+        t = {}
+        for k, (shape, dt) in shapes.items():
+            if k == "logits" and not with_logits:
+                t[k] = None
+                continue
+            t[k] = torch.empty(shape, dtype=dt, device=device)
+        st = MoeRouting(*[_ptr(t[k]) for k in _ROUTING_PTRS], P, R)
+        return cls(t, st)
+
+
+def moe_route(dims, opts, X, Wr, bias, routing: Routing, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(Wr), _ptr(bias),
+                           ctypes.byref(routing.struct), _ptr(ws), ws.numel() * ws.element_size(),
+                           _stream(stream)), "moe_route")
+
+
+def moe_token_round(dims, opts, routing: Routing, ws, stream=None):
+    _check(lib().moe_token_round(ctypes.byref(dims), ctypes.byref(opts), ctypes.byref(routing.struct), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "moe_token_round")
+
+
+def moe_forward(dims, opts, X, W1, W2, routing: Routing, O, H, ws, stream=None):
+    _check(lib().moe_forward(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(W1), _ptr(W2),
+                             ctypes.byref(routing.struct), _ptr(O), _ptr(H), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW2, dWr, ws, stream=None):
+    _check(lib().moe_backward(ctypes.byref(dims), ctypes.byref(opts), _ptr(dO), _ptr(X), _ptr(Wr), _ptr(W1),
+                              _ptr(W2), ctypes.byref(routing.struct), _ptr(H), _ptr(dX), _ptr(dW1), _ptr(dW2),
+                              _ptr(dWr), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_backward")
+
+
+def moe_get_status(stream=None) -> tuple[int, int]:
+    where = c_int32(0)
+    code = lib().moe_get_status(_stream(stream), ctypes.byref(where))
+    return int(code), int(where.value)
+
+
+def moe_set_spin_limit(cycles: int):
+    _check(lib().moe_set_spin_limit(int(cycles)), "moe_set_spin_limit")
+
+
+def moe_selftest_wait_timeout(flag, stream=None):
+    _check(lib().moe_selftest_wait_timeout(_ptr(flag), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+class MoELayer:
+    """All device buffers of one layer shape, allocated once with torch; each
+    method is one library call."""
+
+    def __init__(self, T, d, E, n, K, round_mode=0, router_grad=1, seed=0, device="cuda"):
+        import torch
+        self.dims = dims_of(T, d, E, n, K)
+        self.opts = opts_of(round_mode, router_grad, seed)
+        self.sizes = query_sizes(self.dims, self.opts)
+        self.device = device
+        self.routing = Routing.allocate(self.dims, self.sizes, device)
+        u8, bf = torch.uint8, torch.bfloat16
+        self.ws_route = torch.empty(self.sizes.route_ws, dtype=u8, device=device)
+        self.ws_fwd = torch.empty(self.sizes.fwd_ws, dtype=u8, device=device)
+        self.ws_bwd = torch.empty(self.sizes.bwd_ws, dtype=u8, device=device)
+        self.H = torch.empty(self.sizes.R_max, 2 * n, dtype=bf, device=device)
+        self.O = torch.empty(T, d, dtype=bf, device=device)
+        self.dX = torch.empty(T, d, dtype=bf, device=device)
+        self.dW1 = torch.empty(E, d, 2 * n, dtype=bf, device=device)
+        self.dW2 = torch.empty(E, n, d, dtype=bf, device=device)
+        self.dWr = torch.empty(d, E, dtype=torch.float32, device=device)
+
+    def route(self, X, Wr, bias=None, stream=None):
+        moe_route(self.dims, self.opts, X, Wr, bias, self.routing, self.ws_route, stream)
+        if self.opts.round_mode:
+            moe_token_round(self.dims, self.opts, self.routing, self.ws_route, stream)
+
+    def forward(self, X, W1, W2, stream=None):
+        moe_forward(self.dims, self.opts, X, W1, W2, self.routing, self.O, self.H, self.ws_fwd, stream)
+        return self.O
+
+    def backward(self, dO, X, Wr, W1, W2, stream=None):
+        moe_backward(self.dims, self.opts, dO, X, Wr, W1, W2, self.routing, self.H, self.dX, self.dW1, self.dW2,
+                     self.dWr if self.opts.router_grad else None, self.ws_bwd, stream)
+        return self.dX, self.dW1, self.dW2, self.dWr
+
+    def step(self, X, Wr, bias, W1, W2, dO, stream=None):
+        """One pass of the whole path: route (+ rounding), forward, backward."""
+        self.route(X, Wr, bias, stream)
+        self.forward(X, W1, W2, stream)
+        return self.backward(dO, X, Wr, W1, W2, stream)

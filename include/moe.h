@@ -1,0 +1,194 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) fine-grained MoE expert layer:
+ * top-K routing, permutation into per-expert segments, grouped-GEMM
+ * up-projection with gather and SwiGLU fused, grouped-GEMM down-projection,
+ * gate-weighted aggregation, and the full backward pass with the router-score
+ * gradient computed without caching any per-expert output.
+ *
+ * Sources (scraped pages on SonicMoE):
+ *   [P1] "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE" (news article on the
+ *        SonicMoE Blackwell blog), sections "MoE 与它的隐患",
+ *        "核心创新：一次算法级的重新设计", "软件抽象层 QuACK".
+ *   [P2] "SonicMoE：突破细粒度MoE硬件效率瓶颈，实现高稀疏性下的极致训练加速",
+ *        paragraphs on the algorithm (router gradient without cached
+ *        activations), scheduling (token rounding) and implementation (the
+ *        eight kernels).
+ *
+ * Conventions for every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *     allocates and frees nothing.  Scratch memory is the caller's `ws` buffer,
+ *     sized by moe_query_sizes().  All pointers must be 16-byte aligned.
+ *   - bf16 tensors are passed as `void*` holding IEEE bfloat16 bit patterns.
+ *   - Row-major layouts: X[T,d], Wr[d,E] (fp32), W1[E,d,2n] with columns
+ *     [0,n) the gate projection and [n,2n) the up projection, W2[E,n,d].
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; argument errors are returned synchronously,
+ *     device-side errors (a bounded wait that ran out, a failed check) are
+ *     recorded in a device status word read by moe_get_status().
+ *   - Supported shapes: d % 128 == 0, n % 64 == 0, 1 <= K <= min(E, 32),
+ *     1 <= E <= 1024, 1 <= T < 2^31 / max(K, E).  Anything else returns
+ *     MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* NULL where a pointer is required, misaligned pointer, bad option */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape outside the supported range */
+  MOE_ERR_WORKSPACE = 3,     /* ws NULL or smaller than moe_query_sizes() asks */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch error, no device) */
+  MOE_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out */
+  MOE_ERR_DEVICE_CHECK = 6   /* device: an internal consistency check failed */
+} moe_status;
+
+/* Layer shape: T tokens, model width d, E experts of intermediate width n, top-K. */
+typedef struct {
+  int64_t T;
+  int32_t d, E, n, K;
+} moe_dims;
+
+typedef struct {
+  int32_t round_mode;  /* token rounding used by moe_token_round: 1 nearest, 2 stochastic (0: off) */
+  int32_t router_grad; /* 1: moe_backward adds the router path to dX and writes dWr */
+  uint64_t seed;       /* seed of the stochastic rounding decision */
+} moe_opts;
+
+/*
+ * Routing state, produced by moe_route (and rewritten by moe_token_round),
+ * read by moe_forward / moe_backward.  All device pointers, caller-allocated
+ * with the capacities P_max (pairs) and R_max (rows) from moe_query_sizes.
+ *
+ *   logits[T,E] f32, probs[T,E] f32   router logits z = X Wr (+ bias) and
+ *                                      p = softmax(z) over all E experts
+ *   topk_idx[T,K] i32, topk_gate[T,K]  the K largest logits per token (ties to
+ *                                      the lower expert index, slots in
+ *                                      descending order) and their gates, a
+ *                                      softmax over the selected logits
+ *   tok_ptr[T+1], pair_expert[P_max], pair_gate[P_max], pair_row[P_max]
+ *                                      (token, expert) pairs as CSR over tokens
+ *                                      and the expert-major row of each pair
+ *   counts[E], offsets[E+1]            tokens per expert; segment starts, each
+ *                                      a multiple of 128 (segments are padded
+ *                                      to whole 128-row tiles); offsets[E] is
+ *                                      the number of rows in use
+ *   row_tok[R_max], row_gate[R_max]    token and gate of every row; padding
+ *                                      rows hold token -1 and gate 0; inside a
+ *                                      segment rows ascend in token order
+ *   tile_expert[R_max/128]             expert of each 128-row tile
+ */
+typedef struct {
+  float* logits;
+  float* probs;
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* tok_ptr;
+  int32_t* pair_expert;
+  float* pair_gate;
+  int32_t* pair_row;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* row_tok;
+  float* row_gate;
+  int32_t* tile_expert;
+  int64_t P_max;
+  int64_t R_max;
+} moe_routing;
+
+typedef struct {
+  int64_t P_max;        /* capacity of the pair arrays */
+  int64_t R_max;        /* capacity of the row arrays (a multiple of 128) */
+  size_t route_ws;      /* bytes of ws for moe_route and moe_token_round */
+  size_t fwd_ws;        /* bytes of ws for moe_forward */
+  size_t bwd_ws;        /* bytes of ws for moe_backward */
+  int64_t h_elems;      /* elements of the saved activation H = R_max * 2n (bf16) */
+} moe_sizes;
+
+/* Capacities and workspace sizes for a shape.  Host only; no GPU work. */
+moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes* out);
+
+/*
+ * Router and permutation ([P1] "MoE 与它的隐患": each token is sent to a few
+ * experts chosen by the router; [P1] "第二，IO 感知的算子融合": the grouped
+ * GEMMs gather the routed rows themselves, so routing only produces indices).
+ *   X[T,d] bf16, Wr[d,E] f32, bias[E] f32 (nullable; added to the logits
+ *   before the softmax).  Fills every array of *rt except pair_row's unused
+ *   tail.  rt->logits may be NULL (then kept in ws only).
+ */
+moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
+                     const float* bias, const moe_routing* rt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Token rounding ([P2] scheduling paragraph): rounds every expert's token
+ * count to a multiple of the 128-row GEMM tile with at most one tile of
+ * deviation, keeping the total in expectation (opts->round_mode 2) or rounding
+ * to the nearest multiple (mode 1).  Rounding down drops the routed tokens of
+ * least probability, rounding up adds the unrouted tokens of largest
+ * probability; gates become p renormalised over each token's final experts,
+ * listed in ascending expert order.  Rewrites tok_ptr, pair_*, counts,
+ * offsets, row_*, tile_expert of *rt (topk_idx/topk_gate keep the unrounded
+ * selection).  Must follow moe_route on the same stream.
+ */
+moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * Forward ([P2] implementation paragraph: up-proj (A), down-proj (Y) and
+ * expert aggregation (O) kernels):
+ *   H_r = X[tok_r] W1[e_r]  (gather fused into the GEMM), A_r = silu(g)*u
+ *   fused in its epilogue; Y_r = A_r W2[e_r];  O_t = sum_k gate * Y_row.
+ *   O[T,d] bf16 out.  H[R_max,2n] bf16 out: the only per-row activation kept
+ *   for the backward.  A and Y live in ws only.
+ */
+moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1, const void* W2,
+                       const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward given dO[T,d] bf16 ([P2] implementation and algorithm paragraphs;
+ * [P1] "第一，激活内存与专家粒度解耦"): dH kernel dA'_r = dO[tok_r] W2[e]^T
+ * with H reloaded in its epilogue, the router score gradient
+ * dS_r = <dA'_r, SwiGLU(H_r)> (no Y needed), dSwiGLU; dW2[e] = sum s_r A_r^T
+ * dO[tok_r]; dX~_r = dH_r W1[e]^T; dW1[e] = sum X[tok_r]^T dH_r; dX
+ * aggregation.  Router path (opts->router_grad): dz = s (dS - sum s dS) over
+ * each token's experts, dWr = X^T dz (fp32 out, may be NULL only when
+ * router_grad is 0), dX += dz Wr^T.
+ *   dX[T,d], dW1[E,d,2n], dW2[E,n,d] bf16 out (overwritten, not accumulated).
+ */
+moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X,
+                        const float* Wr, const void* W1, const void* W2, const moe_routing* rt, const void* H,
+                        void* dX, void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, returns the device status word (MOE_OK if no kernel
+ * reported an error since the last call) and clears it.  *where (nullable)
+ * receives the code of the wait or check that failed.
+ */
+moe_status moe_get_status(void* stream, int32_t* where);
+
+/* Number of clock cycles a bounded wait spins before giving up (default 2^31,
+ * about a second).  Values < 1000 are rejected with MOE_ERR_INVALID_ARG. */
+moe_status moe_set_spin_limit(int64_t cycles);
+
+/*
+ * Failure-detection self test: launches one thread that waits, through the
+ * kernels' bounded-wait primitive, on a barrier nothing completes.  On return
+ * (after a stream sync) *waited_ok (device int) is 0 and moe_get_status()
+ * reports MOE_ERR_TIMEOUT.  Meant for tests with a small spin limit.
+ */
+moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream);
+
+/* Static description of a status code. */
+const char* moe_status_str(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,106 @@
+"""Helpers of the GPU parity tests: run the layer through the C ABI and compare
+with the fp64 oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import moe_oracle as orc
+
+# Tolerances: the benchmark spec's bounds.  bf16-path outputs and gradients: max
+# |gpu - ref| / max |ref| per tensor; fp32 router probabilities: absolute.
+TOL_BF16 = 2e-2
+TOL_PROBS = 1e-5
+NEAR_TIE = 1e-4
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def i64(t):
+    return t.detach().to("cpu").long().numpy()
+
+
+def normwise(gpu, ref):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.abs(ref).max()
+    if scale == 0:
+        return float(np.abs(gpu).max())
+    return float(np.abs(gpu - ref).max() / scale)
+
+
+def run_layer(inp, T, d, E, n, K, round_mode=0, router_grad=1, seed=0):
+    import torch
+    from fine_grained_mixture_top_b200 import moe
+    layer = moe.MoELayer(T, d, E, n, K, round_mode=round_mode, router_grad=router_grad, seed=seed)
+    layer.route(inp["X"], inp["Wr"], inp["bias"])
+    layer.forward(inp["X"], inp["W1"], inp["W2"])
+    layer.backward(inp["dO"], inp["X"], inp["Wr"], inp["W1"], inp["W2"])
+    torch.cuda.synchronize()
+    code, where = moe.moe_get_status()
+    assert code == 0, (code, where)
+    return layer
+
+
+def gpu_routing(layer, T):
+    r = layer.routing.tensors
+    tok_ptr = i64(r["tok_ptr"])
+    P = int(tok_ptr[T])
+    return {
+        "logits": f64(r["logits"]), "probs": f64(r["probs"]), "topk_idx": i64(r["topk_idx"]),
+        "topk_gate": f64(r["topk_gate"]), "tok_ptr": tok_ptr, "pair_expert": i64(r["pair_expert"])[:P],
+        "pair_gate": f64(r["pair_gate"])[:P], "pair_row": i64(r["pair_row"])[:P], "counts": i64(r["counts"]),
+        "offsets": i64(r["offsets"]), "row_tok": i64(r["row_tok"]), "row_gate": f64(r["row_gate"]),
+        "tile_expert": i64(r["tile_expert"]),
+    }
+
+
+def check_permutation(g, E):
+    """Bit-exact check of the GPU's expert-major rows against the oracle's
+    permutation of the GPU's own pairs."""
+    perm = orc.permute(g["tok_ptr"], g["pair_expert"], E)
+    np.testing.assert_array_equal(g["counts"], perm["counts"])
+    off = g["offsets"]
+    assert off[0] == 0
+    for e in range(E):
+        c = perm["counts"][e]
+        assert off[e + 1] - off[e] == -(-c // 128) * 128
+        seg = g["row_tok"][off[e]:off[e] + c]
+        np.testing.assert_array_equal(seg, perm["row_tok"][perm["seg"][e]:perm["seg"][e + 1]])
+        assert np.all(g["row_tok"][off[e] + c:off[e + 1]] == -1)
+        assert np.all(g["row_gate"][off[e] + c:off[e + 1]] == 0.0)
+        assert np.all(g["tile_expert"][off[e] // 128:off[e + 1] // 128] == e)
+    # each pair's row: same position inside its segment as in the oracle
+    pe = g["pair_expert"]
+    np.testing.assert_array_equal(g["pair_row"] - off[pe], perm["pair_row"] - perm["seg"][pe])
+    np.testing.assert_array_equal(g["row_gate"][g["pair_row"]], g["pair_gate"])
+    return perm
+
+
+def check_router(g, ref_z, ref_p, K):
+    """probs within 1e-5; top-K exactly the oracle's on the GPU's own fp32
+    logits; equal to the fp64 selection wherever the K-th/(K+1)-th gap is
+    above the near-tie threshold."""
+    assert np.abs(g["probs"] - ref_p).max() <= TOL_PROBS
+    own = orc.topk_select(g["logits"], K)
+    np.testing.assert_array_equal(own, g["topk_idx"])
+    ref_idx = orc.topk_select(ref_z, K)
+    E = ref_z.shape[1]
+    if K < E:
+        zs = np.sort(ref_z, axis=1)[:, ::-1]
+        margin = zs[:, K - 1] - zs[:, K]
+        clear = margin > NEAR_TIE
+    else:
+        clear = np.ones(ref_z.shape[0], bool)
+    np.testing.assert_array_equal(g["topk_idx"][clear], ref_idx[clear])
+    return int((~clear).sum())
+
+
+def expert_rows_to_oracle_order(gpu_rows, g, perm, E):
+    """Gather GPU per-row data (padded segments) into the oracle's packed order."""
+    out = np.zeros((len(perm["row_tok"]),) + gpu_rows.shape[1:], gpu_rows.dtype)
+    for e in range(E):
+        c = perm["counts"][e]
+        out[perm["seg"][e]:perm["seg"][e] + c] = gpu_rows[g["offsets"][e]:g["offsets"][e] + c]
+    return out

@@ -1,0 +1,90 @@
+"""The C-ABI library loads on a host without a GPU, exports every entry point
+include/moe.h declares, and its host-only logic (shape checks, workspace
+sizing, status strings) behaves as documented.  No compute call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from fine_grained_mixture_top_b200 import build
+    build.build()
+    from fine_grained_mixture_top_b200 import moe as m
+    return m
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:moe_status|const char\*)\s+(moe_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("moe_route", "moe_token_round", "moe_forward", "moe_backward", "moe_query_sizes",
+              "moe_get_status", "moe_status_str"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = moe.lib()
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)$", out, re.M))
+    assert set(declared_symbols()) <= exported
+
+
+def test_query_sizes_matches_documented_capacities(moe):
+    T, d, E, n, K = 16384, 1536, 128, 256, 8
+    s = moe.query_sizes(moe.dims_of(T, d, E, n, K), moe.opts_of(0, 1, 0))
+    assert s.P_max == T * K
+    assert s.R_max % 128 == 0 and s.R_max >= T * K + 127 * E
+    assert s.h_elems == s.R_max * 2 * n
+    # forward workspace holds A [R,n] and Y [R,d] in bf16
+    assert s.fwd_ws >= s.R_max * (n + d) * 2
+    # token rounding enlarges the pair capacity by at most one tile per expert
+    s2 = moe.query_sizes(moe.dims_of(T, d, E, n, K), moe.opts_of(2, 1, 7))
+    assert s2.P_max == min(T * E, T * K + 127 * E)
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((512, 100, 16, 64, 2), 2),    # d not a multiple of 128
+    ((512, 128, 16, 48, 2), 2),    # n not a multiple of 64
+    ((512, 128, 4, 64, 5), 2),     # K > E
+    ((512, 128, 2048, 64, 2), 2),  # E > 1024
+    ((512, 128, 64, 64, 33), 2),   # K > 32
+    ((0, 128, 16, 64, 2), 2),      # no tokens
+])
+def test_query_sizes_rejects_unsupported_shapes(moe, shape, code):
+    s = moe.MoeSizes()
+    rc = moe.lib().moe_query_sizes(ctypes.byref(moe.dims_of(*shape)), ctypes.byref(moe.opts_of()), ctypes.byref(s))
+    assert rc == code
+
+
+def test_invalid_options_and_null_arguments(moe):
+    L = moe.lib()
+    s = moe.MoeSizes()
+    dims = moe.dims_of(512, 128, 16, 64, 2)
+    assert L.moe_query_sizes(ctypes.byref(dims), ctypes.byref(moe.opts_of(3, 1, 0)), ctypes.byref(s)) == 1
+    assert L.moe_query_sizes(ctypes.byref(dims), ctypes.byref(moe.opts_of(0, 2, 0)), ctypes.byref(s)) == 1
+    assert L.moe_query_sizes(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None) == 1
+    # argument errors are caught on the host before any GPU call
+    rt = moe.MoeRouting()
+    assert L.moe_route(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, ctypes.byref(rt),
+                       None, 0, None) == 1
+    assert L.moe_forward(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, ctypes.byref(rt),
+                         None, None, None, 0, None) == 1
+    assert L.moe_set_spin_limit(10) == 1
+
+
+def test_status_strings(moe):
+    assert moe.status_str(0) == "ok"
+    assert "timed out" in moe.status_str(5)
+    assert moe.status_str(99) == "unknown status"

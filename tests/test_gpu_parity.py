@@ -1,0 +1,131 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs.  Routing, permutation and token rounding bit-exact (after
+the near-tie rule), floating-point outputs within the stated tolerances."""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as orc
+from workloads import CONFIGS, MoEConfig, make_inputs
+
+import parity as P
+
+torch = pytest.importorskip("torch")
+
+SHAPES = [
+    CONFIGS["tiny"],
+    # BN 256 paths (n % 128 == 0, d % 256 == 0), skewed router
+    MoEConfig("bn256", T=300, d=256, E=8, n=128, K=2, w_std=0.05, bias="normal", seed=11),
+    # BN 128 / 64 paths (d % 256 != 0, n % 128 != 0), several dH N tiles
+    MoEConfig("bn64", T=1000, d=384, E=12, n=192, K=3, w_std=0.05, seed=12),
+    # one expert, top-1: a dense SwiGLU MLP
+    MoEConfig("dense", T=200, d=128, E=1, n=64, K=1, w_std=0.05, seed=13),
+    # fewer tokens than a tile, E not a multiple of 64, empty experts
+    MoEConfig("sparse", T=64, d=128, E=70, n=64, K=4, w_std=0.05, seed=14),
+]
+
+
+def _np_inputs(inp):
+    return (P.f64(inp["X"]), P.f64(inp["Wr"]), None if inp["bias"] is None else P.f64(inp["bias"]),
+            P.f64(inp["W1"]), P.f64(inp["W2"]), P.f64(inp["dO"]))
+
+
+def _compare_layer(layer, cfg, inp, routing=None, router_grad=True):
+    g = P.gpu_routing(layer, cfg.T)
+    X, Wr, b, W1, W2, dO = _np_inputs(inp)
+    if routing is None:
+        fw = orc.forward(X, Wr, b, W1, W2, cfg.K, topk_idx=g["topk_idx"])
+    else:
+        fw = orc.forward(X, Wr, b, W1, W2, cfg.K, routing=routing)
+    np.testing.assert_allclose(g["pair_gate"], fw["pair_gate"], rtol=1e-5, atol=1e-7)
+    perm = P.check_permutation(g, cfg.E)
+    errs = {"O": P.normwise(P.f64(layer.O), fw["O"])}
+    H = P.expert_rows_to_oracle_order(P.f64(layer.H), g, perm, cfg.E)
+    errs["H"] = P.normwise(H, fw["H"])
+    bw = orc.backward(fw, dO, X, Wr, W1, W2, router_grad=router_grad)
+    errs["dX"] = P.normwise(P.f64(layer.dX), bw["dX"])
+    errs["dW1"] = P.normwise(P.f64(layer.dW1), bw["dW1"])
+    errs["dW2"] = P.normwise(P.f64(layer.dW2), bw["dW2"])
+    if router_grad:
+        errs["dWr"] = P.normwise(P.f64(layer.dWr), bw["dWr"])
+    print(cfg.name, {k: f"{v:.2e}" for k, v in errs.items()})
+    for k, v in errs.items():
+        assert v <= P.TOL_BF16, (k, v)
+    return g, fw, bw
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", SHAPES, ids=[c.name for c in SHAPES])
+def test_layer_parity(cfg):
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    g = P.gpu_routing(layer, cfg.T)
+    X, Wr, b, *_ = _np_inputs(inp)
+    z = orc.router_logits(X, Wr, b)
+    P.check_router(g, z, orc.softmax_rows(z), cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
+def test_expert_only_gradient_without_router_path():
+    cfg = SHAPES[1]
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, router_grad=0)
+    _compare_layer(layer, cfg, inp, router_grad=False)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", [1, 2])
+def test_token_rounding_parity(mode):
+    cfg = MoEConfig("tr", T=2048, d=128, E=16, n=64, K=2, w_std=0.05, bias="normal", seed=21)
+    seed = 1234
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=mode, seed=seed)
+    g = P.gpu_routing(layer, cfg.T)
+    tok_ptr0, pe0 = orc.pairs_from_topk(g["topk_idx"])
+    c0 = np.bincount(pe0, minlength=cfg.E)
+    tr = orc.token_round(g["probs"], tok_ptr0, pe0, mode, seed)   # decisions in the GPU's fp32 probs
+    np.testing.assert_array_equal(g["tok_ptr"], tr["tok_ptr"])
+    np.testing.assert_array_equal(g["pair_expert"], tr["pair_expert"])
+    np.testing.assert_allclose(g["pair_gate"], tr["pair_gate"], rtol=2e-6)
+    assert np.all(g["counts"] % 128 == 0)
+    assert np.all(np.abs(g["counts"] - c0) < 128)
+    assert np.any(g["counts"] != c0)
+    X, Wr, b, *_ = _np_inputs(inp)
+    z = orc.router_logits(X, Wr, b)
+    routing = {"z": z, "probs": orc.softmax_rows(z), "topk_idx": g["topk_idx"], "tok_ptr": tr["tok_ptr"],
+               "pair_expert": tr["pair_expert"],
+               "pair_gate": orc.gates_for_sets(z, tr["tok_ptr"], tr["pair_expert"])}
+    _compare_layer(layer, cfg, inp, routing=routing)
+
+
+@pytest.mark.gpu
+def test_bounded_wait_reports_timeout():
+    from fine_grained_mixture_top_b200 import moe
+    assert moe.moe_get_status() == (0, 0)
+    moe.moe_set_spin_limit(2_000_000)          # about a millisecond
+    flag = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    try:
+        moe.moe_selftest_wait_timeout(flag)
+        code, where = moe.moe_get_status()
+    finally:
+        moe.moe_set_spin_limit(1 << 31)
+    assert int(flag.item()) == 0
+    assert (code, where) == (moe.MOE_ERR_TIMEOUT, 999)
+    assert moe.moe_get_status() == (0, 0)      # cleared; the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum().item()) == 4.0
+
+
+@pytest.mark.gpu
+def test_argument_errors_are_synchronous():
+    from fine_grained_mixture_top_b200 import moe
+    layer = moe.MoELayer(512, 128, 16, 64, 2)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    X = torch.zeros(512, 128, dtype=torch.bfloat16, device="cuda")
+    Wr = torch.zeros(128, 16, device="cuda")
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_route(layer.dims, layer.opts, X, Wr, None, layer.routing, small)
+    assert ei.value.code == moe.MOE_ERR_WORKSPACE
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_route(layer.dims, layer.opts, X[:, 1:], Wr, None, layer.routing, layer.ws_route)
+    assert ei.value.code == moe.MOE_ERR_INVALID_ARG
