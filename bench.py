@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained MoE expert layer on B200.
+
+One step = the whole path on one batch: routing (router logits, softmax, top-K,
+permutation), forward (up-proj + SwiGLU, down-proj, aggregation) and backward
+(dH + dS, dW2, dX~, dW1, router backward, dX aggregation), all through the
+library's C ABI.  Workload: the fine-grained 7B-class layer, T=16384 tokens,
+d=1536, E=128, n=256, top-8, skewed router (bias ~ N(0, 0.5)); synthetic seeded
+inputs (workloads package).  Multi-GPU: one process per GPU (torchrun), each
+with its own batch (weak scaling); the weight gradients are all-reduced over
+NCCL as the data-parallel exchange step.
+
+Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle on
+a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd TFLOP/s (bf16) and % of B200 tensor peak; tokens/sec"
+WORKLOAD = ("fine-grained 7B-class MoE layer fwd+bwd: T=16384, d=1536, E=128, n=256, top-8, SwiGLU, "
+            "skewed router (bias ~N(0,0.5))")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="7b")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
+    ap.add_argument("--ref-sample-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work per kernel
+def kernel_work(cfg, R):
+    """Algorithmic FLOPs and HBM bytes of one launch of each kernel (R = routed
+    pairs T*K; bf16 = 2 bytes).  Bytes assume every operand is read once."""
+    T, d, E, n = cfg.T, cfg.d, cfg.E, cfg.n
+    w = {
+        "up_proj_gemm": (4 * R * d * n, 2 * T * d + 4 * E * d * n + 6 * R * n),
+        "down_proj_gemm": (2 * R * d * n, 2 * R * n + 2 * E * d * n + 2 * R * d),
+        "dh_gemm": (2 * R * d * n, 2 * T * d + 2 * E * d * n + 10 * R * n + 4 * R),
+        "dw2_gemm": (2 * R * d * n, 2 * R * n + 2 * T * d + 2 * E * d * n),
+        "dxt_gemm": (4 * R * d * n, 4 * R * n + 4 * E * d * n + 2 * R * d),
+        "dw1_gemm": (4 * R * d * n, 2 * T * d + 4 * R * n + 4 * E * d * n),
+        "aggregate_fwd": (2 * R * d, 2 * R * d + 2 * T * d + 8 * R),
+        "aggregate_bwd": (R * d, 2 * R * d + 2 * T * d + 12 * R),
+        "router_logits_gemm": (2 * T * d * E, 2 * T * d + 4 * d * E + 4 * T * E),
+        "router_dwr_gemm": (2 * T * d * E, 2 * T * d + 4 * T * E + 4 * d * E),
+    }
+    return w
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fine_grained_mixture_top_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload_key):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    if there is none for this kernel and workload or the sources changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        data = json.load(f)
+    rec = data.get(kernel)
+    if not rec or rec.get("src_digest") != source_digest() or rec.get("workload") != workload_key:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+def oracle_step_seconds(cfg, inp_cpu, tokens):
+    """Time the fp64 oracle (as it stands) on the first `tokens` tokens of the
+    batch: route, forward, backward.  Returns (seconds, threads)."""
+    import numpy as np
+    from oracle import moe_oracle as orc
+    X = inp_cpu["X"][:tokens].double().numpy()
+    dO = inp_cpu["dO"][:tokens].double().numpy()
+    W1 = inp_cpu["W1np"]
+    W2 = inp_cpu["W2np"]
+    Wr = inp_cpu["Wr"].double().numpy()
+    b = None if inp_cpu["bias"] is None else inp_cpu["bias"].double().numpy()
+    t0 = time.perf_counter()
+    fw = orc.forward(X, Wr, b, W1, W2, cfg.K)
+    orc.backward(fw, dO, X, Wr, W1, W2)
+    dt = time.perf_counter() - t0
+    return dt, blas_threads()
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_inputs(cfg):
+    from workloads import make_inputs
+    inp = make_inputs(cfg, "cpu")
+    inp["W1np"] = inp["W1"].double().numpy()
+    inp["W2np"] = inp["W2"].double().numpy()
+    return inp
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from workloads import CONFIGS
+    cfg = CONFIGS[args.config]
+    inp = cpu_inputs(cfg)
+    tokens = min(args.ref_sample_tokens, cfg.T)
+    for _ in range(args.warmup):
+        oracle_step_seconds(cfg, inp, tokens)
+    times = []
+    threads = 1
+    for _ in range(args.steps):
+        dt, threads = oracle_step_seconds(cfg, inp, tokens)
+        times.append(dt)
+    tot = sum(times)
+    flops = 18 * tokens * cfg.K * cfg.d * cfg.n
+    value = flops * args.steps / tot / 1e12
+    sample = f"first {tokens} of {cfg.T} tokens per step (full weights), fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
+                   "parallelism": "single host process"},
+        "tokens_per_s": tokens * args.steps / tot,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from fine_grained_mixture_top_b200 import moe
+    from workloads import CONFIGS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    cfg = CONFIGS[args.config]
+    inp = make_inputs(cfg, dev, rank=rank)
+    layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=cfg.round_mode, router_grad=1,
+                         seed=cfg.seed, device=dev)
+    X, Wr, b, W1, W2, dO = (inp[k] for k in ("X", "Wr", "bias", "W1", "W2", "dO"))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.step(X, Wr, b, W1, W2, dO)
+        if world > 1:
+            for g in (layer.dW1, layer.dW2, layer.dWr):
+                dist.all_reduce(g)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    code, where = moe.moe_get_status()
+    if code != 0:
+        raise RuntimeError(f"device status {moe.status_str(code)} at {where}")
+    R = int(layer.routing["tok_ptr"][cfg.T].item())
+    counts = layer.routing["counts"].cpu().tolist()
+
+    # ---- device-timed region
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    smi_index = vis[local_rank].strip() if local_rank < len(vis) and vis[local_rank].strip().isdigit() else local_rank
+    sampler = ClockSampler(smi_index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    moe.moe_profile_enable(True)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    moe.moe_profile_enable(False)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    recs = moe.moe_profile_records()
+    code, where = moe.moe_get_status()
+    if code != 0:
+        raise RuntimeError(f"device status {moe.status_str(code)} at {where}")
+
+    flops_step = 18 * cfg.T * cfg.K * cfg.d * cfg.n
+    ms_step = ms_max / args.steps
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+
+    # ---- per-kernel breakdown and the dominant kernel's roofline
+    peaks, peak_src = load_peaks()
+    per = {}
+    for name, t in recs:
+        per.setdefault(name, []).append(t)
+    work = kernel_work(cfg, R)
+    breakdown = {}
+    for name, ts in per.items():
+        avg = sum(ts) / len(ts)
+        entry = {"launches": len(ts), "avg_us": round(1e3 * avg, 2), "share": round(sum(ts) / max(ms, 1e-9), 4)}
+        if name in work:
+            fl, by = work[name]
+            entry["tflops"] = round(fl / (avg * 1e-3) / 1e12, 1)
+            entry["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
+        breakdown[name] = entry
+    dom = max(per, key=lambda k: sum(per[k]))
+    avg_dom = sum(per[dom]) / len(per[dom])
+    fl, by = work.get(dom, (0, 0))
+    intensity = fl / max(by, 1)
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity >= ridge:
+        achieved = fl / (avg_dom * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s"}
+    else:
+        achieved = by / (avg_dom * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'copy bandwidth'})"
+    roof["traffic"] = measured_traffic(dom, args.config)
+    tensor_peak = peaks["bf16_tflops_sustained"]
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Xh = X.cpu().pin_memory()
+        dOh = dO.cpu().pin_memory()
+        Oh = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+        Xd = torch.empty_like(X)
+        dOd = torch.empty_like(dO)
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            dOd.copy_(dOh, non_blocking=True)
+            layer.step(Xd, Wr, b, W1, W2, dOd)
+            if world > 1:
+                for g in (layer.dW1, layer.dW2, layer.dWr):
+                    dist.all_reduce(g)
+            Oh.copy_(layer.O, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([e0.elapsed_time(e1)], device=dev)
+        if world > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e_ms_step = float(ems.item()) / args.steps
+        e2e = {"value": round(flops_step * world / (e_ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(Xh.numel() * 2 + dOh.numel() * 2),
+               "d2h_bytes_per_step": int(Oh.numel() * 2), "ms_per_step": round(e_ms_step, 4)}
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = cpu_inputs(cfg)
+        tokens = min(args.cpu_sample_tokens, cfg.T)
+        dt, threads = oracle_step_seconds(cfg, inp_cpu, tokens)
+        cpu = {"value": round(18 * tokens * cfg.K * cfg.d * cfg.n / dt / 1e12, 6), "unit": "TFLOP/s",
+               "cores": threads, "kind": "oracle", "seconds": round(dt, 2),
+               "sample": f"first {tokens} of {cfg.T} tokens of the same batch and full weights, one "
+                         "route+forward+backward of the fp64 numpy oracle"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
+                       "router_bias": cfg.bias, "round_mode": cfg.round_mode,
+                       "parallelism": f"dp{world}" + (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else ""),
+                       "l2": "inputs larger than L2 (X+dO+W1+W2 = 402 MB per step, working set ~2 GB)"},
+            "tokens_per_s": round(cfg.T * world / (ms_step * 1e-3), 1),
+            "pct_of_tensor_peak": round(100 * value / world / tensor_peak, 2),
+            "roofline": roof,
+            "kernels": breakdown,
+            "gpu_launches": len(recs),
+            "routed_pairs": R,
+            "expert_load": {"min": min(counts), "max": max(counts), "mean": sum(counts) / len(counts)},
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -42,6 +42,17 @@ bool device_state(int* dev_out, int** status_out, int* sms_out) {
   return true;
 }
 
+// ----------------------------------------------------------------- profiler
+constexpr int kProfCap = 1 << 15;
+struct ProfRec {
+  cudaEvent_t a, b;
+  const char* name;
+};
+ProfRec g_prof[kProfCap];
+int g_prof_n = 0;        // records taken since the last enable
+int g_prof_created = 0;  // event pairs created so far (reused across enables)
+bool g_prof_on = false;
+
 // ----------------------------------------------------------------- TMA encoding
 using EncodeFn = decltype(&cuTensorMapEncodeTiled);
 EncodeFn g_encode = nullptr;
@@ -255,6 +266,23 @@ inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(
 
 }  // namespace
 
+namespace moe {
+ProfScope::ProfScope(cudaStream_t s, const char* name) : stream(s) {
+  if (!g_prof_on || g_prof_n >= kProfCap) return;
+  ProfRec& r = g_prof[g_prof_n];
+  if (g_prof_n >= g_prof_created) {
+    if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return;
+    ++g_prof_created;
+  }
+  r.name = name;
+  slot = g_prof_n++;
+  cudaEventRecord(r.a, stream);
+}
+ProfScope::~ProfScope() {
+  if (slot >= 0) cudaEventRecord(g_prof[slot].b, stream);
+}
+}  // namespace moe
+
 extern "C" {
 
 moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes* out) {
@@ -293,7 +321,10 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
   RouteArgs a = route_args(p, rt, w);
   a.Wr = Wr;
   a.st.word = status;
-  MOE_TRY_CUDA(launch_split_wr(a, st));
+  {
+    ProfScope ps(st, "router_split_wr");
+    MOE_TRY_CUDA(launch_split_wr(a, st));
+  }
 
   GemmParams g = base_params(p, rt, status);
   MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
@@ -302,9 +333,15 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
   g.num_n_tiles = p.Epad / 64;
   g.outf = const_cast<float*>(a.logits);
   g.bias = bias;
-  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+  {
+    ProfScope ps(st, "router_logits_gemm");
+    MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+  }
 
-  MOE_TRY_CUDA(launch_softmax_topk(a, st));
+  {
+    ProfScope ps(st, "router_softmax_topk");
+    MOE_TRY_CUDA(launch_softmax_topk(a, st));
+  }
   MOE_TRY_CUDA(launch_permute(a, st));
   return MOE_OK;
 }
@@ -367,6 +404,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.num_n_tiles = p.n / (p.bn_up / 2);
     g.out0 = static_cast<__nv_bfloat16*>(H);
     g.out1 = w.A;
+    ProfScope ps(st, "up_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   // down-projection: Y = A W2[e]
@@ -376,10 +414,14 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     MOE_TRY_MAP(make_tmap(&g.tmB, W2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 64));
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
+    ProfScope ps(st, "down_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
-  MOE_TRY_CUDA(launch_aggregate_fwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_gate, w.Y,
-                                    static_cast<__nv_bfloat16*>(O), st));
+  {
+    ProfScope ps(st, "aggregate_fwd");
+    MOE_TRY_CUDA(launch_aggregate_fwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_gate, w.Y,
+                                      static_cast<__nv_bfloat16*>(O), st));
+  }
   return MOE_OK;
 }
 
@@ -418,6 +460,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.out0 = w.dH;
     g.out1 = w.Ahat;
     g.outf = w.dS_part;
+    ProfScope ps(st, "dh_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   // dW2[e] = A_hat^T dO[tok]
@@ -429,6 +472,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.n, 128);
     g.num_n_tiles = p.d / p.bn_dw2;
     g.out0 = static_cast<__nv_bfloat16*>(dW2);
+    ProfScope ps(st, "dw2_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
@@ -439,6 +483,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
     g.num_n_tiles = p.d / p.bn_dxt;
     g.out0 = w.dXt;
+    ProfScope ps(st, "dxt_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   // dW1[e] = X[tok]^T dH
@@ -450,13 +495,20 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.d, 128);
     g.num_n_tiles = 2 * p.n / p.bn_dw1;
     g.out0 = static_cast<__nv_bfloat16*>(dW1);
+    ProfScope ps(st, "dw1_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
   if (rg) {
-    MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nts, rt->tok_ptr, rt->pair_row, rt->pair_expert,
-                                   rt->pair_gate, w.dS_part, w.dz_pair, w.dz_split, st));
-    MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
+    {
+      ProfScope ps(st, "router_bwd");
+      MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nts, rt->tok_ptr, rt->pair_row, rt->pair_expert,
+                                     rt->pair_gate, w.dS_part, w.dz_pair, w.dz_split, st));
+    }
+    {
+      ProfScope ps(st, "router_wr_transpose");
+      MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
+    }
     GemmParams g = base_params(p, rt, status);
     MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 64));
     MOE_TRY_MAP(make_tmap(&g.tmB, w.dz_split, (uint64_t)p.T, (uint64_t)2 * p.Epad, 64, 64));
@@ -465,12 +517,21 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.ksplit = p.ksplit;
     g.ksplit_rows = p.ksplit_rows;
     g.outf = w.dWr_part;
-    MOE_TRY_CUDA(launch_gemm(G_DWR, 128, g,
-                             grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st));
-    MOE_TRY_CUDA(launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st));
+    {
+      ProfScope ps(st, "router_dwr_gemm");
+      MOE_TRY_CUDA(launch_gemm(G_DWR, 128, g,
+                               grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st));
+    }
+    {
+      ProfScope ps(st, "router_dwr_reduce");
+      MOE_TRY_CUDA(launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st));
+    }
   }
-  MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_expert, w.dXt, w.dz_pair,
-                                    w.WrT, rg ? 1 : 0, static_cast<__nv_bfloat16*>(dX), st));
+  {
+    ProfScope ps(st, "aggregate_bwd");
+    MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_expert, w.dXt,
+                                      w.dz_pair, w.WrT, rg ? 1 : 0, static_cast<__nv_bfloat16*>(dX), st));
+  }
   return MOE_OK;
 }
 
@@ -501,6 +562,22 @@ moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream) {
   if (launch_wait_selftest(waited_ok, DevStatus{status, g_spin_limit}, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_profile_enable(int32_t on) {
+  if (on != 0 && on != 1) return MOE_ERR_INVALID_ARG;
+  if (on) g_prof_n = 0;
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+int32_t moe_profile_count(void) { return g_prof_n; }
+
+moe_status moe_profile_read(int32_t i, const char** name, float* ms) {
+  if (i < 0 || i >= g_prof_n || !name || !ms) return MOE_ERR_INVALID_ARG;
+  *name = g_prof[i].name;
+  if (cudaEventElapsedTime(ms, g_prof[i].a, g_prof[i].b) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -12,6 +12,15 @@ constexpr int kTile = 128;        // rows per expert tile (segments are padded t
 constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation
 
 cudaError_t launch_gemm(int kind, int bn, const GemmParams& p, int grid, cudaStream_t s);
+
+// Per-kernel timing (moe_profile_enable): while on, each launch site brackets
+// its kernel with two CUDA events recorded on the launching stream.
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t stream;
+  ProfScope(cudaStream_t s, const char* name);
+  ~ProfScope();
+};
 int gemm_smem_bytes(int bn);
 
 // ---- routing (moe_route.cu)

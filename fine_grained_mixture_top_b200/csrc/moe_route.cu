@@ -249,9 +249,18 @@ __global__ void scatter_kernel(RouteArgs a) {
 }
 
 cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s) {
-  rank_kernel<<<a.nchunks, kChunk, (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s>>>(a);
-  scan_kernel<<<1, 1024, 0, s>>>(a);
-  scatter_kernel<<<(a.T + 255) / 256, 256, 0, s>>>(a);
+  {
+    ProfScope ps(s, "permute_rank");
+    rank_kernel<<<a.nchunks, kChunk, (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s>>>(a);
+  }
+  {
+    ProfScope ps(s, "permute_scan");
+    scan_kernel<<<1, 1024, 0, s>>>(a);
+  }
+  {
+    ProfScope ps(s, "permute_scatter");
+    scatter_kernel<<<(a.T + 255) / 256, 256, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -390,13 +399,28 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
   cudaError_t err = cudaMemsetAsync(r.member, 0, mbytes, s);
   if (err != cudaSuccess) return err;
   const int tb = (r.T + 255) / 256;
-  tr_member_kernel<<<tb, 256, 0, s>>>(a.tok_ptr, a.pair_expert, r.T, r.Ew, r.member);
+  {
+    ProfScope ps(s, "round_member");
+    tr_member_kernel<<<tb, 256, 0, s>>>(a.tok_ptr, a.pair_expert, r.T, r.Ew, r.member);
+  }
   err = cudaMemcpyAsync(r.final_, r.member, mbytes, cudaMemcpyDeviceToDevice, s);
   if (err != cudaSuccess) return err;
-  tr_select_kernel<<<r.E, 1024, 0, s>>>(r.T, r.E, r.Ew, r.mode, r.seed, a.counts, r.probs, r.member, r.final_);
-  tr_count_kernel<<<tb, 256, 0, s>>>(r.final_, r.T, r.Ew, r.cnt);
-  tr_ptr_scan_kernel<<<1, 1024, 0, s>>>(r.cnt, r.T, a.tok_ptr);
-  tr_write_kernel<<<tb, 256, 0, s>>>(r.final_, r.probs, r.T, r.E, r.Ew, a.tok_ptr, a.pair_expert, a.pair_gate);
+  {
+    ProfScope ps(s, "round_select");
+    tr_select_kernel<<<r.E, 1024, 0, s>>>(r.T, r.E, r.Ew, r.mode, r.seed, a.counts, r.probs, r.member, r.final_);
+  }
+  {
+    ProfScope ps(s, "round_count");
+    tr_count_kernel<<<tb, 256, 0, s>>>(r.final_, r.T, r.Ew, r.cnt);
+  }
+  {
+    ProfScope ps(s, "round_scan");
+    tr_ptr_scan_kernel<<<1, 1024, 0, s>>>(r.cnt, r.T, a.tok_ptr);
+  }
+  {
+    ProfScope ps(s, "round_write");
+    tr_write_kernel<<<tb, 256, 0, s>>>(r.final_, r.probs, r.T, r.E, r.Ew, a.tok_ptr, a.pair_expert, a.pair_gate);
+  }
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   return launch_permute(a, s);

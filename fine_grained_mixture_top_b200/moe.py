@@ -72,6 +72,12 @@ def lib() -> ctypes.CDLL:
         L.moe_get_status.argtypes = [c_void_p, P(c_int32)]
         L.moe_set_spin_limit.argtypes = [c_int64]
         L.moe_selftest_wait_timeout.argtypes = [c_void_p, c_void_p]
+        L.moe_profile_enable.argtypes = [c_int32]
+        L.moe_profile_enable.restype = c_int32
+        L.moe_profile_count.argtypes = []
+        L.moe_profile_count.restype = c_int32
+        L.moe_profile_read.argtypes = [c_int32, P(ctypes.c_char_p), P(ctypes.c_float)]
+        L.moe_profile_read.restype = c_int32
         L.moe_status_str.argtypes = [c_int32]
         L.moe_status_str.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
@@ -181,6 +187,23 @@ def moe_set_spin_limit(cycles: int):
 
 def moe_selftest_wait_timeout(flag, stream=None):
     _check(lib().moe_selftest_wait_timeout(_ptr(flag), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def moe_profile_enable(on: bool):
+    _check(lib().moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def moe_profile_records() -> list[tuple[str, float]]:
+    """(kernel name, ms) of every launch recorded since moe_profile_enable(True);
+    the streams must have completed."""
+    L = lib()
+    out = []
+    name = ctypes.c_char_p()
+    ms = ctypes.c_float()
+    for i in range(L.moe_profile_count()):
+        _check(L.moe_profile_read(i, ctypes.byref(name), ctypes.byref(ms)), "moe_profile_read")
+        out.append((name.value.decode(), float(ms.value)))
+    return out
 
 
 class MoELayer:

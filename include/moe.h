@@ -184,6 +184,19 @@ moe_status moe_set_spin_limit(int64_t cycles);
  */
 moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream);
 
+/*
+ * Per-kernel timing for benchmarks.  While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on its launching stream
+ * (host-side bookkeeping only; the events are created once and reused).
+ * moe_profile_enable(1) clears earlier records; moe_profile_count() gives the
+ * number of kernel launches recorded; moe_profile_read(i, ...) returns the
+ * name and duration in ms of launch i once its stream has completed.  Not
+ * thread-safe; meant for one benchmarking thread.
+ */
+moe_status moe_profile_enable(int32_t on);
+int32_t moe_profile_count(void);
+moe_status moe_profile_read(int32_t i, const char** name, float* ms);
+
 /* Static description of a status code. */
 const char* moe_status_str(moe_status s);
 

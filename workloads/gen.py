@@ -91,18 +91,20 @@ def _gen(torch, device, seed: int):
     return g
 
 
-def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True) -> dict:
+def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True, rank: int = 0) -> dict:
     """Return the seeded input tensors of `cfg` on `device` (torch tensors).
 
     Large weight tensors are produced one expert at a time so that the fp32
-    temporaries stay small.
+    temporaries stay small.  `rank` selects a different batch of tokens (X and
+    dO) for data-parallel replica `rank`; the weights do not depend on it.
     """
     import torch
 
     dev = torch.device(device)
     base = 1000 * (cfg.seed + 1)
+    data = base + 100 * int(rank)
     out = {}
-    g = _gen(torch, dev, base + 1)
+    g = _gen(torch, dev, data + 1)
     out["X"] = (torch.randn(cfg.T, cfg.d, generator=g, device=dev) * cfg.x_std).to(torch.bfloat16)
 
     def expert_weights(shape_e, seed):
@@ -126,7 +128,7 @@ def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True) -> 
     else:
         out["bias"] = None
     if need_grad_inputs:
-        g = _gen(torch, dev, base + 6)
+        g = _gen(torch, dev, data + 6)
         out["dO"] = torch.randn(cfg.T, cfg.d, generator=g, device=dev).to(torch.bfloat16)
     return out
 
