@@ -1,0 +1,102 @@
+"""Data-parallel exchange step on CPU ranks (gloo, world size 2).
+
+The layer shards by tokens: each rank routes and computes its own batch
+against replicated weights, and the only exchange is the sum of the weight
+gradients.  These tests check that the sum of per-shard oracle gradients is
+the full-batch gradient, and that a rank that fails before the collective is
+detected by the others as an error instead of a hang."""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from oracle import moe_oracle as orc
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _layer(seed=3, T=96, d=16, E=6, n=8):
+    rs = np.random.RandomState(seed)
+    return (rs.randn(T, d), rs.randn(E, d, 2 * n) * 0.3, rs.randn(E, n, d) * 0.3, rs.randn(d, E) * 0.5,
+            rs.randn(E) * 0.5, rs.randn(T, d))
+
+
+def _shard_worker(rank, world, port, K, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    X, W1, W2, Wr, b, dO = _layer()
+    T = X.shape[0]
+    sl = slice(rank * T // world, (rank + 1) * T // world)
+    fw = orc.forward(X[sl], Wr, b, W1, W2, K)
+    bw = orc.backward(fw, dO[sl], X[sl], Wr, W1, W2)
+    grads = [torch.from_numpy(bw[k].copy()) for k in ("dW1", "dW2", "dWr")]
+    for g in grads:
+        dist.all_reduce(g)
+    if rank == 0:
+        out_q.put([g.numpy() for g in grads] + [bw["dX"]])
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sum_of_shard_gradients_is_full_batch_gradient():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world, K = 2, 2
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, K, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W1, W2, Wr, b, dO = _layer()
+    fw = orc.forward(X, Wr, b, W1, W2, K)
+    bw = orc.backward(fw, dO, X, Wr, W1, W2)
+    for mine, k in zip(got[:3], ("dW1", "dW2", "dWr")):
+        np.testing.assert_allclose(mine, bw[k], rtol=1e-10, atol=1e-12)
+    # dX of a shard is that shard's rows of the full-batch dX: no exchange needed
+    np.testing.assert_allclose(got[3], bw["dX"][:X.shape[0] // 2], rtol=1e-10, atol=1e-12)
+
+
+def _failing_worker(rank, world, port, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # this rank fails between steps, before joining the gradient exchange
+        os._exit(3)
+    g = torch.ones(8)
+    try:
+        dist.all_reduce(g)
+        out_q.put("no error")
+    except Exception as e:  # the surviving rank learns of the failure
+        out_q.put(type(e).__name__)
+
+
+def test_rank_failing_before_exchange_is_reported_not_hung():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert res != "no error"
+    assert procs[1].exitcode == 3
