@@ -590,8 +590,85 @@ const char* moe_status_str(moe_status s) {
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_DEVICE_CHECK: return "device consistency check failed";
+    case MOE_ERR_SCRATCH_LIMIT: return "shape needs more scratch than the static array holds";
   }
   return "unknown status";
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------- routing without caller scratch
+// moe_route_noalloc serves callers that cannot allocate device memory at all,
+// such as a plugin that is handed only its input and output buffers by a host
+// runtime, or code running under an allocator that owns the whole device pool
+// and cannot carve out a workspace.  Its scratch (Wr split, per-chunk expert
+// histograms, per-pair ranks) lives in the file-scope array below instead of
+// the caller's ws.  Every byte of it that a call reads is first written by the
+// same call, so the contents left by an earlier call never matter and nothing
+// needs clearing.  All calls on a device share the one array: calls whose GPU
+// work overlaps (different streams, no ordering between them) race.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Set-up, once per device, with that device current: the host-side symbol is
+// only a stand-in, so resolve the array's device address.
+bool noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return false;
+    g_noalloc_scratch_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return true;
+}
+
+size_t carve_noalloc_route(const Plan& p, void* base, RouteWs* w) {
+  Carve c{static_cast<char*>(base)};
+  w->Wr_split = c.take<__nv_bfloat16>((size_t)p.d * 3 * p.Epad);
+  w->hist = c.take<int>((size_t)p.nchunks * p.E);
+  w->local_rank = c.take<int>((size_t)p.T * p.K);
+  w->logits = nullptr;
+  w->member = nullptr;
+  w->final_ = nullptr;
+  w->cnt = nullptr;
+  return c.off;
+}
+}  // namespace
+
+extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
+                                        const float* bias, const moe_routing* rt, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  RouteWs w;
+  if (carve_noalloc_route(p, nullptr, &w) > kNoAllocScratchBytes) return MOE_ERR_SCRATCH_LIMIT;
+  if (!X || !Wr || !aligned16(X) || !aligned16(Wr) || (bias && !aligned16(bias)) || !routing_ok(rt, p, true) ||
+      !rt->logits)
+    return MOE_ERR_INVALID_ARG;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  void* scratch = nullptr;
+  if (!noalloc_scratch(dev, &scratch)) return MOE_ERR_CUDA;
+  carve_noalloc_route(p, scratch, &w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  RouteArgs a = route_args(p, rt, w);
+  a.Wr = Wr;
+  a.st.word = status;
+  MOE_TRY_CUDA(launch_split_wr(a, st));
+  GemmParams g = base_params(p, rt, status);
+  MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
+  MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
+  g.num_m_tiles = (int)cdiv(p.T, 128);
+  g.num_n_tiles = p.Epad / 64;
+  g.outf = rt->logits;
+  g.bias = bias;
+  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+  MOE_TRY_CUDA(launch_softmax_topk(a, st));
+  MOE_TRY_CUDA(launch_permute(a, st));
+  return MOE_OK;
+}

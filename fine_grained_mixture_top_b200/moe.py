@@ -18,7 +18,7 @@ c_int32 = ctypes.c_int32
 c_int64 = ctypes.c_int64
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
-    MOE_ERR_DEVICE_CHECK = range(7)
+    MOE_ERR_DEVICE_CHECK, MOE_ERR_SCRATCH_LIMIT = range(8)
 
 
 class MoeDims(ctypes.Structure):
@@ -63,6 +63,9 @@ def lib() -> ctypes.CDLL:
         L.moe_query_sizes.argtypes = [P(MoeDims), P(MoeOpts), P(MoeSizes)]
         L.moe_route.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
                                 ctypes.c_size_t, c_void_p]
+        L.moe_route_noalloc.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting),
+                                         c_void_p]
+        L.moe_route_noalloc.restype = c_int32
         L.moe_token_round.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, ctypes.c_size_t, c_void_p]
         L.moe_forward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
                                   c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
@@ -155,6 +158,13 @@ def moe_route(dims, opts, X, Wr, bias, routing: Routing, ws, stream=None):
     _check(lib().moe_route(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(Wr), _ptr(bias),
                            ctypes.byref(routing.struct), _ptr(ws), ws.numel() * ws.element_size(),
                            _stream(stream)), "moe_route")
+
+
+def moe_route_noalloc(dims, opts, X, Wr, bias, routing: Routing, stream=None):
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory; its scratch is a 16 MiB static array in the library (see moe.h)."""
+    _check(lib().moe_route_noalloc(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(Wr), _ptr(bias),
+                                   ctypes.byref(routing.struct), _stream(stream)), "moe_route_noalloc")
 
 
 def moe_token_round(dims, opts, routing: Routing, ws, stream=None):

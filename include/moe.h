@@ -46,7 +46,8 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,     /* ws NULL or smaller than moe_query_sizes() asks */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch error, no device) */
   MOE_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out */
-  MOE_ERR_DEVICE_CHECK = 6   /* device: an internal consistency check failed */
+  MOE_ERR_DEVICE_CHECK = 6,  /* device: an internal consistency check failed */
+  MOE_ERR_SCRATCH_LIMIT = 7  /* moe_route_noalloc: the shape needs more than its static scratch */
 } moe_status;
 
 /* Layer shape: T tokens, model width d, E experts of intermediate width n, top-K. */
@@ -196,6 +197,32 @@ moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream);
 moe_status moe_profile_enable(int32_t on);
 int32_t moe_profile_count(void);
 moe_status moe_profile_read(int32_t i, const char** name, float* ms);
+
+/*
+ * moe_route_noalloc -- moe_route for callers that cannot allocate device
+ * memory.  Such callers exist: a plugin that a host runtime hands only its
+ * input and output buffers, or code running under an allocator that owns the
+ * whole device pool and cannot give out a workspace.  The pages have no
+ * counterpart to this entry point; it is a deployment convenience.
+ *
+ * Same inputs and outputs as moe_route (rt->logits must be non-NULL here),
+ * but no ws: the scratch (Wr split, chunk histograms, pair ranks) lives in a
+ * 16 MiB static device array inside the library.  Every GPU that loads the
+ * library holds that array until the process exits.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on each device resolves the array's device address (a
+ *     set-up step done once per device, with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the array, and it keeps the previous call's
+ *     contents (each call writes every scratch byte it reads first).  Calls
+ *     whose GPU work overlaps race on it: order them (one stream, or events).
+ *   - Returns MOE_ERR_SCRATCH_LIMIT, without touching the GPU, when the shape
+ *     needs more than 16 MiB of scratch:
+ *       2*d*3*ceil(E/64)*64 + 4*ceil(T/256)*E + 4*T*K bytes (each part rounded
+ *       up to 256 bytes).
+ */
+moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
+                             const float* bias, const moe_routing* rt, void* stream);
 
 /* Static description of a status code. */
 const char* moe_status_str(moe_status s);
