@@ -74,6 +74,7 @@ constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
 constexpr int kStageBudget = 200 * 1024;
+constexpr int kRtrGroup = 4;  // router logits: k-blocks per promoted hi-part group
 
 template <int BN>
 struct GemmShape {
@@ -259,8 +260,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
   uint64_t* empty = bars + S;
   uint64_t* acc_full = bars + 2 * S;
   uint64_t* acc_empty = bars + 2 * S + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 5);
+  uint64_t* hi_full = bars + 2 * S + 4;   // router logits: promoted hi-part groups
+  uint64_t* hi_empty = bars + 2 * S + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 9);
+  // the router-logit kind keeps one tile buffer of 256 columns: [hi_a | hi_b | mid | lo]
+  constexpr int kTmemCols = (KIND == G_RTR) ? 256 : SH::kTmemCols;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -273,6 +278,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
+      mbar_init(&hi_full[b], 1);
+      mbar_init(&hi_empty[b], 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -282,7 +289,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     if constexpr (!KT::kBGather) tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), SH::kTmemCols);
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -309,6 +316,63 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
           issue_tma<KIND, BN>(p, t, kb, a_s, a_s + kABytes, smem_u32(&full[s]));
         }
       }
+    }
+  } else if (warp == 1 && KIND == G_RTR) {
+    // ---------------- MMA issuer, router logits.  The hi part of Wr (which
+    // carries almost all of each logit) is accumulated in groups of kRtrGroup
+    // k-blocks into two alternating TMEM slots; the epilogue adds every group
+    // into fp32 registers, so the tensor core's long accumulation chain is cut
+    // into short ones.  The mid and lo parts accumulate over the whole K.
+    constexpr uint32_t kIdescHi = idesc_bf16_f32(64, KT::kAMN, KT::kBMN);
+    constexpr uint32_t kIdescMl = idesc_bf16_f32(128, KT::kAMN, KT::kBMN);
+    int it = 0, tcount = 0, hg = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if (!mbar_wait(smem_u32(&acc_empty[0]), (tcount & 1) ^ 1, abort_flag, p.st, KIND * 16 + 7)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int slot = 0;
+      for (int kb = 0; kb < t.nkb && ok; ++kb, ++it) {
+        const bool first = (kb % kRtrGroup) == 0;
+        const bool last = (kb % kRtrGroup) == kRtrGroup - 1 || kb == t.nkb - 1;
+        if (first) {
+          slot = hg & 1;
+          if (!mbar_wait(smem_u32(&hi_empty[slot]), ((hg >> 1) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 8)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int s = it % S;
+        if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_s = base + s * SH::kStageBytes;
+          const uint32_t b_s = a_s + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_s + kk * 32, 16, 1024);
+            const uint64_t bhi = smem_desc_sw128(b_s + kk * 2048, kBoxBytes, 1024);
+            const uint64_t bml = smem_desc_sw128(b_s + kBoxBytes + kk * 2048, kBoxBytes, 1024);
+            tc_mma_bf16(tmem_base + (uint32_t)(slot * 64), ad, bhi, kIdescHi, (first && kk == 0) ? 0u : 1u);
+            tc_mma_bf16(tmem_base + 128u, ad, bml, kIdescMl, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&empty[s]));
+          if (last) tc_commit(smem_u32(&hi_full[slot]));
+        }
+        __syncwarp();
+        if (last) ++hg;
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(smem_u32(&acc_full[0]));
+      __syncwarp();
+      ++tcount;
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -352,6 +416,65 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       __syncwarp();
       ++tcount;
     }
+  } else if (warp < 6 && KIND == G_RTR) {
+    // ---------------- epilogue, router logits: z = sum of promoted hi groups + mid + lo + bias
+    const int q = warp & 3;
+    const int rloc = q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    int tcount = 0, hg = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      float hs[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) hs[i] = 0.f;
+      const int ngroups = (t.nkb + kRtrGroup - 1) / kRtrGroup;
+      for (int grp = 0; grp < ngroups; ++grp, ++hg) {
+        const int slot = hg & 1;
+        if (!mbar_wait(smem_u32(&hi_full[slot]), (hg >> 1) & 1, abort_flag, p.st, KIND * 16 + 9)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_addr + slot * 64, r0);
+        tmem_ld32(lane_addr + slot * 64 + 32, r1);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          hs[i] += __uint_as_float(r0[i]);
+          hs[32 + i] += __uint_as_float(r1[i]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&hi_empty[slot]));
+      }
+      if (!ok) break;
+      if (!mbar_wait(smem_u32(&acc_full[0]), tcount & 1, abort_flag, p.st, KIND * 16 + 4)) break;
+      tc_fence_after();
+      const int trow = t.m0 + rloc;
+      float* dst = p.outf + (size_t)trow * p.E;
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 32) {
+        uint32_t mid[32], lo[32];
+        tmem_ld32(lane_addr + 128 + c, mid);
+        tmem_ld32(lane_addr + 192 + c, lo);
+        tc_wait_ld();
+        if (trow < p.T) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = t.nt * 64 + c + i;
+            if (e < p.E) {
+              float z = (c == 0 ? hs[i] : hs[32 + i]) + (__uint_as_float(mid[i]) + __uint_as_float(lo[i]));
+              if (p.bias) z += __ldg(p.bias + e);
+              dst[e] = z;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[0]));
+      ++tcount;
+    }
   } else if (warp < 6) {
     // ---------------- epilogue: one accumulator row per thread
     const int q = warp & 3;
@@ -380,6 +503,16 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
             for (int c = 0; c < 64; ++c) dst[c] = 0.f;
           }
           continue;
+        }
+      }
+      // dH epilogue: start loading this row's first H chunk while the MMAs run
+      uint4 h_nx[8];
+      if constexpr (KIND == G_DH) {
+        const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)(t.m0 + rloc) * (2 * p.n) + t.n0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          h_nx[q] = __ldg(h4 + q);
+          h_nx[4 + q] = __ldg(h4 + p.n / 8 + q);
         }
       }
       const int b = tcount & 1;
@@ -426,35 +559,67 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       } else if constexpr (KIND == G_DH) {
         const int r = t.m0 + rloc;
         const float s = __ldg(p.row_gate + r);
-        const __nv_bfloat16* Hrow = p.hin + (size_t)r * (2 * p.n);
-        __nv_bfloat16* dHrow = p.out0 + (size_t)r * (2 * p.n);
-        __nv_bfloat16* Ahrow = p.out1 + (size_t)r * p.n;
+        const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)r * (2 * p.n) + t.n0);
+        uint4* dg4 = reinterpret_cast<uint4*>(p.out0 + (size_t)r * (2 * p.n) + t.n0);
+        uint4* ah4 = reinterpret_cast<uint4*>(p.out1 + (size_t)r * p.n + t.n0);
+        const int up8 = p.n / 8;  // offset of the up half in 16-byte units
         float dsum = 0.f;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t a[32];
           tmem_ld32(tacc + c, a);
-          float gv[32], uv[32];
-          load_row32_bf16(Hrow + t.n0 + c, gv);
-          load_row32_bf16(Hrow + p.n + t.n0 + c, uv);
-          tc_wait_ld();
-          float dg[32], du[32], ah[32];
+          uint4 hc[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float dap = __uint_as_float(a[i]);
-            const float g = gv[i], u = uv[i];
-            const float sg = sigmoidf_(g);
-            const float silu = g * sg;
-            const float A = silu * u;
-            dsum = fmaf(dap, A, dsum);
-            const float dA = s * dap;
-            dg[i] = dA * u * sg * (1.0f + g * (1.0f - sg));
-            du[i] = dA * silu;
-            ah[i] = s * A;
+          for (int q = 0; q < 8; ++q) hc[q] = h_nx[q];
+          if (c + 32 < BN) {  // prefetch the next chunk of H
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              h_nx[q] = __ldg(h4 + (c + 32) / 8 + q);
+              h_nx[4 + q] = __ldg(h4 + up8 + (c + 32) / 8 + q);
+            }
           }
-          store_row32_bf16(dHrow + t.n0 + c, dg);
-          store_row32_bf16(dHrow + p.n + t.n0 + c, du);
-          store_row32_bf16(Ahrow + t.n0 + c, ah);
+          tc_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hc[q]);
+            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&hc[4 + q]);
+            float dg[8], du[8], ah[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 gf = __bfloat1622float2(g2[i]);
+              const float2 uf = __bfloat1622float2(u2[i]);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float g = h ? gf.y : gf.x;
+                const float u = h ? uf.y : uf.x;
+                const float dap = __uint_as_float(a[8 * q + 2 * i + h]);
+                const float sg = sigmoidf_(g);
+                const float silu = g * sg;
+                const float A = silu * u;
+                dsum = fmaf(dap, A, dsum);
+                const float dA = s * dap;
+                dg[2 * i + h] = dA * u * sg * (1.0f + g * (1.0f - sg));
+                du[2 * i + h] = dA * silu;
+                ah[2 * i + h] = s * A;
+              }
+            }
+            uint4 w;
+            w.x = pack_bf16x2(dg[0], dg[1]);
+            w.y = pack_bf16x2(dg[2], dg[3]);
+            w.z = pack_bf16x2(dg[4], dg[5]);
+            w.w = pack_bf16x2(dg[6], dg[7]);
+            dg4[c / 8 + q] = w;
+            w.x = pack_bf16x2(du[0], du[1]);
+            w.y = pack_bf16x2(du[2], du[3]);
+            w.z = pack_bf16x2(du[4], du[5]);
+            w.w = pack_bf16x2(du[6], du[7]);
+            dg4[up8 + c / 8 + q] = w;
+            w.x = pack_bf16x2(ah[0], ah[1]);
+            w.y = pack_bf16x2(ah[2], ah[3]);
+            w.z = pack_bf16x2(ah[4], ah[5]);
+            w.w = pack_bf16x2(ah[6], ah[7]);
+            ah4[c / 8 + q] = w;
+          }
         }
         p.outf[(size_t)r * p.num_n_tiles + t.nt] = dsum;
       } else if constexpr (KT::kGroupedK) {
@@ -471,28 +636,6 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
             store_row32_bf16(p.out0 + ((size_t)t.e * M + m) * N + t.n0 + c, v);
-          }
-        }
-      } else if constexpr (KIND == G_RTR) {
-        const int trow = t.m0 + rloc;
-#pragma unroll 1
-        for (int c = 0; c < 64; c += 32) {
-          uint32_t hi[32], mid[32], lo[32];
-          tmem_ld32(tacc + c, hi);
-          tmem_ld32(tacc + 64 + c, mid);
-          tmem_ld32(tacc + 128 + c, lo);
-          tc_wait_ld();
-          if (trow < p.T) {
-            float* dst = p.outf + (size_t)trow * p.E;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int e = t.nt * 64 + c + i;
-              if (e < p.E) {
-                float z = __uint_as_float(hi[i]) + __uint_as_float(mid[i]) + __uint_as_float(lo[i]);
-                if (p.bias) z += __ldg(p.bias + e);
-                dst[e] = z;
-              }
-            }
           }
         }
       } else {  // G_DWR
@@ -559,10 +702,27 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
           }
         }
       } else {
-        // MN-major gathered operand: 64 K-rows (tokens) per k-block
+        // MN-major gathered operand: 64 K-rows (tokens) per k-block.  The row
+        // indices of the next two k-blocks are loaded ahead, so the dependent
+        // index load does not sit in front of every k-block's copies.
         constexpr int nbox = (KIND == G_DW1) ? 2 : BN / 64;
+        int tk[3][4];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tk[q + 1][j] = q < t.nkb ? __ldg(p.row_tok + t.krow0 + q * kBK + line0 + 16 * j) : -1;
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tk[0][j] = tk[1][j];
+            tk[1][j] = tk[2][j];
+          }
+          if (kb + 2 < t.nkb) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tk[2][j] = __ldg(p.row_tok + t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
+          }
           if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
             ok = false;
             break;
@@ -571,7 +731,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int i = line0 + 16 * j;
-            const int tok = __ldg(p.row_tok + t.krow0 + kb * kBK + i);
+            const int tok = tk[0][j];
 #pragma unroll
             for (int bx = 0; bx < nbox; ++bx) {
               const int col = (KIND == G_DW1 ? t.m0 : t.n0) + 64 * bx + chunk * 8;
@@ -603,7 +763,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, SH::kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

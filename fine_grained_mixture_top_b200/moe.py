@@ -243,9 +243,10 @@ class MoELayer:
         if self.opts.round_mode:
             moe_token_round(self.dims, self.opts, self.routing, self.ws_route, stream)
 
-    def forward(self, X, W1, W2, stream=None):
-        moe_forward(self.dims, self.opts, X, W1, W2, self.routing, self.O, self.H, self.ws_fwd, stream)
-        return self.O
+    def forward(self, X, W1, W2, stream=None, O=None):
+        O = self.O if O is None else O
+        moe_forward(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd, stream)
+        return O
 
     def backward(self, dO, X, Wr, W1, W2, stream=None):
         moe_backward(self.dims, self.opts, dO, X, Wr, W1, W2, self.routing, self.H, self.dX, self.dW1, self.dW2,
@@ -257,3 +258,63 @@ class MoELayer:
         self.route(X, Wr, bias, stream)
         self.forward(X, W1, W2, stream)
         return self.backward(dO, X, Wr, W1, W2, stream)
+
+
+class HostFedRunner:
+    """Whole steps (route, forward, backward) on batches held in pinned host
+    memory.  Each step's inputs X and dO are copied to the device on a copy
+    stream and its output O is copied back on a second copy stream as soon as
+    the forward is done, so the copies of consecutive steps overlap with the
+    kernels.  Device input and output buffers alternate between two sets;
+    events keep a buffer from being overwritten while a step still uses it.
+    Weight gradients stay on the device (layer.dW1, layer.dW2, layer.dWr)."""
+
+    def __init__(self, layer: MoELayer):
+        import torch
+        T, d = layer.dims.T, layer.dims.d
+        dev = layer.device
+        bf = torch.bfloat16
+        self.layer = layer
+        self.X = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
+        self.dO = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
+        self.O = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        ev = torch.cuda.Event
+        self.inputs_ready = [ev(), ev()]
+        self.inputs_free = [ev(), ev()]
+        self.fwd_done = [ev(), ev()]
+        self.out_free = [ev(), ev()]
+        self.i = 0
+
+    def step(self, Xh, dOh, Oh, Wr, bias, W1, W2):
+        """Enqueue one step; Xh, dOh, Oh are pinned host tensors [T, d] bf16.
+        Returns immediately; call finish() before reading Oh."""
+        import torch
+        j = self.i & 1
+        compute = torch.cuda.current_stream()
+        L = self.layer
+        with torch.cuda.stream(self.h2d):
+            self.h2d.wait_event(self.inputs_free[j])
+            self.X[j].copy_(Xh, non_blocking=True)
+            self.dO[j].copy_(dOh, non_blocking=True)
+            self.inputs_ready[j].record(self.h2d)
+        compute.wait_event(self.inputs_ready[j])
+        compute.wait_event(self.out_free[j])
+        L.route(self.X[j], Wr, bias)
+        L.forward(self.X[j], W1, W2, O=self.O[j])
+        self.fwd_done[j].record(compute)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.fwd_done[j])
+            Oh.copy_(self.O[j], non_blocking=True)
+            self.out_free[j].record(self.d2h)
+        L.backward(self.dO[j], self.X[j], Wr, W1, W2)
+        self.inputs_free[j].record(compute)
+        self.i += 1
+
+    def finish(self):
+        """Make the current stream wait for every copy enqueued so far."""
+        import torch
+        compute = torch.cuda.current_stream()
+        compute.wait_stream(self.h2d)
+        compute.wait_stream(self.d2h)

@@ -214,7 +214,7 @@ def forward(X, Wr, bias, W1, W2, K, topk_idx=None, routing=None):
     return out
 
 
-def backward(fw, dO, X, Wr, W1, W2, router_grad=True):
+def backward(fw, dO, X, Wr, W1, W2, router_grad=True, weight_grad_experts=None):
     """Layer backward as the method orders it ([P2] implementation paragraph:
     activation-gradient kernels dH (down-proj), the up-proj activation gradient,
     dX aggregation, and the two weight-gradient kernels dW1, dW2).
@@ -224,6 +224,11 @@ def backward(fw, dO, X, Wr, W1, W2, router_grad=True):
     paragraph; [P1] "第一，激活内存与专家粒度解耦": the contraction order is
     rearranged so the down-projection output is not cached, and no extra
     matmul is recomputed).
+
+    weight_grad_experts: None computes dW1/dW2 for every expert as [E, ...]
+    arrays; a list computes them only for those experts and returns dicts
+    {expert: array} (for layers whose full weight gradients do not fit in
+    host memory).  The arithmetic is the same either way.
     """
     X = np.asarray(X, F64)
     dO = np.asarray(dO, F64)
@@ -238,8 +243,16 @@ def backward(fw, dO, X, Wr, W1, W2, router_grad=True):
     Ahat = np.zeros((R, n), F64)
     dS_row = np.zeros(R, F64)
     dXt = np.zeros((R, d), F64)
-    dW1 = np.zeros((E, d, 2 * n), F64)
-    dW2 = np.zeros((E, n, d), F64)
+    if weight_grad_experts is None:
+        dW1 = np.zeros((E, d, 2 * n), F64)
+        dW2 = np.zeros((E, n, d), F64)
+        wanted = set(range(E))
+    else:
+        dW1, dW2 = {}, {}
+        wanted = set(int(e) for e in weight_grad_experts)
+        for e in wanted:
+            dW1[e] = np.zeros((d, 2 * n), F64)
+            dW2[e] = np.zeros((n, d), F64)
     for e in range(E):
         a, b = seg[e], seg[e + 1]
         if b == a:
@@ -261,9 +274,10 @@ def backward(fw, dO, X, Wr, W1, W2, router_grad=True):
         dH[a:b, n:] = du
         Ahat[a:b] = s * A
         # weight gradients and the up-proj activation gradient
-        dW2[e] = Ahat[a:b].T @ dOe
         dXt[a:b] = dH[a:b] @ W1e.T
-        dW1[e] = X[row_tok[a:b]].T @ dH[a:b]
+        if e in wanted:
+            dW2[e] = Ahat[a:b].T @ dOe
+            dW1[e] = X[row_tok[a:b]].T @ dH[a:b]
     # dX aggregation over each token's pairs
     tok_ptr, pair_row, pair_expert, pair_gate = (fw["tok_ptr"], fw["pair_row"],
                                                  fw["pair_expert"], fw["pair_gate"])

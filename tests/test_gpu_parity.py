@@ -129,3 +129,27 @@ def test_argument_errors_are_synchronous():
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_route(layer.dims, layer.opts, X[:, 1:], Wr, None, layer.routing, layer.ws_route)
     assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_host_fed_runner_matches_device_steps():
+    """Steps fed from pinned host memory give the same outputs as steps on
+    device-resident inputs."""
+    from fine_grained_mixture_top_b200 import moe
+    cfg = SHAPES[1]
+    inp = make_inputs(cfg, "cuda")
+    ref = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    runner = moe.HostFedRunner(layer)
+    Xh = inp["X"].cpu().pin_memory()
+    dOh = inp["dO"].cpu().pin_memory()
+    outs = [torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    for Oh in outs:        # three steps in a row, both buffer sets used
+        runner.step(Xh, dOh, Oh, inp["Wr"], inp["bias"], inp["W1"], inp["W2"])
+    runner.finish()
+    torch.cuda.synchronize()
+    assert moe.moe_get_status() == (0, 0)
+    for Oh in outs:
+        assert torch.equal(Oh, ref.O.cpu())
+    for k in ("dX", "dW1", "dW2", "dWr"):
+        assert torch.equal(getattr(layer, k), getattr(ref, k)), k

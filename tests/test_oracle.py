@@ -313,3 +313,15 @@ def test_token_round_tie_order():
     m = out["member"]
     assert list(np.nonzero(m[:, 0])[0]) == list(range(8))           # 8, 9, 10 dropped
     assert list(np.nonzero(m[:, 1])[0]) == [0, 1] + list(range(11, 17))  # 0, 1 added
+
+
+def test_weight_grads_for_an_expert_subset_match_the_full_backward():
+    X, W1, W2, Wr, b, dO = rand_layer(64, 12, 6, 4, 2, 9, bias=True)
+    fw = orc.forward(X, Wr, b, W1, W2, 2)
+    full = orc.backward(fw, dO, X, Wr, W1, W2)
+    part = orc.backward(fw, dO, X, Wr, W1, W2, weight_grad_experts=[1, 4])
+    for e in (1, 4):
+        np.testing.assert_array_equal(part["dW1"][e], full["dW1"][e])
+        np.testing.assert_array_equal(part["dW2"][e], full["dW2"][e])
+    np.testing.assert_array_equal(part["dX"], full["dX"])
+    assert set(part["dW1"]) == {1, 4}
