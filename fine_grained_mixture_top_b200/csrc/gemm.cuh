@@ -29,6 +29,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace moe {
@@ -36,8 +38,10 @@ namespace moe {
 enum GemmKind : int { G_UP = 0, G_DOWN, G_DH, G_DXT, G_DW1, G_DW2, G_RTR, G_DWR };
 
 struct GemmParams {
-  CUtensorMap tmA;  // TMA map of A (kinds whose A is not gathered)
-  CUtensorMap tmB;  // TMA map of B (kinds whose B is not gathered)
+  CUtensorMap tmA;   // TMA map of A (kinds whose A is not gathered)
+  CUtensorMap tmB;   // TMA map of B (kinds whose B is not gathered)
+  CUtensorMap tmC0;  // TMA store map of the first bf16 output (32 x 32 boxes, 64B swizzle)
+  CUtensorMap tmC1;  // TMA store map of the second bf16 output (UP: A, DH: A_hat)
   DevStatus st;
   const int* offsets;      // [E+1] 128-aligned segment starts
   const int* counts;       // [E]
@@ -75,6 +79,7 @@ constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
 constexpr int kStageBudget = 200 * 1024;
 constexpr int kRtrGroup = 4;  // router logits: k-blocks per promoted hi-part group
+constexpr int kStoreBuf = 2048;  // one epilogue staging buffer: 32 rows x 32 bf16
 
 template <int BN>
 struct GemmShape {
@@ -85,7 +90,8 @@ struct GemmShape {
   // accumulator buffers start at power-of-two column offsets
   static constexpr int kAccStride = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);
   static constexpr int kTmemCols = 2 * kAccStride;
-  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kStoreOffset = kStages * kStageBytes;         // epilogue staging
+  static constexpr int kBarOffset = kStoreOffset + 4 * 3 * 2048;      // 4 warps x 3 buffers x 2 KB
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;  // barriers + alignment slack
 };
 
@@ -240,6 +246,24 @@ __device__ __forceinline__ void zero32(float (&v)[32]) {
 }
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
+// Epilogue staging: a 32-row x 32-column bf16 box laid out with the 64-byte
+// swizzle the output tensor maps use; thread `row` writes its row.
+__device__ __forceinline__ uint32_t sw64(int row, int chunk) {
+  return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ uint4 pack8f(const float* v) {
+  uint4 w;
+  w.x = pack_bf16x2(v[0], v[1]);
+  w.y = pack_bf16x2(v[2], v[3]);
+  w.z = pack_bf16x2(v[4], v[5]);
+  w.w = pack_bf16x2(v[6], v[7]);
+  return w;
+}
+__device__ __forceinline__ void stage_row32(uint32_t buf, int row, const float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) st_shared_v4(buf + sw64(row, c), pack8f(v + 8 * c));
+}
+
 // ----------------------------------------------------------------- kernel
 template <int KIND, int BN>
 __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
@@ -247,7 +271,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
   using KT = KindTraits<KIND>;
   using SH = GemmShape<BN>;
   constexpr int S = SH::kStages;
-  constexpr int kLag = S - 1;
+  constexpr int kLag = 1;  // a group is published one k-block after it was issued
   constexpr uint32_t kIdesc = idesc_bf16_f32(BN, KT::kAMN, KT::kBMN);
 
   extern __shared__ uint8_t smem_raw[];
@@ -476,22 +500,45 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       ++tcount;
     }
   } else if (warp < 6) {
-    // ---------------- epilogue: one accumulator row per thread
+    // ---------------- epilogue: one accumulator row per thread.  bf16 results
+    // are staged per warp in shared memory (32 rows x 32 columns) and written
+    // with TMA tensor stores; each warp owns three 2 KB staging buffers.
     const int q = warp & 3;
     const int rloc = q * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    const uint32_t stg = base + SH::kStoreOffset + q * (3 * kStoreBuf);
+    int ring = 0;  // next staging buffer for one-output kinds
+    // Make staging buffer(s) free: `pending` store groups may still be reading.
+    auto stage_wait = [&](auto pending_tag) {
+      constexpr int kPend = decltype(pending_tag)::value;
+      if (lane == 0) bulk_wait_read<kPend>();
+      __syncwarp();
+    };
+    auto stage_publish = [&]() {
+      fence_proxy_async_smem();
+      __syncwarp();
+    };
     int tcount = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      const int row0 = t.m0 + q * 32;  // first output row of this warp's slice
       if constexpr (KT::kGroupedK) {
         if (t.nkb == 0) {  // expert without tokens: its weight gradient is zero
           const int M = (KIND == G_DW1) ? p.d : p.n;
-          const int N = (KIND == G_DW1) ? 2 * p.n : p.d;
-          const int m = t.m0 + rloc;
-          if (m < M) {
+          if (row0 < M) {
             float z[32];
             zero32(z);
-            for (int c = 0; c < BN; c += 32) store_row32_bf16(p.out0 + ((size_t)t.e * M + m) * N + t.n0 + c, z);
+            for (int c = 0; c < BN; c += 32) {
+              const uint32_t buf = stg + ring * kStoreBuf;
+              stage_wait(std::integral_constant<int, 2>{});
+              stage_row32(buf, lane, z);
+              stage_publish();
+              if (lane == 0) {
+                tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
+                bulk_commit();
+              }
+              ring = ring == 2 ? 0 : ring + 1;
+            }
           }
           continue;
         }
@@ -510,9 +557,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       if constexpr (KIND == G_DH) {
         const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)(t.m0 + rloc) * (2 * p.n) + t.n0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          h_nx[q] = __ldg(h4 + q);
-          h_nx[4 + q] = __ldg(h4 + p.n / 8 + q);
+        for (int i = 0; i < 4; ++i) {
+          h_nx[i] = __ldg(h4 + i);
+          h_nx[4 + i] = __ldg(h4 + p.n / 8 + i);
         }
       }
       const int b = tcount & 1;
@@ -523,9 +570,6 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
 
       if constexpr (KIND == G_UP) {
         constexpr int BNh = BN / 2;
-        const int r = t.m0 + rloc;
-        __nv_bfloat16* Hrow = p.out0 + (size_t)r * (2 * p.n);
-        __nv_bfloat16* Arow = p.out1 + (size_t)r * p.n;
 #pragma unroll 1
         for (int c = 0; c < BNh; c += 32) {
           uint32_t g[32], u[32];
@@ -539,29 +583,50 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
             uv[i] = bf16_round(__uint_as_float(u[i]));
             av[i] = gv[i] * sigmoidf_(gv[i]) * uv[i];
           }
-          store_row32_bf16(Hrow + t.n0 + c, gv);
-          store_row32_bf16(Hrow + p.n + t.n0 + c, uv);
-          store_row32_bf16(Arow + t.n0 + c, av);
+          stage_wait(std::integral_constant<int, 0>{});
+          stage_row32(stg, lane, gv);
+          stage_row32(stg + kStoreBuf, lane, uv);
+          stage_row32(stg + 2 * kStoreBuf, lane, av);
+          stage_publish();
+          if (lane == 0) {
+            tma_store_2d(&p.tmC0, stg, t.n0 + c, row0);
+            tma_store_2d(&p.tmC0, stg + kStoreBuf, p.n + t.n0 + c, row0);
+            tma_store_2d(&p.tmC1, stg + 2 * kStoreBuf, t.n0 + c, row0);
+            bulk_commit();
+          }
         }
-      } else if constexpr (KIND == G_DOWN || KIND == G_DXT) {
-        const int r = t.m0 + rloc;
-        __nv_bfloat16* row = p.out0 + (size_t)r * p.d + t.n0;
+      } else if constexpr (KIND == G_DOWN || KIND == G_DXT || KT::kGroupedK) {
+        int orow = row0;
+        bool live = true;
+        if constexpr (KT::kGroupedK) {
+          const int M = (KIND == G_DW1) ? p.d : p.n;
+          live = row0 < M;
+          orow = t.e * M + row0;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t a[32];
           tmem_ld32(tacc + c, a);
           tc_wait_ld();
-          float v[32];
+          if (live) {
+            float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
-          store_row32_bf16(row + c, v);
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+            const uint32_t buf = stg + ring * kStoreBuf;
+            stage_wait(std::integral_constant<int, 2>{});
+            stage_row32(buf, lane, v);
+            stage_publish();
+            if (lane == 0) {
+              tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
+              bulk_commit();
+            }
+            ring = ring == 2 ? 0 : ring + 1;
+          }
         }
       } else if constexpr (KIND == G_DH) {
         const int r = t.m0 + rloc;
         const float s = __ldg(p.row_gate + r);
         const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)r * (2 * p.n) + t.n0);
-        uint4* dg4 = reinterpret_cast<uint4*>(p.out0 + (size_t)r * (2 * p.n) + t.n0);
-        uint4* ah4 = reinterpret_cast<uint4*>(p.out1 + (size_t)r * p.n + t.n0);
         const int up8 = p.n / 8;  // offset of the up half in 16-byte units
         float dsum = 0.f;
 #pragma unroll 1
@@ -570,19 +635,20 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
           tmem_ld32(tacc + c, a);
           uint4 hc[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) hc[q] = h_nx[q];
+          for (int i = 0; i < 8; ++i) hc[i] = h_nx[i];
           if (c + 32 < BN) {  // prefetch the next chunk of H
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              h_nx[q] = __ldg(h4 + (c + 32) / 8 + q);
-              h_nx[4 + q] = __ldg(h4 + up8 + (c + 32) / 8 + q);
+            for (int i = 0; i < 4; ++i) {
+              h_nx[i] = __ldg(h4 + (c + 32) / 8 + i);
+              h_nx[4 + i] = __ldg(h4 + up8 + (c + 32) / 8 + i);
             }
           }
           tc_wait_ld();
+          stage_wait(std::integral_constant<int, 0>{});
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hc[q]);
-            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&hc[4 + q]);
+          for (int qq = 0; qq < 4; ++qq) {
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hc[qq]);
+            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&hc[4 + qq]);
             float dg[8], du[8], ah[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -592,7 +658,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
               for (int h = 0; h < 2; ++h) {
                 const float g = h ? gf.y : gf.x;
                 const float u = h ? uf.y : uf.x;
-                const float dap = __uint_as_float(a[8 * q + 2 * i + h]);
+                const float dap = __uint_as_float(a[8 * qq + 2 * i + h]);
                 const float sg = sigmoidf_(g);
                 const float silu = g * sg;
                 const float A = silu * u;
@@ -603,41 +669,19 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
                 ah[2 * i + h] = s * A;
               }
             }
-            uint4 w;
-            w.x = pack_bf16x2(dg[0], dg[1]);
-            w.y = pack_bf16x2(dg[2], dg[3]);
-            w.z = pack_bf16x2(dg[4], dg[5]);
-            w.w = pack_bf16x2(dg[6], dg[7]);
-            dg4[c / 8 + q] = w;
-            w.x = pack_bf16x2(du[0], du[1]);
-            w.y = pack_bf16x2(du[2], du[3]);
-            w.z = pack_bf16x2(du[4], du[5]);
-            w.w = pack_bf16x2(du[6], du[7]);
-            dg4[up8 + c / 8 + q] = w;
-            w.x = pack_bf16x2(ah[0], ah[1]);
-            w.y = pack_bf16x2(ah[2], ah[3]);
-            w.z = pack_bf16x2(ah[4], ah[5]);
-            w.w = pack_bf16x2(ah[6], ah[7]);
-            ah4[c / 8 + q] = w;
+            st_shared_v4(stg + sw64(lane, qq), pack8f(dg));
+            st_shared_v4(stg + kStoreBuf + sw64(lane, qq), pack8f(du));
+            st_shared_v4(stg + 2 * kStoreBuf + sw64(lane, qq), pack8f(ah));
+          }
+          stage_publish();
+          if (lane == 0) {
+            tma_store_2d(&p.tmC0, stg, t.n0 + c, row0);
+            tma_store_2d(&p.tmC0, stg + kStoreBuf, p.n + t.n0 + c, row0);
+            tma_store_2d(&p.tmC1, stg + 2 * kStoreBuf, t.n0 + c, row0);
+            bulk_commit();
           }
         }
         p.outf[(size_t)r * p.num_n_tiles + t.nt] = dsum;
-      } else if constexpr (KT::kGroupedK) {
-        const int M = (KIND == G_DW1) ? p.d : p.n;
-        const int N = (KIND == G_DW1) ? 2 * p.n : p.d;
-        const int m = t.m0 + rloc;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t a[32];
-          tmem_ld32(tacc + c, a);
-          tc_wait_ld();
-          if (m < M) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
-            store_row32_bf16(p.out0 + ((size_t)t.e * M + m) * N + t.n0 + c, v);
-          }
-        }
       } else {  // G_DWR
         const int m = t.m0 + rloc;
 #pragma unroll 1
@@ -663,6 +707,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       mbar_arrive(smem_u32(&acc_empty[b]));
       ++tcount;
     }
+    if (lane == 0) bulk_wait_all();  // stores finished before the CTA exits
   } else if constexpr (KT::kGather) {
     // ---------------- gather producers (warps 6-9): cp.async rows into the swizzled ring
     const int gt = threadIdx.x - 192;  // 0..127

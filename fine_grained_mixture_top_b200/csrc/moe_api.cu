@@ -8,7 +8,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "moe_internal.h"
 
 using namespace moe;
@@ -69,17 +69,22 @@ bool get_encode() {
   return true;
 }
 
-// 2-D bf16 row-major tensor [rows, cols], box [box_rows, box_cols], 128B swizzle.
+// 2-D bf16 row-major tensor [rows, cols], box [box_rows, box_cols]; operand
+// loads use the 128-byte swizzle, epilogue stores 32 x 32 boxes with the
+// 64-byte swizzle.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-               uint32_t box_rows) {
+               uint32_t box_rows, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+bool make_store_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return make_tmap(m, base, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // ----------------------------------------------------------------- shapes
@@ -404,6 +409,8 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.num_n_tiles = p.n / (p.bn_up / 2);
     g.out0 = static_cast<__nv_bfloat16*>(H);
     g.out1 = w.A;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, H, (uint64_t)p.R_max, (uint64_t)2 * p.n));
+    MOE_TRY_MAP(make_store_map(&g.tmC1, w.A, (uint64_t)p.R_max, (uint64_t)p.n));
     ProfScope ps(st, "up_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -414,6 +421,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     MOE_TRY_MAP(make_tmap(&g.tmB, W2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 64));
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "down_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -460,6 +468,8 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.out0 = w.dH;
     g.out1 = w.Ahat;
     g.outf = w.dS_part;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n));
+    MOE_TRY_MAP(make_store_map(&g.tmC1, w.Ahat, (uint64_t)p.R_max, (uint64_t)p.n));
     ProfScope ps(st, "dh_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -472,6 +482,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.n, 128);
     g.num_n_tiles = p.d / p.bn_dw2;
     g.out0 = static_cast<__nv_bfloat16*>(dW2);
+    MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
@@ -483,6 +494,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
     g.num_n_tiles = p.d / p.bn_dxt;
     g.out0 = w.dXt;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "dxt_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -495,6 +507,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.d, 128);
     g.num_n_tiles = 2 * p.n / p.bn_dw1;
     g.out0 = static_cast<__nv_bfloat16*>(dW1);
+    MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
