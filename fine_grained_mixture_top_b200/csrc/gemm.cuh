@@ -60,6 +60,8 @@ struct GemmParams {
   const __nv_bfloat16* hin;
   float* outf;
   const float* bias;
+  int* sched;                // weight-gradient kinds: zeroed tile counter of the dynamic scheduler
+  const int* expert_order;   // weight-gradient kinds: experts by descending token count
 };
 
 template <int KIND>
@@ -80,6 +82,7 @@ constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
 constexpr int kStageBudget = 200 * 1024;
 constexpr int kRtrGroup = 4;  // router logits: k-blocks per promoted hi-part group
 constexpr int kStoreBuf = 2048;  // one epilogue staging buffer: 32 rows x 32 bf16
+constexpr int kTileQ = 4;        // depth of the dynamic scheduler's tile queue
 
 template <int BN>
 struct GemmShape {
@@ -130,8 +133,9 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
     t.nkb = K / kBK;
   } else if constexpr (KT::kGroupedK) {
     const int per_e = p.num_m_tiles * p.num_n_tiles;
-    t.e = tile / per_e;
-    const int rem = tile - t.e * per_e;
+    const int ei = tile / per_e;
+    t.e = p.expert_order ? __ldg(p.expert_order + ei) : ei;  // largest experts first
+    const int rem = tile - ei * per_e;
     t.mt = rem / p.num_n_tiles;
     t.nt = rem - t.mt * p.num_n_tiles;
     t.m0 = t.mt * kBM;
@@ -286,8 +290,11 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
   uint64_t* acc_empty = bars + 2 * S + 2;
   uint64_t* hi_full = bars + 2 * S + 4;   // router logits: promoted hi-part groups
   uint64_t* hi_empty = bars + 2 * S + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 9);
+  uint64_t* tq_full = bars + 2 * S + 8;   // dynamic scheduler: tile queue
+  uint64_t* tq_empty = bars + 2 * S + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 17);
+  volatile int* tq_slots = reinterpret_cast<volatile int*>(bars + 2 * S + 18);  // [kTileQ]
   // the router-logit kind keeps one tile buffer of 256 columns: [hi_a | hi_b | mid | lo]
   constexpr int kTmemCols = (KIND == G_RTR) ? 256 : SH::kTmemCols;
 
@@ -304,6 +311,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       mbar_init(&acc_empty[b], 128);
       mbar_init(&hi_full[b], 1);
       mbar_init(&hi_empty[b], 128);
+    }
+    for (int b = 0; b < kTileQ; ++b) {
+      mbar_init(&tq_full[b], 1);
+      mbar_init(&tq_empty[b], KT::kGather ? 9 : 5);  // consumer warps: MMA, 4 epilogue, (4 gather)
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -323,12 +334,50 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
 
   const int num_tiles = gemm_num_tiles<KIND, BN>(p);
 
+  // Tile order.  Static kinds walk tiles round-robin.  The weight-gradient
+  // kinds, whose tiles differ in length with the expert's token count, take
+  // tiles dynamically: the TMA thread draws the next tile from a global
+  // counter and hands it to the other roles through a shared-memory queue.
+  constexpr bool kDyn = KT::kGroupedK;
+  auto produce_tile = [&](int i, bool& good) -> int {
+    if constexpr (kDyn) {
+      const int tile = i == 0 ? (int)blockIdx.x : atomicAdd(p.sched, 1) + (int)gridDim.x;
+      const int slot = i % kTileQ;
+      if (!mbar_wait(smem_u32(&tq_empty[slot]), ((i / kTileQ) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 10)) {
+        good = false;
+        return num_tiles;
+      }
+      tq_slots[slot] = tile;
+      mbar_arrive(smem_u32(&tq_full[slot]));
+      return tile;
+    } else {
+      return (int)blockIdx.x + i * (int)gridDim.x;
+    }
+  };
+  auto consume_tile = [&](int i, bool& good) -> int {
+    if constexpr (kDyn) {
+      const int slot = i % kTileQ;
+      if (!mbar_wait(smem_u32(&tq_full[slot]), (i / kTileQ) & 1, abort_flag, p.st, KIND * 16 + 11)) {
+        good = false;
+        return num_tiles;
+      }
+      const int tile = tq_slots[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tq_empty[slot]));
+      return tile;
+    } else {
+      return (int)blockIdx.x + i * (int)gridDim.x;
+    }
+  };
+
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int ti = 0; ok; ++ti) {
+        const int tile = produce_tile(ti, ok);
+        if (!ok || tile >= num_tiles) break;
         const TileInfo t = gemm_tile<KIND, BN>(p, tile);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
@@ -351,7 +400,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     constexpr uint32_t kIdescMl = idesc_bf16_f32(128, KT::kAMN, KT::kBMN);
     int it = 0, tcount = 0, hg = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int ti = 0; ok; ++ti) {
+      const int tile = consume_tile(ti, ok);
+      if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (!mbar_wait(smem_u32(&acc_empty[0]), (tcount & 1) ^ 1, abort_flag, p.st, KIND * 16 + 7)) {
         ok = false;
@@ -402,7 +453,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     // ---------------- MMA issuer
     int it = 0, tcount = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int ti = 0; ok; ++ti) {
+      const int tile = consume_tile(ti, ok);
+      if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (t.nkb == 0) continue;
       const int b = tcount & 1;
@@ -447,7 +500,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
     int tcount = 0, hg = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int ti = 0; ok; ++ti) {
+      const int tile = consume_tile(ti, ok);
+      if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       float hs[64];
 #pragma unroll
@@ -519,7 +574,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       __syncwarp();
     };
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    bool ok = true;
+    for (int ti = 0; ok; ++ti) {
+      const int tile = consume_tile(ti, ok);
+      if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       const int row0 = t.m0 + q * 32;  // first output row of this warp's slice
       if constexpr (KT::kGroupedK) {
@@ -716,7 +774,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     int it = 0;
     int pending = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int ti = 0; ok; ++ti) {
+      const int tile = consume_tile(ti, ok);
+      if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if constexpr (KIND == G_UP || KIND == G_DH) {
         // A tile = 128 gathered rows x 64 columns; this thread: lines line0 + 16 j
@@ -792,6 +852,17 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
             mbar_arrive(smem_u32(&full[(it - kLag) % S]));
           } else {
             ++pending;
+          }
+        }
+        if constexpr (kDyn) {
+          // Publish the tile's last k-blocks before taking the next tile from
+          // the queue: a stage held back across tiles would make the MMA wait
+          // on a tile the producer cannot publish while the queue is full.
+          if (ok && pending > 0) {
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&full[(it - k) % S]));
+            pending = 0;
           }
         }
       }

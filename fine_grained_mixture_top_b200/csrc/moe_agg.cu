@@ -205,6 +205,27 @@ cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pa
   return cudaGetLastError();
 }
 
+// Experts sorted by descending token count (ties: lower index first); the
+// weight-gradient GEMMs take their tiles in this order so that the longest
+// tiles start first.
+__global__ void __launch_bounds__(1024) expert_order_kernel(int E, const int* __restrict__ counts,
+                                                            int* __restrict__ order) {
+  __shared__ int c[1024];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) c[e] = counts[e];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int ce = c[e];
+    int rank = 0;
+    for (int j = 0; j < E; ++j) rank += (c[j] > ce) || (c[j] == ce && j < e);
+    order[rank] = e;
+  }
+}
+
+cudaError_t launch_expert_order(int E, const int* counts, int* order, cudaStream_t s) {
+  expert_order_kernel<<<1, 1024, 0, s>>>(E, counts, order);
+  return cudaGetLastError();
+}
+
 // Failure-detection self test: one thread waits on an mbarrier that nothing
 // will ever complete, through the same bounded wait the GEMM kernels use, and
 // must come back with ST_TIMEOUT recorded in the status word.

@@ -185,6 +185,7 @@ size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
 struct BwdWs {
   __nv_bfloat16 *dH, *Ahat, *dXt, *dz_split;
   float *dS_part, *dz_pair, *WrT, *dWr_part;
+  int *sched, *expert_order;
 };
 size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   Carve c{static_cast<char*>(ws)};
@@ -196,6 +197,8 @@ size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   w->dz_pair = c.take<float>((size_t)p.P_max);
   w->WrT = c.take<float>((size_t)p.E * p.d);
   w->dWr_part = c.take<float>((size_t)p.ksplit * p.d * p.Epad);
+  w->sched = c.take<int>(16);
+  w->expert_order = c.take<int>((size_t)p.E);
   return c.off;
 }
 
@@ -456,6 +459,13 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
   const int64_t mtiles = p.R_max / kTile;
   const __nv_bfloat16* dOb = static_cast<const __nv_bfloat16*>(dO);
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  // dynamic-scheduler counters of the weight-gradient GEMMs, and the expert
+  // order (largest first) in which they take their tiles
+  MOE_TRY_CUDA(cudaMemsetAsync(w.sched, 0, 16 * sizeof(int), st));
+  {
+    ProfScope ps(st, "expert_order");
+    MOE_TRY_CUDA(launch_expert_order(p.E, rt->counts, w.expert_order, st));
+  }
 
   // dH kernel: dA' = dO[tok] W2[e]^T; epilogue: H -> A, dS partials, dSwiGLU, A_hat
   {
@@ -482,6 +492,8 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.n, 128);
     g.num_n_tiles = p.d / p.bn_dw2;
     g.out0 = static_cast<__nv_bfloat16*>(dW2);
+    g.sched = w.sched + 0;
+    g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, g,
@@ -507,6 +519,8 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.num_m_tiles = (int)cdiv(p.d, 128);
     g.num_n_tiles = 2 * p.n / p.bn_dw1;
     g.out0 = static_cast<__nv_bfloat16*>(dW1);
+    g.sched = w.sched + 1;
+    g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, g,

@@ -73,5 +73,6 @@ cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pa
                                  const __nv_bfloat16* dXt, const float* dz_pair, const float* WrT, int router_grad,
                                  __nv_bfloat16* dX, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
+cudaError_t launch_expert_order(int E, const int* counts, int* order, cudaStream_t s);
 
 }  // namespace moe
