@@ -244,6 +244,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     cfg = CONFIGS[args.config]
+    if args.config != "7b":
+        workload = (f"{args.config} MoE layer fwd+bwd: T={cfg.T}, d={cfg.d}, E={cfg.E}, n={cfg.n}, "
+                    f"top-{cfg.K}, SwiGLU, router bias {cfg.bias}, rounding mode {cfg.round_mode}")
+    else:
+        workload = WORKLOAD
     inp = make_inputs(cfg, dev, rank=rank)
     layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=cfg.round_mode, router_grad=1,
                          seed=cfg.seed, device=dev)
@@ -390,10 +395,11 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
+            "config": {"workload": workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
                        "router_bias": cfg.bias, "round_mode": cfg.round_mode,
                        "parallelism": f"dp{world}" + (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else ""),
-                       "l2": "inputs larger than L2 (X+dO+W1+W2 = 402 MB per step, working set ~2 GB)"},
+                       "l2": "inputs larger than L2 (%d MB of X, dO, W1, W2 per step)" % (
+                           (4 * cfg.T * cfg.d + 6 * cfg.E * cfg.d * cfg.n) // 2**20)},
             "tokens_per_s": round(cfg.T * world / (ms_step * 1e-3), 1),
             "pct_of_tensor_peak": round(100 * value / world / tensor_peak, 2),
             "roofline": roof,

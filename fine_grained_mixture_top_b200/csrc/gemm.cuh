@@ -248,7 +248,7 @@ __device__ __forceinline__ void zero32(float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = 0.f;
 }
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 // Epilogue staging: a 32-row x 32-column bf16 box laid out with the 64-byte
 // swizzle the output tensor maps use; thread `row` writes its row.

@@ -199,20 +199,32 @@ __global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
   }
 }
 
-// One block: per-expert counts, 128-padded segment offsets, absolute chunk
-// bases, the tile -> expert list, and the padding rows (token -1, gate 0).
-__global__ void __launch_bounds__(1024) scan_kernel(RouteArgs a) {
-  __shared__ int sh[33];
-  for (int e = threadIdx.x; e < a.E; e += 1024) {
-    int run = 0;
-    for (int c = 0; c < a.nchunks; ++c) {
-      const int h = a.hist[(size_t)c * a.E + e];
-      a.hist[(size_t)c * a.E + e] = run;
-      run += h;
+// Per expert (one warp each, many blocks): exclusive scan over the chunks of
+// its per-chunk counts (chunk bases relative to the expert's segment) and
+// the expert's total count.
+__global__ void __launch_bounds__(256) chunk_scan_kernel(RouteArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  if (e >= a.E) return;
+  int carry = 0;
+  for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
+    const int c = c0 + lane;
+    const int h = c < a.nchunks ? a.hist[(size_t)c * a.E + e] : 0;
+    int x = h;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    a.counts[e] = run;
+    if (c < a.nchunks) a.hist[(size_t)c * a.E + e] = carry + x - h;
+    carry += __shfl_sync(0xffffffffu, x, 31);
   }
-  __syncthreads();
+  if (lane == 0) a.counts[e] = carry;
+}
+
+// One block: 128-padded segment offsets (exclusive scan over experts).
+__global__ void __launch_bounds__(1024) offsets_kernel(RouteArgs a) {
+  __shared__ int sh[33];
   int carry = 0;
   for (int e0 = 0; e0 < a.E; e0 += 1024) {
     const int e = e0 + threadIdx.x;
@@ -223,16 +235,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(RouteArgs a) {
     carry += total;
   }
   if (threadIdx.x == 0) a.offsets[a.E] = carry;
-  __syncthreads();
-  for (int e = threadIdx.x; e < a.E; e += 1024) {
-    const int base = a.offsets[e];
-    for (int c = 0; c < a.nchunks; ++c) a.hist[(size_t)c * a.E + e] += base;
-    const int end = a.offsets[e + 1];
-    for (int tt = base / kTile; tt < end / kTile; ++tt) a.tile_expert[tt] = e;
-    for (int r = base + a.counts[e]; r < end; ++r) {
-      a.row_tok[r] = -1;
-      a.row_gate[r] = 0.f;
-    }
+}
+
+// Per expert (one warp each): the tile -> expert list and the padding rows
+// (token -1, gate 0) of its segment.
+__global__ void __launch_bounds__(256) segment_fill_kernel(RouteArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  if (e >= a.E) return;
+  const int base = a.offsets[e];
+  const int end = a.offsets[e + 1];
+  for (int tt = base / kTile + lane; tt < end / kTile; tt += 32) a.tile_expert[tt] = e;
+  for (int r = base + a.counts[e] + lane; r < end; r += 32) {
+    a.row_tok[r] = -1;
+    a.row_gate[r] = 0.f;
   }
 }
 
@@ -241,7 +257,8 @@ __global__ void scatter_kernel(RouteArgs a) {
   if (t >= a.T) return;
   const int* base = a.hist + (size_t)(t / kChunk) * a.E;
   for (int p = a.tok_ptr[t]; p < a.tok_ptr[t + 1]; ++p) {
-    const int row = base[a.pair_expert[p]] + a.local_rank[p];
+    const int e = a.pair_expert[p];
+    const int row = a.offsets[e] + base[e] + a.local_rank[p];
     a.row_tok[row] = t;
     a.row_gate[row] = a.pair_gate[p];
     a.pair_row[p] = row;
@@ -253,9 +270,18 @@ cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s) {
     ProfScope ps(s, "permute_rank");
     rank_kernel<<<a.nchunks, kChunk, (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s>>>(a);
   }
+  const int eb = (a.E + 7) / 8;
   {
-    ProfScope ps(s, "permute_scan");
-    scan_kernel<<<1, 1024, 0, s>>>(a);
+    ProfScope ps(s, "permute_chunk_scan");
+    chunk_scan_kernel<<<eb, 256, 0, s>>>(a);
+  }
+  {
+    ProfScope ps(s, "permute_offsets");
+    offsets_kernel<<<1, 1024, 0, s>>>(a);
+  }
+  {
+    ProfScope ps(s, "permute_segment_fill");
+    segment_fill_kernel<<<eb, 256, 0, s>>>(a);
   }
   {
     ProfScope ps(s, "permute_scatter");

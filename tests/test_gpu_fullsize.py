@@ -13,7 +13,7 @@ import parity as P
 
 torch = pytest.importorskip("torch")
 
-FULL = ["7b", "qwen3", "dsv3"] + sorted(k for k in CONFIGS if k.startswith("sweep"))
+FULL = ["7b", "qwen3", "dsv3", "olmoe"] + sorted(k for k in CONFIGS if k.startswith("sweep"))
 
 
 def _budget(cfg):

@@ -74,6 +74,8 @@ CONFIGS: dict[str, MoEConfig] = {
     "qwen3": MoEConfig("qwen3", T=32768, d=2048, E=128, n=768, K=8, seed=2),
     # DeepSeek-V3-shaped layer, Zipf(1.1) expert popularity
     "dsv3": MoEConfig("dsv3", T=8192, d=7168, E=256, n=2048, K=8, bias="zipf", seed=4),
+    # OLMoE-shaped layer (the pages' runtime-breakdown workload), balanced router
+    "olmoe": MoEConfig("olmoe", T=32768, d=2048, E=64, n=1024, K=8, seed=5),
 }
 for _i, (_E, _n) in enumerate([(64, 512), (128, 256), (256, 128), (512, 64)]):
     for _tr in (False, True):
