@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="7b")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
@@ -118,7 +118,7 @@ class ClockSampler:
             os.close(fd)
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -270,6 +270,24 @@ def main():
     R = int(layer.routing["tok_ptr"][cfg.T].item())
     counts = layer.routing["counts"].cpu().tolist()
 
+    # ---- breakdown pass (outside the timed region): every launch bracketed
+    # by CUDA events on its stream, to find the dominant kernel and the launch
+    # count of a step.  Bracketing every launch costs about 0.2 ms per step, so
+    # the timed region below brackets only the dominant kernel.
+    n_breakdown = 3
+    moe.moe_profile_select(None)
+    moe.moe_profile_enable(True)
+    for _ in range(n_breakdown):
+        step()
+    torch.cuda.synchronize()
+    moe.moe_profile_enable(False)
+    recs_all = moe.moe_profile_records()
+    launches_per_step = len(recs_all) // n_breakdown
+    per = {}
+    for name, t in recs_all:
+        per.setdefault(name, []).append(t)
+    dom = max(per, key=lambda k: sum(per[k]))
+
     # ---- device-timed region
     vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
     smi_index = vis[local_rank].strip() if local_rank < len(vis) and vis[local_rank].strip().isdigit() else local_rank
@@ -278,7 +296,8 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.2)
+    moe.moe_profile_select(dom)
     moe.moe_profile_enable(True)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -288,6 +307,7 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     moe.moe_profile_enable(False)
+    moe.moe_profile_select(None)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
@@ -296,7 +316,7 @@ def main():
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
-    recs = moe.moe_profile_records()
+    recs_dom = moe.moe_profile_records()
     code, where = moe.moe_get_status()
     if code != 0:
         raise RuntimeError(f"device status {moe.status_str(code)} at {where}")
@@ -305,23 +325,23 @@ def main():
     ms_step = ms_max / args.steps
     value = flops_step * world / (ms_step * 1e-3) / 1e12
 
-    # ---- per-kernel breakdown and the dominant kernel's roofline
+    # ---- per-kernel breakdown (breakdown pass) and the dominant kernel's
+    # roofline (its launches inside the timed region)
     peaks, peak_src = load_peaks()
-    per = {}
-    for name, t in recs:
-        per.setdefault(name, []).append(t)
     work = kernel_work(cfg, R)
+    step_bd = sum(t for _, t in recs_all) / n_breakdown
     breakdown = {}
     for name, ts in per.items():
         avg = sum(ts) / len(ts)
-        entry = {"launches": len(ts), "avg_us": round(1e3 * avg, 2), "share": round(sum(ts) / max(ms, 1e-9), 4)}
+        entry = {"launches_per_step": len(ts) // n_breakdown, "avg_us": round(1e3 * avg, 2),
+                 "share": round(sum(ts) / n_breakdown / max(step_bd, 1e-9), 4)}
         if name in work:
             fl, by = work[name]
             entry["tflops"] = round(fl / (avg * 1e-3) / 1e12, 1)
             entry["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
         breakdown[name] = entry
-    dom = max(per, key=lambda k: sum(per[k]))
-    avg_dom = sum(per[dom]) / len(per[dom])
+    dom_times = [t for n, t in recs_dom if n == dom]
+    avg_dom = sum(dom_times) / len(dom_times)
     fl, by = work.get(dom, (0, 0))
     intensity = fl / max(by, 1)
     ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -404,7 +424,9 @@ def main():
             "pct_of_tensor_peak": round(100 * value / world / tensor_peak, 2),
             "roofline": roof,
             "kernels": breakdown,
-            "gpu_launches": len(recs),
+            "kernels_note": (f"per-kernel CUDA events from {n_breakdown} steps with every launch bracketed, run "
+                             "before the timed region; the timed region brackets only the dominant kernel"),
+            "gpu_launches": launches_per_step * args.steps,
             "routed_pairs": R,
             "expert_load": {"min": min(counts), "max": max(counts), "mean": sum(counts) / len(counts)},
             "clocks": clocks,

@@ -52,6 +52,7 @@ ProfRec g_prof[kProfCap];
 int g_prof_n = 0;        // records taken since the last enable
 int g_prof_created = 0;  // event pairs created so far (reused across enables)
 bool g_prof_on = false;
+char g_prof_only[64] = {0};  // when set, only launches of this name are recorded
 
 // ----------------------------------------------------------------- TMA encoding
 using EncodeFn = decltype(&cuTensorMapEncodeTiled);
@@ -277,6 +278,7 @@ inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(
 namespace moe {
 ProfScope::ProfScope(cudaStream_t s, const char* name) : stream(s) {
   if (!g_prof_on || g_prof_n >= kProfCap) return;
+  if (g_prof_only[0] && std::strcmp(g_prof_only, name) != 0) return;
   ProfRec& r = g_prof[g_prof_n];
   if (g_prof_n >= g_prof_created) {
     if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return;
@@ -596,6 +598,16 @@ moe_status moe_profile_enable(int32_t on) {
   if (on != 0 && on != 1) return MOE_ERR_INVALID_ARG;
   if (on) g_prof_n = 0;
   g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_select(const char* name) {
+  if (!name) {
+    g_prof_only[0] = 0;
+    return MOE_OK;
+  }
+  if (std::strlen(name) >= sizeof(g_prof_only)) return MOE_ERR_INVALID_ARG;
+  std::strcpy(g_prof_only, name);
   return MOE_OK;
 }
 

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.moe_selftest_wait_timeout.argtypes = [c_void_p, c_void_p]
         L.moe_profile_enable.argtypes = [c_int32]
         L.moe_profile_enable.restype = c_int32
+        L.moe_profile_select.argtypes = [ctypes.c_char_p]
+        L.moe_profile_select.restype = c_int32
         L.moe_profile_count.argtypes = []
         L.moe_profile_count.restype = c_int32
         L.moe_profile_read.argtypes = [c_int32, P(ctypes.c_char_p), P(ctypes.c_float)]
@@ -201,6 +203,11 @@ def moe_selftest_wait_timeout(flag, stream=None):
 
 def moe_profile_enable(on: bool):
     _check(lib().moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def moe_profile_select(name: str | None):
+    """Record only launches of `name` (None: record every launch)."""
+    _check(lib().moe_profile_select(None if name is None else name.encode()), "moe_profile_select")
 
 
 def moe_profile_records() -> list[tuple[str, float]]:

@@ -195,6 +195,10 @@ moe_status moe_selftest_wait_timeout(int32_t* waited_ok, void* stream);
  * thread-safe; meant for one benchmarking thread.
  */
 moe_status moe_profile_enable(int32_t on);
+/* Restrict recording to launches of one kernel name (as reported by
+ * moe_profile_read); NULL records every launch again.  Bracketing a single
+ * kernel keeps the event overhead out of the rest of the timed work. */
+moe_status moe_profile_select(const char* name);
 int32_t moe_profile_count(void);
 moe_status moe_profile_read(int32_t i, const char** name, float* ms);
 
