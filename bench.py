@@ -67,10 +67,11 @@ def kernel_work(cfg, R):
         "down_proj_gemm": (2 * R * d * n, 2 * R * n + 2 * E * d * n + 2 * R * d),
         "dh_gemm": (2 * R * d * n, 2 * T * d + 2 * E * d * n + 10 * R * n + 4 * R),
         "dw2_gemm": (2 * R * d * n, 2 * R * n + 2 * T * d + 2 * E * d * n),
-        "dxt_gemm": (4 * R * d * n, 4 * R * n + 4 * E * d * n + 2 * R * d),
+        # dX~ with the router path dz * Wr^T added in its epilogue
+        "dxt_gemm": (4 * R * d * n + 2 * R * d, 4 * R * n + 4 * E * d * n + 2 * R * d + 4 * E * d + 8 * R),
         "dw1_gemm": (4 * R * d * n, 2 * T * d + 4 * R * n + 4 * E * d * n),
         "aggregate_fwd": (2 * R * d, 2 * R * d + 2 * T * d + 8 * R),
-        "aggregate_bwd": (R * d, 2 * R * d + 2 * T * d + 12 * R),
+        "aggregate_bwd": (R * d, 2 * R * d + 2 * T * d + 4 * R + 4 * T),
         "router_logits_gemm": (2 * T * d * E, 2 * T * d + 4 * d * E + 4 * T * E),
         "router_dwr_gemm": (2 * T * d * E, 2 * T * d + 4 * T * E + 4 * d * E),
     }
@@ -340,6 +341,23 @@ def main():
             entry["tflops"] = round(fl / (avg * 1e-3) / 1e12, 1)
             entry["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
         breakdown[name] = entry
+    # forward / backward split of the breakdown pass (routing counted apart)
+    fwd_k = {"up_proj_gemm", "down_proj_gemm", "aggregate_fwd"}
+    route_us = fwd_us = bwd_us = 0.0
+    for name, ts in per.items():
+        us = 1e3 * sum(ts) / n_breakdown
+        if name.startswith(("router_split", "router_logits", "router_softmax", "permute_", "round_")):
+            route_us += us
+        elif name in fwd_k:
+            fwd_us += us
+        else:
+            bwd_us += us
+    fl_tok = cfg.T * cfg.K * cfg.d * cfg.n
+    phases = {"route_us": round(route_us, 1), "fwd_us": round(fwd_us, 1), "bwd_us": round(bwd_us, 1),
+              "fwd_tflops": round(6 * fl_tok / (fwd_us * 1e-6) / 1e12, 1),
+              "bwd_tflops": round(12 * fl_tok / (bwd_us * 1e-6) / 1e12, 1),
+              "note": "sums of the breakdown pass's kernel times; fwd = up-proj, down-proj, aggregation; "
+                      "route = router logits/softmax/top-K, permutation and token rounding"}
     dom_times = [t for n, t in recs_dom if n == dom]
     avg_dom = sum(dom_times) / len(dom_times)
     fl, by = work.get(dom, (0, 0))
@@ -423,6 +441,7 @@ def main():
             "tokens_per_s": round(cfg.T * world / (ms_step * 1e-3), 1),
             "pct_of_tensor_peak": round(100 * value / world / tensor_peak, 2),
             "roofline": roof,
+            "phases": phases,
             "kernels": breakdown,
             "kernels_note": (f"per-kernel CUDA events from {n_breakdown} steps with every launch bracketed, run "
                              "before the timed region; the timed region brackets only the dominant kernel"),

@@ -8,7 +8,7 @@
 //   DOWN Y_r = A_r W2[e]
 //   DH   dA'_r = dO[tok_r] W2[e]^T (gather on A); epilogue reloads H, forms
 //        dS partials, dSwiGLU -> dH, and A_hat = s_r * A_r
-//   DXT  dX~_r = dH_r W1[e]^T
+//   DXT  dX~_r = dH_r W1[e]^T (+ dz_r Wr[:, e]^T, the router path, when given)
 //   DW1  dW1[e] = X[tok]^T dH   (K runs over the rows of expert e; gather on A)
 //   DW2  dW2[e] = A_hat^T dO[tok] (K runs over the rows of expert e; gather on B)
 //   RTR  router logits X Wr with Wr split into three bf16 parts (hi+mid+lo)
@@ -62,6 +62,8 @@ struct GemmParams {
   const float* bias;
   int* sched;                // weight-gradient kinds: zeroed tile counter of the dynamic scheduler
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
+  const float* rvec;         // DXT router path: Wr transposed [E, d], or null
+  const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
 };
 
 template <int KIND>
@@ -75,27 +77,52 @@ struct KindTraits {
   static constexpr bool kBMN = !(KIND == G_DH || KIND == G_DXT);
 };
 
+// Epilogue configuration: EPI = 4 or 8 epilogue warps.  With 8, two warps
+// share each TMEM lane quarter and each takes half of the tile's columns;
+// that pays where the epilogue, not the main loop, bounds a tile (the dH
+// epilogue with its H reload and three outputs, or a short K loop).
+template <int KIND, int EPI>
+struct EpiCfg {
+  static_assert(EPI == 4 || EPI == 8, "4 or 8 epilogue warps");
+  static constexpr int kWarps = EPI;
+  static constexpr int kColSplit = EPI / 4;
+  // 2 KB staging buffers per warp: the up-proj and dH epilogues store three
+  // outputs per chunk; the others ring through 3 buffers (2 with 8 warps, so
+  // that the stage ring keeps its depth)
+  static constexpr int kBufs = (KIND == G_UP || KIND == G_DH) ? 3 : (EPI == 8 ? 2 : 3);
+  static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
+  // registers per thread for one resident block (multiple of 8, at most 255);
+  // 448-thread blocks stay under 61440 registers
+  static constexpr int kMaxRegRaw = (kThreads > 320 ? 61440 / kThreads : 65536 / kThreads) & ~7;
+  static constexpr int kMaxReg = kMaxRegRaw > 255 ? 255 : kMaxRegRaw;
+};
+
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
 constexpr int kStageBudget = 200 * 1024;
+constexpr int kSmemLimit = 227 * 1024;  // dynamic shared memory per block
 constexpr int kRtrGroup = 4;  // router logits: k-blocks per promoted hi-part group
 constexpr int kStoreBuf = 2048;  // one epilogue staging buffer: 32 rows x 32 bf16
 constexpr int kTileQ = 4;        // depth of the dynamic scheduler's tile queue
 
-template <int BN>
+template <int BN, int NBUF = 12>
 struct GemmShape {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStagesRaw = kStageBudget / kStageBytes;
+  static constexpr int kStoreBytes = NBUF * kStoreBuf;  // epilogue staging: NBUF buffers of 2 KB
+  static constexpr int kBudget = (kSmemLimit - 2048 - kStoreBytes) < kStageBudget
+                                     ? (kSmemLimit - 2048 - kStoreBytes) : kStageBudget;
+  static constexpr int kStagesRaw = kBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   // accumulator buffers start at power-of-two column offsets
   static constexpr int kAccStride = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);
   static constexpr int kTmemCols = 2 * kAccStride;
   static constexpr int kStoreOffset = kStages * kStageBytes;         // epilogue staging
-  static constexpr int kBarOffset = kStoreOffset + 4 * 3 * 2048;      // 4 warps x 3 buffers x 2 KB
+  static constexpr int kBarOffset = kStoreOffset + kStoreBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;  // barriers + alignment slack
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
 struct TileInfo {
@@ -269,11 +296,13 @@ __device__ __forceinline__ void stage_row32(uint32_t buf, int row, const float (
 }
 
 // ----------------------------------------------------------------- kernel
-template <int KIND, int BN>
-__global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
+template <int KIND, int BN, int EPI>
+__global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     moe_gemm_kernel(const __grid_constant__ GemmParams p) {
   using KT = KindTraits<KIND>;
-  using SH = GemmShape<BN>;
+  using EC = EpiCfg<KIND, EPI>;
+  using SH = GemmShape<BN, EPI * EC::kBufs>;
+  constexpr int kEpiEnd = 2 + EPI;  // epilogue warps are [2, kEpiEnd)
   constexpr int S = SH::kStages;
   constexpr int kLag = 1;  // a group is published one k-block after it was issued
   constexpr uint32_t kIdesc = idesc_bf16_f32(BN, KT::kAMN, KT::kBMN);
@@ -308,13 +337,13 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 32 * EPI);
       mbar_init(&hi_full[b], 1);
       mbar_init(&hi_empty[b], 128);
     }
     for (int b = 0; b < kTileQ; ++b) {
       mbar_init(&tq_full[b], 1);
-      mbar_init(&tq_empty[b], KT::kGather ? 9 : 5);  // consumer warps: MMA, 4 epilogue, (4 gather)
+      mbar_init(&tq_empty[b], 1 + EPI + (KT::kGather ? 4 : 0));  // consumer warps: MMA, epilogue, gather
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -493,7 +522,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       __syncwarp();
       ++tcount;
     }
-  } else if (warp < 6 && KIND == G_RTR) {
+  } else if (warp < kEpiEnd && KIND == G_RTR) {
     // ---------------- epilogue, router logits: z = sum of promoted hi groups + mid + lo + bias
     const int q = warp & 3;
     const int rloc = q * 32 + lane;
@@ -554,14 +583,17 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       mbar_arrive(smem_u32(&acc_empty[0]));
       ++tcount;
     }
-  } else if (warp < 6) {
+  } else if (warp < kEpiEnd) {
     // ---------------- epilogue: one accumulator row per thread.  bf16 results
     // are staged per warp in shared memory (32 rows x 32 columns) and written
-    // with TMA tensor stores; each warp owns three 2 KB staging buffers.
+    // with TMA tensor stores; each warp owns three 2 KB staging buffers.  A
+    // warp reaches TMEM lanes [32 (warp % 4), +32) only.
     const int q = warp & 3;
+    const int ew = warp - 2;
+    const int half = ew >> 2;  // column part of this warp (EC::kColSplit parts)
     const int rloc = q * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-    const uint32_t stg = base + SH::kStoreOffset + q * (3 * kStoreBuf);
+    const uint32_t stg = base + SH::kStoreOffset + ew * (EC::kBufs * kStoreBuf);
     int ring = 0;  // next staging buffer for one-output kinds
     // Make staging buffer(s) free: `pending` store groups may still be reading.
     auto stage_wait = [&](auto pending_tag) {
@@ -588,14 +620,14 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
             zero32(z);
             for (int c = 0; c < BN; c += 32) {
               const uint32_t buf = stg + ring * kStoreBuf;
-              stage_wait(std::integral_constant<int, 2>{});
+              stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
               stage_row32(buf, lane, z);
               stage_publish();
               if (lane == 0) {
                 tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
                 bulk_commit();
               }
-              ring = ring == 2 ? 0 : ring + 1;
+              ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
             }
           }
           continue;
@@ -610,14 +642,31 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
           continue;
         }
       }
-      // dH epilogue: start loading this row's first H chunk while the MMAs run
-      uint4 h_nx[8];
+      // dH epilogue: start loading this row's first 16 columns of H (gate
+      // and up) while the MMAs run
+      uint4 h_nx[4];
+      constexpr int kCols = BN / EC::kColSplit;  // accumulator columns of this warp
       if constexpr (KIND == G_DH) {
-        const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)(t.m0 + rloc) * (2 * p.n) + t.n0);
+        const uint4* h4 =
+            reinterpret_cast<const uint4*>(p.hin + (size_t)(t.m0 + rloc) * (2 * p.n) + t.n0 + half * kCols);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
           h_nx[i] = __ldg(h4 + i);
-          h_nx[4 + i] = __ldg(h4 + p.n / 8 + i);
+          h_nx[2 + i] = __ldg(h4 + p.n / 8 + i);
+        }
+      }
+      // dX~ router path: load this tile's first 32 values of row e of Wr^T
+      // (the same for every row of the tile) while the MMAs run
+      float rz = 0.f;
+      const float4* rv = nullptr;
+      float4 r_nx[8];
+      if constexpr (KIND == G_DXT) {
+        if (p.rvec) {
+          const int r = t.m0 + rloc;
+          rz = __ldg(p.row_tok + r) >= 0 ? __ldg(p.rscale + r) : 0.f;
+          rv = reinterpret_cast<const float4*>(p.rvec + (size_t)t.e * p.d + t.n0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) r_nx[i] = __ldg(rv + half * kCols / 4 + i);
         }
       }
       const int b = tcount & 1;
@@ -627,9 +676,11 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
       const uint32_t tacc = lane_addr + (uint32_t)(b * SH::kAccStride);
 
       if constexpr (KIND == G_UP) {
-        constexpr int BNh = BN / 2;
+        constexpr int BNh = BN / 2;  // gate columns [0, BNh), up columns [BNh, BN)
+        constexpr int kHalfCols = BNh / EC::kColSplit;
+        const int c0 = half * kHalfCols;
 #pragma unroll 1
-        for (int c = 0; c < BNh; c += 32) {
+        for (int c = c0; c < c0 + kHalfCols; c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(tacc + c, g);
           tmem_ld32(tacc + BNh + c, u);
@@ -661,85 +712,118 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
           live = row0 < M;
           orow = t.e * M + row0;
         }
+        const int c0 = half * kCols;  // this warp's columns: [c0, c0 + kCols)
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = c0; c < c0 + kCols; c += 32) {
           uint32_t a[32];
           tmem_ld32(tacc + c, a);
+          float4 r_cur[8];
+          if constexpr (KIND == G_DXT) {
+            if (rv) {  // router path: this chunk's Wr^T values; prefetch the next chunk's
+#pragma unroll
+              for (int i = 0; i < 8; ++i) r_cur[i] = r_nx[i];
+              if (c + 32 < c0 + kCols) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) r_nx[i] = __ldg(rv + (c + 32) / 4 + i);
+              }
+            }
+          }
           tc_wait_ld();
           if (live) {
             float v[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+            if constexpr (KIND == G_DXT) {
+              if (rv) {  // + dz_r * Wr[n0 + c + j, e]
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 w = r_cur[i];
+                  v[4 * i + 0] = fmaf(rz, w.x, v[4 * i + 0]);
+                  v[4 * i + 1] = fmaf(rz, w.y, v[4 * i + 1]);
+                  v[4 * i + 2] = fmaf(rz, w.z, v[4 * i + 2]);
+                  v[4 * i + 3] = fmaf(rz, w.w, v[4 * i + 3]);
+                }
+              }
+            }
             const uint32_t buf = stg + ring * kStoreBuf;
-            stage_wait(std::integral_constant<int, 2>{});
+            stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
             stage_row32(buf, lane, v);
             stage_publish();
             if (lane == 0) {
               tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
               bulk_commit();
             }
-            ring = ring == 2 ? 0 : ring + 1;
+            ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
           }
         }
       } else if constexpr (KIND == G_DH) {
+        // 16 columns at a time (register budget of 8 epilogue warps); the H
+        // values of the next 16 columns are loaded one step ahead
         const int r = t.m0 + rloc;
         const float s = __ldg(p.row_gate + r);
-        const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)r * (2 * p.n) + t.n0);
+        const int c0 = half * kCols;  // this warp's first column in the tile
+        const uint4* h4 = reinterpret_cast<const uint4*>(p.hin + (size_t)r * (2 * p.n) + t.n0 + c0);
         const int up8 = p.n / 8;  // offset of the up half in 16-byte units
         float dsum = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t a[32];
-          tmem_ld32(tacc + c, a);
-          uint4 hc[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) hc[i] = h_nx[i];
-          if (c + 32 < BN) {  // prefetch the next chunk of H
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              h_nx[i] = __ldg(h4 + (c + 32) / 8 + i);
-              h_nx[4 + i] = __ldg(h4 + up8 + (c + 32) / 8 + i);
-            }
-          }
-          tc_wait_ld();
+        for (int c = 0; c < kCols; c += 32) {
           stage_wait(std::integral_constant<int, 0>{});
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hc[qq]);
-            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&hc[4 + qq]);
-            float dg[8], du[8], ah[8];
+          for (int sub = 0; sub < 2; ++sub) {
+            const int cc = c + 16 * sub;
+            uint32_t a[16];
+            tmem_ld16(tacc + c0 + cc, a);
+            uint4 hc[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 gf = __bfloat1622float2(g2[i]);
-              const float2 uf = __bfloat1622float2(u2[i]);
+            for (int i = 0; i < 4; ++i) hc[i] = h_nx[i];
+            if (cc + 16 < kCols) {  // prefetch the next 16 columns of H
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const float g = h ? gf.y : gf.x;
-                const float u = h ? uf.y : uf.x;
-                const float dap = __uint_as_float(a[8 * qq + 2 * i + h]);
-                const float sg = sigmoidf_(g);
-                const float silu = g * sg;
-                const float A = silu * u;
-                dsum = fmaf(dap, A, dsum);
-                const float dA = s * dap;
-                dg[2 * i + h] = dA * u * sg * (1.0f + g * (1.0f - sg));
-                du[2 * i + h] = dA * silu;
-                ah[2 * i + h] = s * A;
+              for (int i = 0; i < 2; ++i) {
+                h_nx[i] = __ldg(h4 + (cc + 16) / 8 + i);
+                h_nx[2 + i] = __ldg(h4 + up8 + (cc + 16) / 8 + i);
               }
             }
-            st_shared_v4(stg + sw64(lane, qq), pack8f(dg));
-            st_shared_v4(stg + kStoreBuf + sw64(lane, qq), pack8f(du));
-            st_shared_v4(stg + 2 * kStoreBuf + sw64(lane, qq), pack8f(ah));
+            tc_wait_ld();
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&hc[qq]);
+              const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&hc[2 + qq]);
+              float dg[8], du[8], ah[8];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 gf = __bfloat1622float2(g2[i]);
+                const float2 uf = __bfloat1622float2(u2[i]);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const float g = h ? gf.y : gf.x;
+                  const float u = h ? uf.y : uf.x;
+                  const float dap = __uint_as_float(a[8 * qq + 2 * i + h]);
+                  const float sg = sigmoidf_(g);
+                  const float silu = g * sg;
+                  const float A = silu * u;
+                  dsum = fmaf(dap, A, dsum);
+                  const float dA = s * dap;
+                  dg[2 * i + h] = dA * u * sg * (1.0f + g * (1.0f - sg));
+                  du[2 * i + h] = dA * silu;
+                  ah[2 * i + h] = s * A;
+                }
+              }
+              const int q16 = 2 * sub + qq;  // 16-byte unit of the 32-column staging row
+              st_shared_v4(stg + sw64(lane, q16), pack8f(dg));
+              st_shared_v4(stg + kStoreBuf + sw64(lane, q16), pack8f(du));
+              st_shared_v4(stg + 2 * kStoreBuf + sw64(lane, q16), pack8f(ah));
+            }
           }
           stage_publish();
           if (lane == 0) {
-            tma_store_2d(&p.tmC0, stg, t.n0 + c, row0);
-            tma_store_2d(&p.tmC0, stg + kStoreBuf, p.n + t.n0 + c, row0);
-            tma_store_2d(&p.tmC1, stg + 2 * kStoreBuf, t.n0 + c, row0);
+            tma_store_2d(&p.tmC0, stg, t.n0 + c0 + c, row0);
+            tma_store_2d(&p.tmC0, stg + kStoreBuf, p.n + t.n0 + c0 + c, row0);
+            tma_store_2d(&p.tmC1, stg + 2 * kStoreBuf, t.n0 + c0 + c, row0);
             bulk_commit();
           }
         }
-        p.outf[(size_t)r * p.num_n_tiles + t.nt] = dsum;
+        // one dS partial per (N tile, column part)
+        p.outf[((size_t)r * p.num_n_tiles + t.nt) * EC::kColSplit + half] = dsum;
       } else {  // G_DWR
         const int m = t.m0 + rloc;
 #pragma unroll 1
@@ -767,8 +851,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kGather ? 320 : 192, 1)
     }
     if (lane == 0) bulk_wait_all();  // stores finished before the CTA exits
   } else if constexpr (KT::kGather) {
-    // ---------------- gather producers (warps 6-9): cp.async rows into the swizzled ring
-    const int gt = threadIdx.x - 192;  // 0..127
+    // ---------------- gather producers (the last 4 warps): cp.async rows into the swizzled ring
+    const int gt = threadIdx.x - 32 * kEpiEnd;  // 0..127
     const int chunk = gt & 7;
     const int line0 = gt >> 3;         // 0..15
     int it = 0;

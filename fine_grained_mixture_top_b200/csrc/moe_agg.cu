@@ -66,16 +66,17 @@ cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pa
 }
 
 // One warp per token.  dS_p = sum of the dH kernel's per-N-tile partials of
-// row(p); dz_p = s_p (dS_p - sum_j s_j dS_j).  Writes dz per pair (fp32) and
-// the token's dense dz row split into bf16 hi + lo parts for the tensor-core
-// dWr = X^T dz GEMM (layout: group g of 64 experts at columns [128 g, 128 g +
-// 128): hi parts then lo parts).
+// row(p); dz_p = s_p (dS_p - sum_j s_j dS_j).  Writes dz per padded row
+// (fp32, dz_row[row(p)]; padding rows are not written) for the dX~ epilogue,
+// and the token's dense dz row split into bf16 hi + lo parts for the
+// tensor-core dWr = X^T dz GEMM (layout: group g of 64 experts at columns
+// [128 g, 128 g + 128): hi parts then lo parts).
 __global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad, int nts,
                                                          const int* __restrict__ tok_ptr,
                                                          const int* __restrict__ pair_row,
                                                          const int* __restrict__ pair_expert,
                                                          const float* __restrict__ pair_gate,
-                                                         const float* __restrict__ dS_part, float* __restrict__ dz_pair,
+                                                         const float* __restrict__ dS_part, float* __restrict__ dz_row,
                                                          __nv_bfloat16* __restrict__ dz_split) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad,
     const float* part = dS_part + (size_t)pair_row[p] * nts;
     float ds = 0.f;
     for (int j = 0; j < nts; ++j) ds += part[j];
-    dz_pair[p] = ds;  // dS for now
+    dz_row[pair_row[p]] = ds;  // dS for now
     inner += pair_gate[p] * ds;
   }
 #pragma unroll
@@ -97,8 +98,9 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad,
   for (int c = lane; c < 2 * Epad; c += 32) row[c] = zero;
   __syncwarp();
   for (int p = p0 + lane; p < p1; p += 32) {
-    const float dz = pair_gate[p] * (dz_pair[p] - inner);
-    dz_pair[p] = dz;
+    const int r = pair_row[p];
+    const float dz = pair_gate[p] * (dz_row[r] - inner);
+    dz_row[r] = dz;
     const int e = pair_expert[p];
     const __nv_bfloat16 hi = __float2bfloat16_rn(dz);
     const __nv_bfloat16 lo = __float2bfloat16_rn(dz - __bfloat162float(hi));
@@ -110,9 +112,9 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad,
 
 cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
                               const int* pair_expert, const float* pair_gate, const float* dS_part,
-                              float* dz_pair, __nv_bfloat16* dz_split, cudaStream_t s) {
+                              float* dz_row, __nv_bfloat16* dz_split, cudaStream_t s) {
   router_bwd_kernel<<<(T + 7) / 8, 256, 0, s>>>(T, E, Epad, nts, tok_ptr, pair_row, pair_expert, pair_gate,
-                                                dS_part, dz_pair, dz_split);
+                                                dS_part, dz_row, dz_split);
   return cudaGetLastError();
 }
 
@@ -154,13 +156,11 @@ cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* p
   return cudaGetLastError();
 }
 
-// dX[t, 8c .. 8c+8) = sum_p dX~[row_p, ...] (+ sum_p dz_p WrT[e_p, ...])
+// dX[t, 8c .. 8c+8) = sum_p dX~[row_p, ...]  (the router path's dz_p Wr[:, e_p]
+// is already inside dX~, added by the dX~ GEMM's epilogue)
 __global__ void __launch_bounds__(256) aggregate_bwd_kernel(int T, int d8, const int* __restrict__ tok_ptr,
                                                             const int* __restrict__ pair_row,
-                                                            const int* __restrict__ pair_expert,
                                                             const uint4* __restrict__ dXt,
-                                                            const float* __restrict__ dz_pair,
-                                                            const float4* __restrict__ WrT, int router_grad,
                                                             uint4* __restrict__ dX) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)T * d8) return;
@@ -176,32 +176,15 @@ __global__ void __launch_bounds__(256) aggregate_bwd_kernel(int T, int d8, const
     for (int j = 0; j < 4; ++j) acc8(acc, v[j], 1.0f);
   }
   for (; p < p1; ++p) acc8(acc, __ldg(dXt + (size_t)__ldg(pair_row + p) * d8 + c), 1.0f);
-  if (router_grad) {
-    for (p = p0; p < p1; ++p) {
-      const float dz = __ldg(dz_pair + p);
-      const float4* w = WrT + ((size_t)__ldg(pair_expert + p) * d8 + c) * 2;
-      const float4 a = __ldg(w), b = __ldg(w + 1);
-      acc[0] = fmaf(dz, a.x, acc[0]);
-      acc[1] = fmaf(dz, a.y, acc[1]);
-      acc[2] = fmaf(dz, a.z, acc[2]);
-      acc[3] = fmaf(dz, a.w, acc[3]);
-      acc[4] = fmaf(dz, b.x, acc[4]);
-      acc[5] = fmaf(dz, b.y, acc[5]);
-      acc[6] = fmaf(dz, b.z, acc[6]);
-      acc[7] = fmaf(dz, b.w, acc[7]);
-    }
-  }
   dX[idx] = pack8(acc);
 }
 
-cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const int* pair_expert,
-                                 const __nv_bfloat16* dXt, const float* dz_pair, const float* WrT, int router_grad,
+cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const __nv_bfloat16* dXt,
                                  __nv_bfloat16* dX, cudaStream_t s) {
   const int d8 = d / 8;
   const int64_t n = (int64_t)T * d8;
   aggregate_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-      T, d8, tok_ptr, pair_row, pair_expert, reinterpret_cast<const uint4*>(dXt), dz_pair,
-      reinterpret_cast<const float4*>(WrT), router_grad, reinterpret_cast<uint4*>(dX));
+      T, d8, tok_ptr, pair_row, reinterpret_cast<const uint4*>(dXt), reinterpret_cast<uint4*>(dX));
   return cudaGetLastError();
 }
 

@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -94,7 +95,9 @@ struct Plan {
   int d, E, n, K, Epad, Ew, nchunks;
   int64_t P_max, R_max;
   int bn_up, bn_down, bn_dh, bn_dxt, bn_dw1, bn_dw2;
-  int nts;  // N tiles of the dH kernel (dS partials per row)
+  int nts;  // N tiles of the dH kernel
+  int nds;  // dS partials per row: N tiles x column parts of the dH epilogue
+  int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
   int ksplit, ksplit_rows;
 };
 
@@ -130,6 +133,13 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   p.bn_dw1 = ((2 * n) % 256 == 0) ? 256 : 128;
   p.bn_dw2 = p.bn_down;
   p.nts = n / p.bn_dh;
+  // Eight epilogue warps where the epilogue bounds a tile: the dH tile's
+  // epilogue (H reload, three outputs) outlasts a main loop of up to 24
+  // k-blocks (d <= 1536); the dX~ epilogue outlasts a main loop of up to 16
+  // k-blocks (2n <= 1024).  Longer main loops keep 4 warps and a deeper ring.
+  p.epi_dh = (d / 64 <= 24) ? 8 : 4;
+  p.epi_dxt = (2 * n / 64 <= 16) ? 8 : 4;
+  p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
   int64_t ks = std::max<int64_t>(1, cdiv(296, mn_tiles));
@@ -185,7 +195,7 @@ size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
 
 struct BwdWs {
   __nv_bfloat16 *dH, *Ahat, *dXt, *dz_split;
-  float *dS_part, *dz_pair, *WrT, *dWr_part;
+  float *dS_part, *dz_row, *WrT, *dWr_part;
   int *sched, *expert_order;
 };
 size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
@@ -193,9 +203,9 @@ size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   w->dH = c.take<__nv_bfloat16>((size_t)p.R_max * 2 * p.n);
   w->Ahat = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
   w->dXt = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
-  w->dS_part = c.take<float>((size_t)p.R_max * p.nts);
+  w->dS_part = c.take<float>((size_t)p.R_max * p.nds);
   w->dz_split = c.take<__nv_bfloat16>((size_t)p.T * 2 * p.Epad);
-  w->dz_pair = c.take<float>((size_t)p.P_max);
+  w->dz_row = c.take<float>((size_t)p.R_max);
   w->WrT = c.take<float>((size_t)p.E * p.d);
   w->dWr_part = c.take<float>((size_t)p.ksplit * p.d * p.Epad);
   w->sched = c.take<int>(16);
@@ -264,9 +274,20 @@ GemmParams base_params(const Plan& p, const moe_routing* rt, int* status) {
 
 inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, sms)); }
 
-#define MOE_TRY_CUDA(x)                         \
-  do {                                          \
-    if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
+// The last CUDA runtime error a call returned, with the source line that saw
+// it (read back through moe_last_error).
+thread_local char g_last_error[256] = "";
+
+moe_status cuda_failed(cudaError_t e, int line) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s (%s) at moe_api.cu:%d", cudaGetErrorName(e),
+                cudaGetErrorString(e), line);
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_TRY_CUDA(x)                                   \
+  do {                                                    \
+    const cudaError_t moe_e_ = (x);                       \
+    if (moe_e_ != cudaSuccess) return cuda_failed(moe_e_, __LINE__); \
   } while (0)
 #define MOE_TRY_MAP(x)                                 \
   do {                                                 \
@@ -345,7 +366,7 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
   g.bias = bias;
   {
     ProfScope ps(st, "router_logits_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_RTR, 192, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
   }
 
   {
@@ -417,7 +438,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     MOE_TRY_MAP(make_store_map(&g.tmC0, H, (uint64_t)p.R_max, (uint64_t)2 * p.n));
     MOE_TRY_MAP(make_store_map(&g.tmC1, w.A, (uint64_t)p.R_max, (uint64_t)p.n));
     ProfScope ps(st, "up_proj_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   // down-projection: Y = A W2[e]
   {
@@ -428,7 +449,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "down_proj_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   {
     ProfScope ps(st, "aggregate_fwd");
@@ -483,7 +504,19 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     MOE_TRY_MAP(make_store_map(&g.tmC0, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n));
     MOE_TRY_MAP(make_store_map(&g.tmC1, w.Ahat, (uint64_t)p.R_max, (uint64_t)p.n));
     ProfScope ps(st, "dh_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, p.epi_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  // router path, dz = s * (dS - sum_j s_j dS_j), before dX~ which consumes it
+  if (rg) {
+    {
+      ProfScope ps(st, "router_bwd");
+      MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nds, rt->tok_ptr, rt->pair_row, rt->pair_expert,
+                                     rt->pair_gate, w.dS_part, w.dz_row, w.dz_split, st));
+    }
+    {
+      ProfScope ps(st, "router_wr_transpose");
+      MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
+    }
   }
   // dW2[e] = A_hat^T dO[tok]
   {
@@ -498,7 +531,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, g,
+    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, 4, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
   // dX~ = dH W1[e]^T
@@ -508,9 +541,13 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
     g.num_n_tiles = p.d / p.bn_dxt;
     g.out0 = w.dXt;
+    if (rg) {
+      g.rvec = w.WrT;
+      g.rscale = w.dz_row;
+    }
     MOE_TRY_MAP(make_store_map(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "dxt_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   // dW1[e] = X[tok]^T dH
   {
@@ -525,19 +562,10 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, g,
+    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, 4, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
   if (rg) {
-    {
-      ProfScope ps(st, "router_bwd");
-      MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nts, rt->tok_ptr, rt->pair_row, rt->pair_expert,
-                                     rt->pair_gate, w.dS_part, w.dz_pair, w.dz_split, st));
-    }
-    {
-      ProfScope ps(st, "router_wr_transpose");
-      MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
-    }
     GemmParams g = base_params(p, rt, status);
     MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 64));
     MOE_TRY_MAP(make_tmap(&g.tmB, w.dz_split, (uint64_t)p.T, (uint64_t)2 * p.Epad, 64, 64));
@@ -548,7 +576,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     g.outf = w.dWr_part;
     {
       ProfScope ps(st, "router_dwr_gemm");
-      MOE_TRY_CUDA(launch_gemm(G_DWR, 128, g,
+      MOE_TRY_CUDA(launch_gemm(G_DWR, 128, 4, g,
                                grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st));
     }
     {
@@ -558,8 +586,8 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
   }
   {
     ProfScope ps(st, "aggregate_bwd");
-    MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_expert, w.dXt,
-                                      w.dz_pair, w.WrT, rg ? 1 : 0, static_cast<__nv_bfloat16*>(dX), st));
+    MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, w.dXt,
+                                      static_cast<__nv_bfloat16*>(dX), st));
   }
   return MOE_OK;
 }
@@ -619,6 +647,8 @@ moe_status moe_profile_read(int32_t i, const char** name, float* ms) {
   if (cudaEventElapsedTime(ms, g_prof[i].a, g_prof[i].b) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
+
+const char* moe_last_error(void) { return g_last_error; }
 
 const char* moe_status_str(moe_status s) {
   switch (s) {
@@ -706,7 +736,7 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* op
   g.num_n_tiles = p.Epad / 64;
   g.outf = rt->logits;
   g.bias = bias;
-  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
   MOE_TRY_CUDA(launch_softmax_topk(a, st));
   MOE_TRY_CUDA(launch_permute(a, st));
   return MOE_OK;

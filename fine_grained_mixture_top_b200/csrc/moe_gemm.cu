@@ -6,12 +6,12 @@
 
 namespace moe {
 
-template <int KIND, int BN>
+template <int KIND, int BN, int EPI>
 static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream) {
-  using KT = KindTraits<KIND>;
-  constexpr int smem = GemmShape<BN>::kSmemBytes;
-  constexpr int threads = KT::kGather ? 320 : 192;
-  auto fn = moe_gemm_kernel<KIND, BN>;
+  using EC = EpiCfg<KIND, EPI>;
+  constexpr int smem = GemmShape<BN, EPI * EC::kBufs>::kSmemBytes;
+  constexpr int threads = EC::kThreads;
+  auto fn = moe_gemm_kernel<KIND, BN, EPI>;
   static int configured_dev = -1;  // per-process; the library serves one device at a time
   int dev = 0;
   cudaGetDevice(&dev);
@@ -25,24 +25,29 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int kind, int bn, const GemmParams& p, int grid, cudaStream_t s) {
-#define MOE_CASE(K, B) \
-  if (kind == K && bn == B) return launch_one<K, B>(p, grid, s);
-  MOE_CASE(G_UP, 128)
-  MOE_CASE(G_UP, 256)
-  MOE_CASE(G_DOWN, 128)
-  MOE_CASE(G_DOWN, 256)
-  MOE_CASE(G_DH, 64)
-  MOE_CASE(G_DH, 128)
-  MOE_CASE(G_DH, 256)
-  MOE_CASE(G_DXT, 128)
-  MOE_CASE(G_DXT, 256)
-  MOE_CASE(G_DW1, 128)
-  MOE_CASE(G_DW1, 256)
-  MOE_CASE(G_DW2, 128)
-  MOE_CASE(G_DW2, 256)
-  MOE_CASE(G_RTR, 192)
-  MOE_CASE(G_DWR, 128)
+cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s) {
+#define MOE_CASE(K, B, W) \
+  if (kind == K && bn == B && epi == W) return launch_one<K, B, W>(p, grid, s);
+  MOE_CASE(G_UP, 128, 4)
+  MOE_CASE(G_UP, 256, 4)
+  MOE_CASE(G_DOWN, 128, 4)
+  MOE_CASE(G_DOWN, 256, 4)
+  MOE_CASE(G_DH, 64, 4)
+  MOE_CASE(G_DH, 128, 4)
+  MOE_CASE(G_DH, 256, 4)
+  MOE_CASE(G_DH, 64, 8)
+  MOE_CASE(G_DH, 128, 8)
+  MOE_CASE(G_DH, 256, 8)
+  MOE_CASE(G_DXT, 128, 4)
+  MOE_CASE(G_DXT, 256, 4)
+  MOE_CASE(G_DXT, 128, 8)
+  MOE_CASE(G_DXT, 256, 8)
+  MOE_CASE(G_DW1, 128, 4)
+  MOE_CASE(G_DW1, 256, 4)
+  MOE_CASE(G_DW2, 128, 4)
+  MOE_CASE(G_DW2, 256, 4)
+  MOE_CASE(G_RTR, 192, 4)
+  MOE_CASE(G_DWR, 128, 4)
 #undef MOE_CASE
   return cudaErrorInvalidValue;
 }
@@ -56,5 +61,7 @@ int gemm_smem_bytes(int bn) {
   }
   return 0;
 }
+
+
 
 }  // namespace moe

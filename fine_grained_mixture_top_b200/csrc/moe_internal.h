@@ -11,7 +11,8 @@ namespace moe {
 constexpr int kTile = 128;        // rows per expert tile (segments are padded to it)
 constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation
 
-cudaError_t launch_gemm(int kind, int bn, const GemmParams& p, int grid, cudaStream_t s);
+// epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
+cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
 
 // Per-kernel timing (moe_profile_enable): while on, each launch site brackets
 // its kernel with two CUDA events recorded on the launching stream.
@@ -66,11 +67,10 @@ cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pa
                                  const __nv_bfloat16* Y, __nv_bfloat16* O, cudaStream_t s);
 cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
                               const int* pair_expert, const float* pair_gate, const float* dS_part,
-                              float* dz_pair, __nv_bfloat16* dz_split, cudaStream_t s);
+                              float* dz_row, __nv_bfloat16* dz_split, cudaStream_t s);
 cudaError_t launch_transpose_wr(int d, int E, const float* Wr, float* WrT, cudaStream_t s);
 cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s);
-cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const int* pair_expert,
-                                 const __nv_bfloat16* dXt, const float* dz_pair, const float* WrT, int router_grad,
+cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const __nv_bfloat16* dXt,
                                  __nv_bfloat16* dX, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
 cudaError_t launch_expert_order(int E, const int* counts, int* order, cudaStream_t s);

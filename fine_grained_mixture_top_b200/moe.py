@@ -44,7 +44,10 @@ class MoeSizes(ctypes.Structure):
 
 class MoEError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {status_str(code)} ({code})")
+        msg = f"{what}: {status_str(code)} ({code})"
+        if code == MOE_ERR_CUDA:
+            msg += f": {last_error()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -85,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_read.restype = c_int32
         L.moe_status_str.argtypes = [c_int32]
         L.moe_status_str.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = []
+        L.moe_last_error.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
                   "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout"):
             getattr(L, f).restype = c_int32
@@ -94,6 +99,11 @@ def lib() -> ctypes.CDLL:
 
 def status_str(code: int) -> str:
     return lib().moe_status_str(int(code)).decode()
+
+
+def last_error() -> str:
+    """The CUDA runtime error behind this thread's most recent MOE_ERR_CUDA."""
+    return lib().moe_last_error().decode()
 
 
 def _check(code: int, what: str):

@@ -231,6 +231,12 @@ moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* opts, const v
 /* Static description of a status code. */
 const char* moe_status_str(moe_status s);
 
+/* The CUDA runtime error behind the calling thread's most recent
+ * MOE_ERR_CUDA: error name, message and the library source line that saw it.
+ * Empty if no call on this thread has failed that way.  The string is owned
+ * by the library and stays valid until the thread's next failing call. */
+const char* moe_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif
