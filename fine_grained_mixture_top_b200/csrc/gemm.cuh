@@ -107,21 +107,37 @@ constexpr int kRtrGroup = 4;  // router logits: k-blocks per promoted hi-part gr
 constexpr int kStoreBuf = 2048;  // one epilogue staging buffer: 32 rows x 32 bf16
 constexpr int kTileQ = 4;        // depth of the dynamic scheduler's tile queue
 
-template <int BN, int NBUF = 12>
+// Shared-memory rings of k-blocks (A slots of 16 KB, B slots of BN x 64
+// bf16).  The up-proj and dH kernels, whose A rows are gathered with cp.async
+// and published a few k-blocks after they are issued, give A and B separate
+// rings so that A's is deeper.  The other kinds keep one ring of (A, B)
+// stages with one barrier pair per stage: fewer barrier operations per
+// k-block where the main loop runs near the tensor-core rate.
+template <int KIND, int BN, int NBUF = 12>
 struct GemmShape {
+  using KT = KindTraits<KIND>;
+  static constexpr bool kSplit = (KIND == G_UP || KIND == G_DH);
   static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStoreBytes = NBUF * kStoreBuf;  // epilogue staging: NBUF buffers of 2 KB
   static constexpr int kBudget = (kSmemLimit - 2048 - kStoreBytes) < kStageBudget
                                      ? (kSmemLimit - 2048 - kStoreBytes) : kStageBudget;
-  static constexpr int kStagesRaw = kBudget / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int cap8(int x) { return x > 8 ? 8 : x; }
+  static constexpr int kStages = cap8(kBudget / (kABytes + kBBytes));  // one (A, B) ring
+  static constexpr int kSBs = (kBudget - 3 * kBBytes >= 5 * kABytes) ? (kBBytes >= 32768 ? 3 : 4) : 2;
+  static constexpr int kSA = kSplit ? cap8((kBudget - kSBs * kBBytes) / kABytes) : kStages;
+  static constexpr int kSB = kSplit ? kSBs : kStages;
+  // cp.async publication lag of a gathered operand (k-blocks in flight per
+  // thread = lag + 1; the MMA keeps ring - lag - 1 published k-blocks queued)
+  static constexpr int kLag = kSplit ? ((kSA - 3 > 3) ? 3 : ((kSA - 3 < 1) ? 1 : kSA - 3)) : 1;
+  static constexpr int kAOffset = 0;
+  static constexpr int kBOffset = kSA * kABytes;
   // accumulator buffers start at power-of-two column offsets
   static constexpr int kAccStride = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);
   static constexpr int kTmemCols = 2 * kAccStride;
-  static constexpr int kStoreOffset = kStages * kStageBytes;         // epilogue staging
+  static constexpr int kStoreOffset = kBOffset + kSB * kBBytes;  // epilogue staging
   static constexpr int kBarOffset = kStoreOffset + kStoreBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;  // barriers + alignment slack
+  static_assert(kSA >= 2 && kSB >= 2 && kSA <= 8 && kSB <= 8, "ring depths");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
@@ -199,48 +215,65 @@ __device__ __forceinline__ uint32_t sw128(int line, int chunk) {
 }
 
 // ----------------------------------------------------------------- producer
+// TMA loads of k-block kb: A into a_s (completing on bar_a), B into b_s
+// (completing on bar_b); an operand the gather warps stream is skipped.
 template <int KIND, int BN>
 __device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t, int kb, uint32_t a_s,
-                                          uint32_t b_s, uint32_t bar) {
+                                          uint32_t bar_a, uint32_t b_s, uint32_t bar_b) {
   const void* tA = &p.tmA;
   const void* tB = &p.tmB;
   const int k0 = kb * kBK;
+  constexpr int nb = BN / 64;
+  // one ring: a single arrive.expect_tx covers both operands' bytes
+  constexpr bool kOne = !GemmShape<KIND, BN>::kSplit;
+  constexpr uint32_t kTxA = (KIND == G_UP || KIND == G_DH || KIND == G_DW1) ? 0u : (uint32_t)kABytes;
+  constexpr uint32_t kTxB = (KIND == G_DW2) ? 0u : (uint32_t)(nb * kBoxBytes);
+  if constexpr (kOne) {
+    mbar_arrive_expect_tx(bar_a, kTxA + kTxB);
+    bar_b = bar_a;
+  }
+  auto expect_a = [&](uint32_t bytes) {
+    if constexpr (!kOne) mbar_arrive_expect_tx(bar_a, bytes);
+  };
+  auto expect_b = [&](uint32_t bytes) {
+    if constexpr (!kOne) mbar_arrive_expect_tx(bar_b, bytes);
+  };
   if constexpr (KIND == G_UP) {
-    constexpr int nb = BN / 64, half = nb / 2;
-    mbar_arrive_expect_tx(bar, nb * kBoxBytes);
+    constexpr int half = nb / 2;
+    expect_b(nb * kBoxBytes);
     for (int j = 0; j < nb; ++j) {
       const int col = (j < half) ? (t.n0 + 64 * j) : (p.n + t.n0 + 64 * (j - half));
-      tma_load_2d(b_s + j * kBoxBytes, tB, bar, col, t.e * p.d + k0);
+      tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, col, t.e * p.d + k0);
     }
   } else if constexpr (KIND == G_DOWN) {
-    constexpr int nb = BN / 64;
-    mbar_arrive_expect_tx(bar, kABytes + nb * kBoxBytes);
-    tma_load_2d(a_s, tA, bar, k0, t.m0);
-    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.e * p.n + k0);
+    expect_a(kABytes);
+    tma_load_2d(a_s, tA, bar_a, k0, t.m0);
+    expect_b(nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, t.n0 + 64 * j, t.e * p.n + k0);
   } else if constexpr (KIND == G_DH) {
-    mbar_arrive_expect_tx(bar, BN * 128);
-    tma_load_2d(b_s, tB, bar, k0, t.e * p.n + t.n0);
+    expect_b(BN * 128);
+    tma_load_2d(b_s, tB, bar_b, k0, t.e * p.n + t.n0);
   } else if constexpr (KIND == G_DXT) {
-    mbar_arrive_expect_tx(bar, kABytes + BN * 128);
-    tma_load_2d(a_s, tA, bar, k0, t.m0);
-    tma_load_2d(b_s, tB, bar, k0, t.e * p.d + t.n0);
+    expect_a(kABytes);
+    tma_load_2d(a_s, tA, bar_a, k0, t.m0);
+    expect_b(BN * 128);
+    tma_load_2d(b_s, tB, bar_b, k0, t.e * p.d + t.n0);
   } else if constexpr (KIND == G_DW1) {
-    constexpr int nb = BN / 64;
-    mbar_arrive_expect_tx(bar, nb * kBoxBytes);
-    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.krow0 + k0);
+    expect_b(nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, t.n0 + 64 * j, t.krow0 + k0);
   } else if constexpr (KIND == G_DW2) {
-    mbar_arrive_expect_tx(bar, 2 * kBoxBytes);
-    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar, t.m0 + 64 * h, t.krow0 + k0);
+    expect_a(2 * kBoxBytes);
+    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar_a, t.m0 + 64 * h, t.krow0 + k0);
   } else if constexpr (KIND == G_RTR) {
-    constexpr int nb = BN / 64;
-    mbar_arrive_expect_tx(bar, kABytes + nb * kBoxBytes);
-    tma_load_2d(a_s, tA, bar, k0, t.m0);
-    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, k0);
+    expect_a(kABytes);
+    tma_load_2d(a_s, tA, bar_a, k0, t.m0);
+    expect_b(nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, t.n0 + 64 * j, k0);
   } else {  // G_DWR
-    constexpr int nb = BN / 64;
-    mbar_arrive_expect_tx(bar, 2 * kBoxBytes + nb * kBoxBytes);
-    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar, t.m0 + 64 * h, t.krow0 + k0);
-    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar, t.n0 + 64 * j, t.krow0 + k0);
+    expect_a(2 * kBoxBytes);
+    for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar_a, t.m0 + 64 * h, t.krow0 + k0);
+    expect_b(nb * kBoxBytes);
+    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, t.n0 + 64 * j, t.krow0 + k0);
   }
 }
 
@@ -301,10 +334,12 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     moe_gemm_kernel(const __grid_constant__ GemmParams p) {
   using KT = KindTraits<KIND>;
   using EC = EpiCfg<KIND, EPI>;
-  using SH = GemmShape<BN, EPI * EC::kBufs>;
+  using SH = GemmShape<KIND, BN, EPI * EC::kBufs>;
   constexpr int kEpiEnd = 2 + EPI;  // epilogue warps are [2, kEpiEnd)
-  constexpr int S = SH::kStages;
-  constexpr int kLag = 1;  // a group is published one k-block after it was issued
+  constexpr bool kSplit = SH::kSplit;  // separate A and B rings
+  constexpr int SA = SH::kSA;      // A ring slots
+  constexpr int SB = SH::kSB;      // B ring slots
+  constexpr int kLag = SH::kLag;   // gathered k-blocks are published kLag k-blocks after issue
   constexpr uint32_t kIdesc = idesc_bf16_f32(BN, KT::kAMN, KT::kBMN);
 
   extern __shared__ uint8_t smem_raw[];
@@ -313,17 +348,21 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   uint8_t* smem = smem_raw + (base - raw);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SH::kBarOffset);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + S;
-  uint64_t* acc_full = bars + 2 * S;
-  uint64_t* acc_empty = bars + 2 * S + 2;
-  uint64_t* hi_full = bars + 2 * S + 4;   // router logits: promoted hi-part groups
-  uint64_t* hi_empty = bars + 2 * S + 6;
-  uint64_t* tq_full = bars + 2 * S + 8;   // dynamic scheduler: tile queue
-  uint64_t* tq_empty = bars + 2 * S + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 17);
-  volatile int* tq_slots = reinterpret_cast<volatile int*>(bars + 2 * S + 18);  // [kTileQ]
+  uint64_t* full_a = bars;         // [SA] A ring (the (A, B) ring without kSplit)
+  uint64_t* empty_a = bars + 8;
+  uint64_t* full_b = kSplit ? bars + 16 : full_a;  // [SB] B ring
+  uint64_t* empty_b = kSplit ? bars + 24 : empty_a;
+  uint64_t* acc_full = bars + 32;
+  uint64_t* acc_empty = bars + 34;
+  uint64_t* hi_full = bars + 36;   // router logits: promoted hi-part groups
+  uint64_t* hi_empty = bars + 38;
+  uint64_t* tq_full = bars + 40;   // dynamic scheduler: tile queue
+  uint64_t* tq_empty = bars + 44;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 48);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 49);
+  volatile int* tq_slots = reinterpret_cast<volatile int*>(bars + 50);  // [kTileQ]
+  auto a_slot = [&](int i) -> uint32_t { return base + SH::kAOffset + (uint32_t)(i * kABytes); };
+  auto b_slot = [&](int i) -> uint32_t { return base + SH::kBOffset + (uint32_t)(i * SH::kBBytes); };
   // the router-logit kind keeps one tile buffer of 256 columns: [hi_a | hi_b | mid | lo]
   constexpr int kTmemCols = (KIND == G_RTR) ? 256 : SH::kTmemCols;
 
@@ -331,9 +370,20 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1 + (KT::kGather ? 128 : 0));
-      mbar_init(&empty[s], 1);
+    if constexpr (kSplit) {  // A gathered (128 threads), B by the TMA thread
+      for (int s = 0; s < SA; ++s) {
+        mbar_init(&full_a[s], 128);
+        mbar_init(&empty_a[s], 1);
+      }
+      for (int s = 0; s < SB; ++s) {
+        mbar_init(&full_b[s], 1);
+        mbar_init(&empty_b[s], 1);
+      }
+    } else {  // the TMA thread (+ 128 gather threads)
+      for (int s = 0; s < SA; ++s) {
+        mbar_init(&full_a[s], 1 + (KT::kGather ? 128 : 0));
+        mbar_init(&empty_a[s], 1);
+      }
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -409,13 +459,19 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         if (!ok || tile >= num_tiles) break;
         const TileInfo t = gemm_tile<KIND, BN>(p, tile);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
-            ok = false;
-            break;
+          const int sa = it % SA, sb = it % SB;
+          if constexpr (!kSplit) {
+            if (!mbar_wait(smem_u32(&empty_a[sa]), ((it / SA) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
+              ok = false;
+              break;
+            }
+          } else {
+            if (!mbar_wait(smem_u32(&empty_b[sb]), ((it / SB) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 12)) {
+              ok = false;
+              break;
+            }
           }
-          const uint32_t a_s = base + s * SH::kStageBytes;
-          issue_tma<KIND, BN>(p, t, kb, a_s, a_s + kABytes, smem_u32(&full[s]));
+          issue_tma<KIND, BN>(p, t, kb, a_slot(sa), smem_u32(&full_a[sa]), b_slot(sb), smem_u32(&full_b[sb]));
         }
       }
     }
@@ -450,15 +506,16 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           }
           tc_fence_after();
         }
-        const int s = it % S;
-        if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)) {
+        const int sa = it % SA, sb = it % SB;
+        if (!mbar_wait(smem_u32(&full_a[sa]), (it / SA) & 1, abort_flag, p.st, KIND * 16 + 3) ||
+            (kSplit && !mbar_wait(smem_u32(&full_b[sb]), (it / SB) & 1, abort_flag, p.st, KIND * 16 + 13))) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_s = base + s * SH::kStageBytes;
-          const uint32_t b_s = a_s + kABytes;
+          const uint32_t a_s = a_slot(sa);
+          const uint32_t b_s = b_slot(sb);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(a_s + kk * 32, 16, 1024);
@@ -467,7 +524,8 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
             tc_mma_bf16(tmem_base + (uint32_t)(slot * 64), ad, bhi, kIdescHi, (first && kk == 0) ? 0u : 1u);
             tc_mma_bf16(tmem_base + 128u, ad, bml, kIdescMl, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(smem_u32(&empty[s]));
+          tc_commit(smem_u32(&empty_a[sa]));
+          if (kSplit) tc_commit(smem_u32(&empty_b[sb]));
           if (last) tc_commit(smem_u32(&hi_full[slot]));
         }
         __syncwarp();
@@ -496,15 +554,16 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(b * SH::kAccStride);
       for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-        const int s = it % S;
-        if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)) {
+        const int sa = it % SA, sb = it % SB;
+        if (!mbar_wait(smem_u32(&full_a[sa]), (it / SA) & 1, abort_flag, p.st, KIND * 16 + 3) ||
+            (kSplit && !mbar_wait(smem_u32(&full_b[sb]), (it / SB) & 1, abort_flag, p.st, KIND * 16 + 13))) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_s = base + s * SH::kStageBytes;
-          const uint32_t b_s = a_s + kABytes;
+          const uint32_t a_s = a_slot(sa);
+          const uint32_t b_s = b_slot(sb);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = KT::kAMN ? smem_desc_sw128(a_s + kk * 2048, kBoxBytes, 1024)
@@ -513,7 +572,8 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
                                          : smem_desc_sw128(b_s + kk * 32, 16, 1024);
             tc_mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(smem_u32(&empty[s]));
+          tc_commit(smem_u32(&empty_a[sa]));
+          if (kSplit) tc_commit(smem_u32(&empty_b[sb]));
         }
         __syncwarp();
       }
@@ -855,6 +915,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     const int gt = threadIdx.x - 32 * kEpiEnd;  // 0..127
     const int chunk = gt & 7;
     const int line0 = gt >> 3;         // 0..15
+    // the gathered operand's ring: A for up-proj, dH and dW1; B for dW2
+    // (dW1 and dW2 share one ring with the TMA operand)
+    constexpr int GS = KT::kAGather ? SA : SB;
+    uint64_t* g_full = KT::kAGather ? full_a : full_b;
+    uint64_t* g_empty = KT::kAGather ? empty_a : empty_b;
     int it = 0;
     int pending = 0;
     bool ok = true;
@@ -873,19 +938,19 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           nbytes[j] = tok < 0 ? 0u : 16u;
         }
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 5)) {
+          const int s = it % GS;
+          if (!mbar_wait(smem_u32(&g_empty[s]), ((it / GS) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 5)) {
             ok = false;
             break;
           }
-          const uint32_t a_s = base + s * SH::kStageBytes;
+          const uint32_t a_s = a_slot(s);
 #pragma unroll
           for (int j = 0; j < 8; ++j) cp_async_16(a_s + sw128(line0 + 16 * j, chunk), src[j] + kb * kBK, nbytes[j]);
           cp_async_commit();
           if (pending == kLag) {
             cp_async_wait<kLag>();
             fence_proxy_async_smem();
-            mbar_arrive(smem_u32(&full[(it - kLag) % S]));
+            mbar_arrive(smem_u32(&g_full[(it - kLag) % GS]));
           } else {
             ++pending;
           }
@@ -902,7 +967,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           for (int j = 0; j < 4; ++j)
             tk[q + 1][j] = q < t.nkb ? __ldg(p.row_tok + t.krow0 + q * kBK + line0 + 16 * j) : -1;
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
-          const int s = it % S;
+          const int s = it % GS;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             tk[0][j] = tk[1][j];
@@ -912,11 +977,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
 #pragma unroll
             for (int j = 0; j < 4; ++j) tk[2][j] = __ldg(p.row_tok + t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
           }
-          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
+          if (!mbar_wait(smem_u32(&g_empty[s]), ((it / GS) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
             ok = false;
             break;
           }
-          const uint32_t dst0 = base + s * SH::kStageBytes + (KIND == G_DW1 ? 0 : kABytes);
+          const uint32_t dst0 = KT::kAGather ? a_slot(s) : b_slot(s);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int i = line0 + 16 * j;
@@ -933,7 +998,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           if (pending == kLag) {
             cp_async_wait<kLag>();
             fence_proxy_async_smem();
-            mbar_arrive(smem_u32(&full[(it - kLag) % S]));
+            mbar_arrive(smem_u32(&g_full[(it - kLag) % GS]));
           } else {
             ++pending;
           }
@@ -945,7 +1010,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           if (ok && pending > 0) {
             cp_async_wait<0>();
             fence_proxy_async_smem();
-            for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&full[(it - k) % S]));
+            for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&g_full[(it - k) % GS]));
             pending = 0;
           }
         }
@@ -955,7 +1020,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     cp_async_wait<0>();
     fence_proxy_async_smem();
     if (ok) {
-      for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&full[(it - k) % S]));
+      for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&g_full[(it - k) % GS]));
     }
   }
 

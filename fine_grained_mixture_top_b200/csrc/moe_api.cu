@@ -135,8 +135,10 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   p.nts = n / p.bn_dh;
   // Eight epilogue warps where the epilogue bounds a tile: the dH tile's
   // epilogue (H reload, three outputs) outlasts a main loop of up to 24
-  // k-blocks (d <= 1536); the dX~ epilogue outlasts a main loop of up to 16
-  // k-blocks (2n <= 1024).  Longer main loops keep 4 warps and a deeper ring.
+  // k-blocks (d <= 1536); the dX~ epilogue (a 64 KB store per tile plus the
+  // router path) outlasts a main loop of up to 16 k-blocks (2n <= 1024).
+  // Longer main loops keep 4 warps.  (The down-proj kernel measured slower
+  // with 8: its short main loop is bound by the Y stores, not the epilogue.)
   p.epi_dh = (d / 64 <= 24) ? 8 : 4;
   p.epi_dxt = (2 * n / 64 <= 16) ? 8 : 4;
   p.nds = p.nts * (p.epi_dh / 4);

@@ -9,7 +9,7 @@ namespace moe {
 template <int KIND, int BN, int EPI>
 static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream) {
   using EC = EpiCfg<KIND, EPI>;
-  constexpr int smem = GemmShape<BN, EPI * EC::kBufs>::kSmemBytes;
+  constexpr int smem = GemmShape<KIND, BN, EPI * EC::kBufs>::kSmemBytes;
   constexpr int threads = EC::kThreads;
   auto fn = moe_gemm_kernel<KIND, BN, EPI>;
   static int configured_dev = -1;  // per-process; the library serves one device at a time
@@ -52,15 +52,6 @@ cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid
   return cudaErrorInvalidValue;
 }
 
-int gemm_smem_bytes(int bn) {
-  switch (bn) {
-    case 64: return GemmShape<64>::kSmemBytes;
-    case 128: return GemmShape<128>::kSmemBytes;
-    case 192: return GemmShape<192>::kSmemBytes;
-    case 256: return GemmShape<256>::kSmemBytes;
-  }
-  return 0;
-}
 
 
 

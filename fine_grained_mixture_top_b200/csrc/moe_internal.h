@@ -22,7 +22,6 @@ struct ProfScope {
   ProfScope(cudaStream_t s, const char* name);
   ~ProfScope();
 };
-int gemm_smem_bytes(int bn);
 
 // ---- routing (moe_route.cu)
 struct RouteArgs {
