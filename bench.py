@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--ref-sample-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--comm-sms", type=int, default=16,
+                    help="N>1: SMs left to NCCL while the gradient all-reduces overlap the backward "
+                         "(0: all-reduce after the step, no overlap)")
     return ap.parse_args()
 
 
@@ -241,6 +244,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    overlap = world > 1 and args.comm_sms > 0
+    if overlap:  # NCCL reads this when its communicator is created
+        os.environ.setdefault("NCCL_MAX_CTAS", str(args.comm_sms))
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
@@ -255,8 +261,15 @@ def main():
                          seed=cfg.seed, device=dev)
     X, Wr, b, W1, W2, dO = (inp[k] for k in ("X", "Wr", "bias", "W1", "W2", "dO"))
     stream = torch.cuda.current_stream()
+    if overlap:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        moe.moe_set_sm_budget(sms - args.comm_sms)
+        reducer = moe.OverlappedGradReduce(layer)
 
     def step():
+        if overlap:
+            reducer.step(X, Wr, b, W1, W2, dO)
+            return
         layer.step(X, Wr, b, W1, W2, dO)
         if world > 1:
             for g in (layer.dW1, layer.dW2, layer.dWr):
@@ -435,7 +448,9 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
                        "router_bias": cfg.bias, "round_mode": cfg.round_mode,
-                       "parallelism": f"dp{world}" + (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else ""),
+                       "parallelism": f"dp{world}" + ((" (NCCL all-reduce of dW2, dW1, dWr overlapping the backward, "
+                                                       f"{args.comm_sms} SMs left to NCCL)") if overlap else
+                                                      (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else "")),
                        "l2": "inputs larger than L2 (%d MB of X, dO, W1, W2 per step)" % (
                            (4 * cfg.T * cfg.d + 6 * cfg.E * cfg.d * cfg.n) // 2**20)},
             "tokens_per_s": round(cfg.T * world / (ms_step * 1e-3), 1),

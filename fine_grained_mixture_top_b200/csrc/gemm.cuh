@@ -232,6 +232,7 @@ __device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t
     mbar_arrive_expect_tx(bar_a, kTxA + kTxB);
     bar_b = bar_a;
   }
+  (void)bar_b;  // unused by the kinds whose B is gathered
   auto expect_a = [&](uint32_t bytes) {
     if constexpr (!kOne) mbar_arrive_expect_tx(bar_a, bytes);
   };

@@ -23,6 +23,7 @@ constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
 long long g_spin_limit = 1ll << 31;
+int g_sm_budget = 0;  // CTAs of a persistent GEMM at most (0: one per SM)
 std::mutex g_mu;
 
 bool device_state(int* dev_out, int** status_out, int* sms_out) {
@@ -39,7 +40,7 @@ bool device_state(int* dev_out, int** status_out, int* sms_out) {
   }
   *dev_out = dev;
   *status_out = g_status_ptr[dev];
-  *sms_out = g_num_sms[dev];
+  *sms_out = (g_sm_budget > 0 && g_sm_budget < g_num_sms[dev]) ? g_sm_budget : g_num_sms[dev];
   return true;
 }
 
@@ -166,6 +167,7 @@ struct Carve {
 struct RouteWs {
   __nv_bfloat16* Wr_split;
   float* logits;
+  int* sync;  // [1] blocks done, for the last-block offsets scan of the permutation
   int* hist;
   int* local_rank;
   uint32_t* member;
@@ -176,6 +178,7 @@ size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
   Carve c{static_cast<char*>(ws)};
   w->Wr_split = c.take<__nv_bfloat16>((size_t)p.d * 3 * p.Epad);
   w->logits = c.take<float>((size_t)p.T * p.E);
+  w->sync = c.take<int>(4);
   w->hist = c.take<int>((size_t)p.nchunks * p.E);
   w->local_rank = c.take<int>((size_t)p.P_max);
   w->member = c.take<uint32_t>((size_t)p.T * p.Ew);
@@ -250,6 +253,7 @@ RouteArgs route_args(const Plan& p, const moe_routing* rt, const RouteWs& w) {
   a.row_tok = rt->row_tok;
   a.row_gate = rt->row_gate;
   a.tile_expert = rt->tile_expert;
+  a.sync = w.sync;
   a.hist = w.hist;
   a.local_rank = w.local_rank;
   a.nchunks = p.nchunks;
@@ -272,6 +276,12 @@ GemmParams base_params(const Plan& p, const moe_routing* rt, int* status) {
   g.E = p.E;
   g.Epad = p.Epad;
   return g;
+}
+
+// Records event grad_ready[i] (a cudaEvent_t, may be null) on the stream.
+// Recording cannot fail on a valid event; a failure surfaces at the next sync.
+inline void record_ready(void* const* grad_ready, int i, cudaStream_t st) {
+  if (grad_ready && grad_ready[i]) cudaEventRecord(static_cast<cudaEvent_t>(grad_ready[i]), st);
 }
 
 inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, sms)); }
@@ -464,6 +474,13 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
 moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X, const float* Wr,
                         const void* W1, const void* W2, const moe_routing* rt, const void* H, void* dX, void* dW1,
                         void* dW2, float* dWr, void* ws, size_t ws_bytes, void* stream) {
+  return moe_backward_ev(dims, opts, dO, X, Wr, W1, W2, rt, H, dX, dW1, dW2, dWr, ws, ws_bytes, nullptr, stream);
+}
+
+moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X, const float* Wr,
+                           const void* W1, const void* W2, const moe_routing* rt, const void* H, void* dX,
+                           void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes, void* const* grad_ready,
+                           void* stream) {
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -536,21 +553,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, 4, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
-  // dX~ = dH W1[e]^T
-  {
-    GemmParams g = base_params(p, rt, status);
-    MOE_TRY_MAP(make_tmap(&g.tmA, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n, 64, 128));
-    MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
-    g.num_n_tiles = p.d / p.bn_dxt;
-    g.out0 = w.dXt;
-    if (rg) {
-      g.rvec = w.WrT;
-      g.rscale = w.dz_row;
-    }
-    MOE_TRY_MAP(make_store_map(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
-    ProfScope ps(st, "dxt_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
-  }
+  record_ready(grad_ready, 0, st);  // dW2 final
   // dW1[e] = X[tok]^T dH
   {
     GemmParams g = base_params(p, rt, status);
@@ -566,6 +569,22 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
     ProfScope ps(st, "dw1_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, 4, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+  }
+  record_ready(grad_ready, 1, st);  // dW1 final
+  // dX~ = dH W1[e]^T
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap(&g.tmA, w.dH, (uint64_t)p.R_max, (uint64_t)2 * p.n, 64, 128));
+    MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
+    g.num_n_tiles = p.d / p.bn_dxt;
+    g.out0 = w.dXt;
+    if (rg) {
+      g.rvec = w.WrT;
+      g.rscale = w.dz_row;
+    }
+    MOE_TRY_MAP(make_store_map(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
+    ProfScope ps(st, "dxt_gemm");
+    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
   if (rg) {
     GemmParams g = base_params(p, rt, status);
@@ -586,6 +605,7 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
       MOE_TRY_CUDA(launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st));
     }
   }
+  record_ready(grad_ready, 2, st);  // dWr final (or nothing to wait for without the router path)
   {
     ProfScope ps(st, "aggregate_bwd");
     MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, w.dXt,
@@ -605,6 +625,13 @@ moe_status moe_get_status(void* stream, int32_t* where) {
   if (cudaMemcpy(status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
   if (where) *where = h[1];
   return static_cast<moe_status>(h[0]);
+}
+
+moe_status moe_set_sm_budget(int32_t sms) {
+  if (sms < 0) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_sm_budget = sms;
+  return MOE_OK;
 }
 
 moe_status moe_set_spin_limit(int64_t cycles) {
@@ -699,6 +726,7 @@ bool noalloc_scratch(int dev, void** out) {
 size_t carve_noalloc_route(const Plan& p, void* base, RouteWs* w) {
   Carve c{static_cast<char*>(base)};
   w->Wr_split = c.take<__nv_bfloat16>((size_t)p.d * 3 * p.Epad);
+  w->sync = c.take<int>(4);
   w->hist = c.take<int>((size_t)p.nchunks * p.E);
   w->local_rank = c.take<int>((size_t)p.T * p.K);
   w->logits = nullptr;

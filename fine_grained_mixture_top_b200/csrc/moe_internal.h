@@ -41,6 +41,7 @@ struct RouteArgs {
   int* row_tok;             // [R_max]
   float* row_gate;          // [R_max]
   int* tile_expert;         // [R_max/128]
+  int* sync;                // [1] blocks done (zeroed by the rank kernel)
   int* hist;                // [nchunks, E]
   int* local_rank;          // [P_max]
   int nchunks;

@@ -85,63 +85,77 @@ cudaError_t launch_split_wr(const RouteArgs& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------- softmax + top-K
-// One warp per token.  p = softmax(z) over all E; the K largest logits are
-// selected (ties to the lower expert index, slots in descending order); the
-// gates are a softmax over the selected logits (= p renormalised).
+// One warp per token; lane l holds the logits of experts l, l + 32, ... in
+// registers (PER of them).  p = softmax(z) over all E.  The K largest logits
+// are selected in K rounds (ties to the lower expert index, slots in
+// descending order): each lane offers its best unselected logit, one
+// warp-wide max over order-preserving integer keys finds the value and one
+// warp-wide min finds the lowest expert holding it.  The gates are a softmax
+// over the selected logits (= p renormalised).
 constexpr int kTopkWarps = 8;
 
+// Unsigned key with the order of the float (no NaNs among logits).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int PER>
 __global__ void __launch_bounds__(256) softmax_topk_kernel(RouteArgs a) {
-  extern __shared__ float sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* z = sh + warp * a.E;
-  uint32_t* sel = reinterpret_cast<uint32_t*>(sh + kTopkWarps * a.E) + warp * 32;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= a.T) return;  // warp-uniform
   const float* lg = a.logits + (size_t)t * a.E;
+  float z[PER];
   float m = -FLT_MAX;
-  for (int e = lane; e < a.E; e += 32) {
-    const float v = lg[e];
-    z[e] = v;
-    m = fmaxf(m, v);
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = lane + 32 * j;
+    z[j] = e < a.E ? lg[e] : -FLT_MAX;
+    if (e < a.E) m = fmaxf(m, z[j]);
   }
-  sel[lane] = 0u;
   m = warp_max(m);
   float sum = 0.f;
-  for (int e = lane; e < a.E; e += 32) sum += expf(z[e] - m);
+#pragma unroll
+  for (int j = 0; j < PER; ++j)
+    if (lane + 32 * j < a.E) sum += expf(z[j] - m);
   sum = warp_sum(sum);
   const float inv = 1.0f / sum;
   float* pr = a.probs + (size_t)t * a.E;
-  for (int e = lane; e < a.E; e += 32) pr[e] = expf(z[e] - m) * inv;
-  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < PER; ++j)
+    if (lane + 32 * j < a.E) pr[lane + 32 * j] = expf(z[j] - m) * inv;
 
+  uint32_t taken = 0u;  // bit j: expert lane + 32 j already selected
   float my_v = 0.f;
   int my_e = 0;
   for (int k = 0; k < a.K; ++k) {
-    float bv = -FLT_MAX;
-    int be = INT_MAX;
-    for (int e = lane; e < a.E; e += 32) {
-      if ((sel[e >> 5] >> (e & 31)) & 1u) continue;
-      const float v = z[e];
-      if (be == INT_MAX || v > bv || (v == bv && e < be)) {
-        bv = v;
-        be = e;
-      }
-    }
+    uint32_t best = 0u;   // 0: nothing left on this lane (below every real key)
+    uint32_t best_e = 0xFFFFFFFFu;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-        bv = ov;
-        be = oe;
+    for (int j = 0; j < PER; ++j) {
+      const int e = lane + 32 * j;
+      if (e < a.E && !((taken >> j) & 1u)) {
+        const uint32_t key = order_key(z[j] == 0.f ? 0.f : z[j]);  // -0 ties with +0
+        if (key > best) {  // strict: the lower expert of a lane wins a tie
+          best = key;
+          best_e = (uint32_t)e;
+        }
       }
     }
-    if (lane == 0) sel[be >> 5] |= 1u << (be & 31);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, best == kmax ? best_e : 0xFFFFFFFFu);
+    const int owner = (int)(win & 31u);
+    if (lane == owner) taken |= 1u << (win >> 5);
+    float v_win = 0.f;
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+      if ((int)(win >> 5) == j) v_win = z[j];
+    v_win = __shfl_sync(0xffffffffu, v_win, owner);
     if (lane == k) {
-      my_v = bv;
-      my_e = be;
+      my_v = v_win;
+      my_e = (int)win;
     }
-    __syncwarp();
   }
   const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
   const float ex = lane < a.K ? expf(my_v - vmax) : 0.f;
@@ -162,18 +176,26 @@ __global__ void __launch_bounds__(256) softmax_topk_kernel(RouteArgs a) {
 
 cudaError_t launch_softmax_topk(const RouteArgs& a, cudaStream_t s) {
   const int blocks = (a.T + kTopkWarps - 1) / kTopkWarps;
-  const size_t smem = (size_t)kTopkWarps * a.E * sizeof(float) + kTopkWarps * 32 * sizeof(uint32_t);
-  softmax_topk_kernel<<<blocks, 256, smem, s>>>(a);
+  const int per = (a.E + 31) / 32;
+  if (per <= 1) softmax_topk_kernel<1><<<blocks, 256, 0, s>>>(a);
+  else if (per <= 2) softmax_topk_kernel<2><<<blocks, 256, 0, s>>>(a);
+  else if (per <= 4) softmax_topk_kernel<4><<<blocks, 256, 0, s>>>(a);
+  else if (per <= 8) softmax_topk_kernel<8><<<blocks, 256, 0, s>>>(a);
+  else if (per <= 16) softmax_topk_kernel<16><<<blocks, 256, 0, s>>>(a);
+  else if (per <= 32) softmax_topk_kernel<32><<<blocks, 256, 0, s>>>(a);
+  else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- permutation
-// Stable counting sort of all (token, expert) pairs by expert.  Tokens are cut
-// into chunks of 256; inside a chunk the rank of token t among the chunk's
-// tokens routed to e is a popcount over a per-expert bit mask, so the result
-// does not depend on the order in which threads run.
+// Stable counting sort of all (token, expert) pairs by expert, in three
+// launches.  Tokens are cut into chunks of 256; inside a chunk the rank of
+// token t among the chunk's tokens routed to e is a popcount over a
+// per-expert bit mask, so the result does not depend on the order in which
+// threads run.
 __global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
   extern __shared__ uint32_t bits[];  // [E][8]
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.sync = 0;  // for chunk_scan_kernel's last block
   const int words = kChunk / 32;
   for (int i = threadIdx.x; i < a.E * words; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
@@ -199,60 +221,93 @@ __global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
   }
 }
 
-// Per expert (one warp each, many blocks): exclusive scan over the chunks of
-// its per-chunk counts (chunk bases relative to the expert's segment) and
-// the expert's total count.
-__global__ void __launch_bounds__(256) chunk_scan_kernel(RouteArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 8 + warp;
-  if (e >= a.E) return;
-  int carry = 0;
-  for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
-    const int c = c0 + lane;
-    const int h = c < a.nchunks ? a.hist[(size_t)c * a.E + e] : 0;
-    int x = h;
+// Exclusive scan over a block of kScanThreads threads; *total gets the sum.
+constexpr int kScanThreads = 256;
+__device__ int block_exclusive_scan_256(int v, int* sh /*[8]*/, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kScanThreads / 32;
+  int x = v;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (c < a.nchunks) a.hist[(size_t)c * a.E + e] = carry + x - h;
-    carry += __shfl_sync(0xffffffffu, x, 31);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  if (lane == 0) a.counts[e] = carry;
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  int prefix = 0, sum = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) {
+    const int wv = sh[i];
+    if (i < warp) prefix += wv;
+    sum += wv;
+  }
+  __syncthreads();
+  *total = sum;
+  return prefix + x - v;
 }
 
-// One block: 128-padded segment offsets (exclusive scan over experts).
-__global__ void __launch_bounds__(1024) offsets_kernel(RouteArgs a) {
-  __shared__ int sh[33];
+// Per expert (one warp each, several blocks): exclusive scan over the chunks
+// of its per-chunk counts (chunk bases relative to the expert's segment) and
+// the expert's total count.  The last block to finish then computes the
+// 128-padded segment offsets (exclusive scan over experts).
+__global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(RouteArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (kScanThreads / 32) + warp;
+  if (e < a.E) {
+    int carry = 0;
+    for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int h = c < a.nchunks ? a.hist[(size_t)c * a.E + e] : 0;
+      int x = h;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (c < a.nchunks) a.hist[(size_t)c * a.E + e] = carry + x - h;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) a.counts[e] = carry;
+  }
+  // The last block to arrive sees every block's counts: each block fences its
+  // writes before it counts itself done, and the last one fences before reading.
+  __shared__ int is_last;
+  __shared__ int sh[kScanThreads / 32];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(a.sync, 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
   int carry = 0;
-  for (int e0 = 0; e0 < a.E; e0 += 1024) {
-    const int e = e0 + threadIdx.x;
-    const int padded = e < a.E ? ((a.counts[e] + kTile - 1) / kTile) * kTile : 0;
+  for (int e0 = 0; e0 < a.E; e0 += kScanThreads) {
+    const int ee = e0 + threadIdx.x;
+    const int padded = ee < a.E ? ((__ldcg(a.counts + ee) + kTile - 1) / kTile) * kTile : 0;
     int total;
-    const int ex = block_exclusive_scan_1024(padded, sh, &total);
-    if (e < a.E) a.offsets[e] = carry + ex;
+    const int ex = block_exclusive_scan_256(padded, sh, &total);
+    if (ee < a.E) a.offsets[ee] = carry + ex;
     carry += total;
   }
   if (threadIdx.x == 0) a.offsets[a.E] = carry;
 }
 
-// Per expert (one warp each): the tile -> expert list and the padding rows
-// (token -1, gate 0) of its segment.
-__global__ void __launch_bounds__(256) segment_fill_kernel(RouteArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 8 + warp;
-  if (e >= a.E) return;
-  const int base = a.offsets[e];
-  const int end = a.offsets[e + 1];
-  for (int tt = base / kTile + lane; tt < end / kTile; tt += 32) a.tile_expert[tt] = e;
-  for (int r = base + a.counts[e] + lane; r < end; r += 32) {
-    a.row_tok[r] = -1;
-    a.row_gate[r] = 0.f;
+// Blocks [0, token_blocks): one thread per token writes its pairs' rows.
+// The blocks after those: one warp per expert writes the tile -> expert list
+// and the padding rows (token -1, gate 0) of its segment.
+__global__ void __launch_bounds__(256) scatter_kernel(RouteArgs a, int token_blocks) {
+  if ((int)blockIdx.x >= token_blocks) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = ((int)blockIdx.x - token_blocks) * 8 + warp;
+    if (e >= a.E) return;
+    const int base = a.offsets[e];
+    const int end = a.offsets[e + 1];
+    for (int tt = base / kTile + lane; tt < end / kTile; tt += 32) a.tile_expert[tt] = e;
+    for (int r = base + a.counts[e] + lane; r < end; r += 32) {
+      a.row_tok[r] = -1;
+      a.row_gate[r] = 0.f;
+    }
+    return;
   }
-}
-
-__global__ void scatter_kernel(RouteArgs a) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= a.T) return;
   const int* base = a.hist + (size_t)(t / kChunk) * a.E;
@@ -270,22 +325,14 @@ cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s) {
     ProfScope ps(s, "permute_rank");
     rank_kernel<<<a.nchunks, kChunk, (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s>>>(a);
   }
-  const int eb = (a.E + 7) / 8;
   {
-    ProfScope ps(s, "permute_chunk_scan");
-    chunk_scan_kernel<<<eb, 256, 0, s>>>(a);
-  }
-  {
-    ProfScope ps(s, "permute_offsets");
-    offsets_kernel<<<1, 1024, 0, s>>>(a);
-  }
-  {
-    ProfScope ps(s, "permute_segment_fill");
-    segment_fill_kernel<<<eb, 256, 0, s>>>(a);
+    ProfScope ps(s, "permute_scan");
+    chunk_scan_kernel<<<(a.E + 7) / 8, kScanThreads, 0, s>>>(a);
   }
   {
     ProfScope ps(s, "permute_scatter");
-    scatter_kernel<<<(a.T + 255) / 256, 256, 0, s>>>(a);
+    const int token_blocks = (a.T + 255) / 256;
+    scatter_kernel<<<token_blocks + (a.E + 7) / 8, 256, 0, s>>>(a, token_blocks);
   }
   return cudaGetLastError();
 }

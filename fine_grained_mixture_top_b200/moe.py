@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.moe_backward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    ctypes.c_size_t, c_void_p]
+        L.moe_backward_ev.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      ctypes.c_size_t, P(c_void_p), c_void_p]
+        L.moe_set_sm_budget.argtypes = [c_int32]
         L.moe_get_status.argtypes = [c_void_p, P(c_int32)]
         L.moe_set_spin_limit.argtypes = [c_int64]
         L.moe_selftest_wait_timeout.argtypes = [c_void_p, c_void_p]
@@ -91,7 +95,8 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
-                  "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout"):
+                  "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout", "moe_backward_ev",
+                  "moe_set_sm_budget"):
             getattr(L, f).restype = c_int32
         _lib = L
     return _lib
@@ -190,11 +195,26 @@ def moe_forward(dims, opts, X, W1, W2, routing: Routing, O, H, ws, stream=None):
                              ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
 
 
-def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW2, dWr, ws, stream=None):
-    _check(lib().moe_backward(ctypes.byref(dims), ctypes.byref(opts), _ptr(dO), _ptr(X), _ptr(Wr), _ptr(W1),
-                              _ptr(W2), ctypes.byref(routing.struct), _ptr(H), _ptr(dX), _ptr(dW1), _ptr(dW2),
-                              _ptr(dWr), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
-           "moe_backward")
+def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW2, dWr, ws, stream=None,
+                 grad_events=None):
+    """grad_events: None, or three torch.cuda.Event (or None) recorded once
+    dW2, dW1 and dWr are final."""
+    args = (ctypes.byref(dims), ctypes.byref(opts), _ptr(dO), _ptr(X), _ptr(Wr), _ptr(W1), _ptr(W2),
+            ctypes.byref(routing.struct), _ptr(H), _ptr(dX), _ptr(dW1), _ptr(dW2), _ptr(dWr), _ptr(ws),
+            ws.numel() * ws.element_size())
+    if grad_events is None:
+        _check(lib().moe_backward(*args, _stream(stream)), "moe_backward")
+        return
+    for e in grad_events:
+        if e is not None and not e.cuda_event:  # torch creates its event on the first record
+            e.record()
+    evs = (c_void_p * 3)(*[None if e is None else e.cuda_event for e in grad_events])
+    _check(lib().moe_backward_ev(*args, evs, _stream(stream)), "moe_backward_ev")
+
+
+def moe_set_sm_budget(sms: int):
+    """At most `sms` CTAs per persistent GEMM (0: one per SM)."""
+    _check(lib().moe_set_sm_budget(int(sms)), "moe_set_sm_budget")
 
 
 def moe_get_status(stream=None) -> tuple[int, int]:
@@ -265,16 +285,48 @@ class MoELayer:
         moe_forward(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd, stream)
         return O
 
-    def backward(self, dO, X, Wr, W1, W2, stream=None):
+    def backward(self, dO, X, Wr, W1, W2, stream=None, grad_events=None):
         moe_backward(self.dims, self.opts, dO, X, Wr, W1, W2, self.routing, self.H, self.dX, self.dW1, self.dW2,
-                     self.dWr if self.opts.router_grad else None, self.ws_bwd, stream)
+                     self.dWr if self.opts.router_grad else None, self.ws_bwd, stream, grad_events)
         return self.dX, self.dW1, self.dW2, self.dWr
 
-    def step(self, X, Wr, bias, W1, W2, dO, stream=None):
+    def step(self, X, Wr, bias, W1, W2, dO, stream=None, grad_events=None):
         """One pass of the whole path: route (+ rounding), forward, backward."""
         self.route(X, Wr, bias, stream)
         self.forward(X, W1, W2, stream)
-        return self.backward(dO, X, Wr, W1, W2, stream)
+        return self.backward(dO, X, Wr, W1, W2, stream, grad_events)
+
+
+class OverlappedGradReduce:
+    """Data-parallel steps whose weight-gradient sums over `group` overlap the
+    backward.  The backward records an event as soon as dW2, then dW1, then dWr
+    are written (moe_backward_ev computes dW2 and dW1 before dX~); each
+    all-reduce waits on its event on a separate stream, so the reductions of
+    dW2 and dW1 run while the dX~ GEMM and the dX aggregation do.  The current
+    stream waits for the reductions at the end of the step, before the next
+    step can overwrite the gradients."""
+
+    def __init__(self, layer, group=None):
+        import torch
+        self.layer = layer
+        self.group = group
+        self.comm = torch.cuda.Stream()
+        self.events = [torch.cuda.Event() for _ in range(3)]
+
+    def step(self, X, Wr, bias, W1, W2, dO):
+        import torch
+        import torch.distributed as dist
+        L = self.layer
+        L.step(X, Wr, bias, W1, W2, dO, grad_events=self.events)
+        grads = (L.dW2, L.dW1, L.dWr if L.opts.router_grad else None)
+        with torch.cuda.stream(self.comm):
+            for ev, g in zip(self.events, grads):
+                if g is None:
+                    continue
+                self.comm.wait_event(ev)
+                dist.all_reduce(g, group=self.group)
+        torch.cuda.current_stream().wait_stream(self.comm)
+        return L.dX, L.dW1, L.dW2, L.dWr
 
 
 class HostFedRunner:

@@ -167,6 +167,31 @@ moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* 
                         void* dX, void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_backward that also reports when each weight gradient is final, so that
+ * a data-parallel caller can start reducing it across ranks while the rest of
+ * the backward runs (the pages train their layer data-parallel; the reduction
+ * is the caller's).  grad_ready may be NULL, else it points to three
+ * cudaEvent_t handles (each may be NULL), recorded on `stream`:
+ *   grad_ready[0] once dW2 is written, grad_ready[1] once dW1 is written,
+ *   grad_ready[2] once dWr is written (router_grad = 0: at the same point).
+ * dW2 and dW1 are computed before dX~, so their reductions overlap the dX~
+ * GEMM and the dX aggregation.  Events are caller-owned; everything else is
+ * as for moe_backward.
+ */
+moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X,
+                           const float* Wr, const void* W1, const void* W2, const moe_routing* rt, const void* H,
+                           void* dX, void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes,
+                           void* const* grad_ready, void* stream);
+
+/*
+ * At most `sms` CTAs for each persistent GEMM kernel launched from now on by
+ * this process (0, the default: one per SM).  A caller that overlaps a
+ * communication kernel with the backward leaves SMs for it this way; results
+ * do not depend on the budget.  Negative values: MOE_ERR_INVALID_ARG.
+ */
+moe_status moe_set_sm_budget(int32_t sms);
+
+/*
  * Synchronises `stream`, returns the device status word (MOE_OK if no kernel
  * reported an error since the last call) and clears it.  *where (nullable)
  * receives the code of the wait or check that failed.

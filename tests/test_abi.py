@@ -82,6 +82,11 @@ def test_invalid_options_and_null_arguments(moe):
     assert L.moe_forward(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, ctypes.byref(rt),
                          None, None, None, 0, None) == 1
     assert L.moe_set_spin_limit(10) == 1
+    assert L.moe_set_sm_budget(-1) == 1
+    assert L.moe_set_sm_budget(0) == 0
+    assert L.moe_backward_ev(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, None, None,
+                             ctypes.byref(rt), None, None, None, None, None, None, 0, None, None) == 1
+    assert moe.last_error() == ""  # no CUDA error on this thread
 
 
 def test_status_strings(moe):

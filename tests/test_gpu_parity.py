@@ -153,3 +153,74 @@ def test_host_fed_runner_matches_device_steps():
         assert torch.equal(Oh, ref.O.cpu())
     for k in ("dX", "dW1", "dW2", "dWr"):
         assert torch.equal(getattr(layer, k), getattr(ref, k)), k
+
+
+@pytest.mark.gpu
+def test_sm_budget_does_not_change_results():
+    """Persistent GEMMs on fewer CTAs (SMs left to a communication kernel)
+    give bitwise the same outputs: every tile's arithmetic is independent of
+    which CTA computes it."""
+    from fine_grained_mixture_top_b200 import moe
+    cfg = SHAPES[2]
+    inp = make_inputs(cfg, "cuda")
+    ref = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    try:
+        moe.moe_set_sm_budget(37)
+        lim = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    finally:
+        moe.moe_set_sm_budget(0)
+    rows = int(ref.routing["offsets"][cfg.E].item())  # H rows past the last segment are never written
+    assert torch.equal(lim.H[:rows], ref.H[:rows])
+    for k in ("O", "dX", "dW1", "dW2", "dWr"):
+        assert torch.equal(getattr(lim, k), getattr(ref, k)), k
+
+
+@pytest.mark.gpu
+def test_grad_ready_events_mark_final_gradients():
+    """A copy of dW2, dW1 and dWr taken on another stream right after their
+    events equals the gradient at the end of the backward."""
+    from fine_grained_mixture_top_b200 import moe
+    cfg = SHAPES[1]
+    inp = make_inputs(cfg, "cuda")
+    layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    evs = [torch.cuda.Event() for _ in range(3)]
+    side = torch.cuda.Stream()
+    for _ in range(2):   # the second step overwrites the first step's gradients
+        layer.step(inp["X"], inp["Wr"], inp["bias"], inp["W1"], inp["W2"], inp["dO"], grad_events=evs)
+        with torch.cuda.stream(side):
+            copies = []
+            for ev, g in zip(evs, (layer.dW2, layer.dW1, layer.dWr)):
+                side.wait_event(ev)
+                copies.append(g.clone())
+        torch.cuda.synchronize()
+        for c, g in zip(copies, (layer.dW2, layer.dW1, layer.dWr)):
+            assert torch.equal(c, g)
+    assert moe.moe_get_status() == (0, 0)
+
+
+@pytest.mark.gpu
+def test_overlapped_reduce_on_one_rank_equals_plain_step():
+    """The overlapped data-parallel step on a one-rank NCCL group (the sum over
+    one rank is the identity) gives the plain step's outputs."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from fine_grained_mixture_top_b200 import moe
+    cfg = SHAPES[1]
+    inp = make_inputs(cfg, "cuda")
+    ref = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+        red = moe.OverlappedGradReduce(layer)
+        for _ in range(2):
+            red.step(inp["X"], inp["Wr"], inp["bias"], inp["W1"], inp["W2"], inp["dO"])
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for k in ("dX", "dW1", "dW2", "dWr"):
+        assert torch.equal(getattr(layer, k), getattr(ref, k)), k
