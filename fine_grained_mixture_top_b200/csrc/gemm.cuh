@@ -87,9 +87,13 @@ struct EpiCfg {
   static constexpr int kWarps = EPI;
   static constexpr int kColSplit = EPI / 4;
   // 2 KB staging buffers per warp: the up-proj and dH epilogues store three
-  // outputs per chunk; the others ring through 3 buffers (2 with 8 warps, so
-  // that the stage ring keeps its depth)
-  static constexpr int kBufs = (KIND == G_UP || KIND == G_DH) ? 3 : (EPI == 8 ? 2 : 3);
+  // outputs per chunk; the others ring through 3 buffers.  With 8 warps the
+  // dX~ kernel keeps 2 (so that its stage ring keeps its depth), while the
+  // weight-gradient kinds, which get 8 warps when their tiles are store-bound
+  // (few rows per expert), keep 4 bulk stores in flight per warp.
+  static constexpr int kBufs = (KIND == G_UP || KIND == G_DH)
+                                   ? 3
+                                   : (EPI == 8 ? (KindTraits<KIND>::kGroupedK ? 4 : 2) : 3);
   static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
   // registers per thread for one resident block (multiple of 8, at most 255);
   // 448-thread blocks stay under 61440 registers
@@ -675,21 +679,22 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       const int row0 = t.m0 + q * 32;  // first output row of this warp's slice
       if constexpr (KT::kGroupedK) {
         if (t.nkb == 0) {  // expert without tokens: its weight gradient is zero
+          // one staged box of zeros, stored to each 32-column chunk of this
+          // warp's rows as one bulk group
           const int M = (KIND == G_DW1) ? p.d : p.n;
           if (row0 < M) {
             float z[32];
             zero32(z);
-            for (int c = 0; c < BN; c += 32) {
-              const uint32_t buf = stg + ring * kStoreBuf;
-              stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
-              stage_row32(buf, lane, z);
-              stage_publish();
-              if (lane == 0) {
-                tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
-                bulk_commit();
-              }
-              ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
+            const uint32_t buf = stg + ring * kStoreBuf;
+            stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
+            stage_row32(buf, lane, z);
+            stage_publish();
+            if (lane == 0) {
+              constexpr int kC = BN / EC::kColSplit;
+              for (int c = half * kC; c < half * kC + kC; c += 32) tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
+              bulk_commit();
             }
+            ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
           }
           continue;
         }

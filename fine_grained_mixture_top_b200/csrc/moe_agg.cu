@@ -71,15 +71,15 @@ cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pa
 // and the token's dense dz row split into bf16 hi + lo parts for the
 // tensor-core dWr = X^T dz GEMM (layout: group g of 64 experts at columns
 // [128 g, 128 g + 128): hi parts then lo parts).
-__global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad, int nts,
-                                                         const int* __restrict__ tok_ptr,
-                                                         const int* __restrict__ pair_row,
-                                                         const int* __restrict__ pair_expert,
-                                                         const float* __restrict__ pair_gate,
-                                                         const float* __restrict__ dS_part, float* __restrict__ dz_row,
-                                                         __nv_bfloat16* __restrict__ dz_split) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
+__device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, int lane) {
+  const int T = a.T, Epad = a.Epad, nts = a.nds;
+  const int* __restrict__ tok_ptr = a.tok_ptr;
+  const int* __restrict__ pair_row = a.pair_row;
+  const int* __restrict__ pair_expert = a.pair_expert;
+  const float* __restrict__ pair_gate = a.pair_gate;
+  const float* __restrict__ dS_part = a.dS_part;
+  float* __restrict__ dz_row = a.dz_row;
+  __nv_bfloat16* __restrict__ dz_split = a.dz_split;
   if (t >= T) return;
   const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
   float inner = 0.f;
@@ -110,36 +110,28 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(int T, int E, int Epad,
   }
 }
 
-cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
-                              const int* pair_expert, const float* pair_gate, const float* dS_part,
-                              float* dz_row, __nv_bfloat16* dz_split, cudaStream_t s) {
-  router_bwd_kernel<<<(T + 7) / 8, 256, 0, s>>>(T, E, Epad, nts, tok_ptr, pair_row, pair_expert, pair_gate,
-                                                dS_part, dz_row, dz_split);
-  return cudaGetLastError();
-}
 
 // WrT[e, i] = Wr[i, e]
-__global__ void transpose_kernel(const float* __restrict__ in, float* __restrict__ out, int rows, int cols) {
+// 32 x 32 tile (bx, by) of the transpose, 256 threads (32 x 8)
+__device__ __forceinline__ void transpose_tile(const float* __restrict__ in, float* __restrict__ out, int rows,
+                                               int cols, int bx, int by) {
   __shared__ float tile[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < rows && c < cols) tile[i][threadIdx.x] = in[(size_t)r * cols + c];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int c0 = bx * 32, r0 = by * 32;
+  for (int i = ty; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + tx;
+    if (r < rows && c < cols) tile[i][tx] = in[(size_t)r * cols + c];
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][i];
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + tx;
+    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[tx][i];
   }
 }
 
-cudaError_t launch_transpose_wr(int d, int E, const float* Wr, float* WrT, cudaStream_t s) {
-  dim3 grid((E + 31) / 32, (d + 31) / 32), block(32, 8);
-  transpose_kernel<<<grid, block, 0, s>>>(Wr, WrT, d, E);
-  return cudaGetLastError();
-}
 
-// dWr[i, e] = sum over K splits of the split-K partials
+
+// dWr[i, e] = sum over K splits of the split-K partials, in split order
 __global__ void dwr_reduce_kernel(int d, int E, int Epad, int splits, const float* __restrict__ part,
                                   float* __restrict__ dWr) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -191,8 +183,7 @@ cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pa
 // Experts sorted by descending token count (ties: lower index first); the
 // weight-gradient GEMMs take their tiles in this order so that the longest
 // tiles start first.
-__global__ void __launch_bounds__(1024) expert_order_kernel(int E, const int* __restrict__ counts,
-                                                            int* __restrict__ order) {
+__device__ __forceinline__ void expert_order_block(int E, const int* __restrict__ counts, int* __restrict__ order) {
   __shared__ int c[1024];
   for (int e = threadIdx.x; e < E; e += blockDim.x) c[e] = counts[e];
   __syncthreads();
@@ -204,10 +195,36 @@ __global__ void __launch_bounds__(1024) expert_order_kernel(int E, const int* __
   }
 }
 
-cudaError_t launch_expert_order(int E, const int* counts, int* order, cudaStream_t s) {
-  expert_order_kernel<<<1, 1024, 0, s>>>(E, counts, order);
+// One launch before the weight-gradient GEMMs (after the dH kernel):
+//   blocks [0, tok_blocks)              router backward, one warp per token
+//   next tr_blocks blocks               Wr^T for the dX~ epilogue's router path
+//   last block                          expert order (largest first) for the
+//                                       weight-gradient scheduler; zeroes its
+//                                       tile counters
+__global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
+  const int b = blockIdx.x;
+  if (b < a.tok_blocks) {
+    router_bwd_token(a, b * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+    return;
+  }
+  if (b < a.tok_blocks + a.tr_blocks) {
+    const int i = b - a.tok_blocks;
+    const int nbx = (a.E + 31) / 32;
+    transpose_tile(a.Wr, a.WrT, a.d, a.E, i % nbx, i / nbx);
+    return;
+  }
+  if (threadIdx.x < 16) a.sched[threadIdx.x] = 0;
+  expert_order_block(a.E, a.counts, a.expert_order);
+}
+
+cudaError_t launch_bwd_prep(const BwdPrepArgs& a0, cudaStream_t s) {
+  BwdPrepArgs a = a0;
+  a.tok_blocks = a.router ? (a.T + 7) / 8 : 0;
+  a.tr_blocks = a.router ? ((a.E + 31) / 32) * ((a.d + 31) / 32) : 0;
+  bwd_prep_kernel<<<a.tok_blocks + a.tr_blocks + 1, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
+
 
 // Failure-detection self test: one thread waits on an mbarrier that nothing
 // will ever complete, through the same bounded wait the GEMM kernels use, and

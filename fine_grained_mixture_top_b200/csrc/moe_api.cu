@@ -99,6 +99,7 @@ struct Plan {
   int nts;  // N tiles of the dH kernel
   int nds;  // dS partials per row: N tiles x column parts of the dH epilogue
   int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
+  int epi_dw;           // epilogue warps of the weight-gradient kernels
   int ksplit, ksplit_rows;
 };
 
@@ -142,6 +143,10 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   // with 8: its short main loop is bound by the Y stores, not the epilogue.)
   p.epi_dh = (d / 64 <= 24) ? 8 : 4;
   p.epi_dxt = (2 * n / 64 <= 16) ? 8 : 4;
+  // The weight-gradient tiles run K over an expert's rows; with few rows per
+  // expert (at most 8 k-blocks on average) a tile is bound by storing its
+  // 128 x BN result, so the epilogue gets 8 warps.
+  p.epi_dw = (T * K / E <= 8 * 64) ? 8 : 4;
   p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
@@ -170,9 +175,11 @@ struct RouteWs {
   int* sync;  // [1] blocks done, for the last-block offsets scan of the permutation
   int* hist;
   int* local_rank;
-  uint32_t* member;
-  uint32_t* final_;
-  int* cnt;
+  uint32_t* memberT;  // token rounding: [E, ceil(T/32)]
+  uint32_t* finalT;   // token rounding: [E, ceil(T/32)]
+  float* probsT;      // token rounding: [E, T]
+  int* local;         // token rounding: [T]
+  int* blk;           // token rounding: [ceil(T/256) + 1]
 };
 size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
   Carve c{static_cast<char*>(ws)};
@@ -181,9 +188,12 @@ size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
   w->sync = c.take<int>(4);
   w->hist = c.take<int>((size_t)p.nchunks * p.E);
   w->local_rank = c.take<int>((size_t)p.P_max);
-  w->member = c.take<uint32_t>((size_t)p.T * p.Ew);
-  w->final_ = c.take<uint32_t>((size_t)p.T * p.Ew);
-  w->cnt = c.take<int>((size_t)p.T);
+  const size_t W = (size_t)cdiv(p.T, 32);
+  w->memberT = c.take<uint32_t>((size_t)p.E * W);
+  w->finalT = c.take<uint32_t>((size_t)p.E * W);
+  w->probsT = c.take<float>((size_t)p.E * p.T);
+  w->local = c.take<int>((size_t)p.T);
+  w->blk = c.take<int>((size_t)cdiv(p.T, 256) + 1);
   return c.off;
 }
 
@@ -411,10 +421,12 @@ moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe
   r.mode = opts->round_mode;
   r.seed = (unsigned long long)opts->seed;
   r.probs = rt->probs;
-  r.member = w.member;
-  r.final_ = w.final_;
-  r.cnt = w.cnt;
-  r.Ew = p.Ew;
+  r.probsT = w.probsT;
+  r.memberT = w.memberT;
+  r.finalT = w.finalT;
+  r.local = w.local;
+  r.blk = w.blk;
+  r.sync = w.sync + 1;
   MOE_TRY_CUDA(launch_token_round(a, r, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
@@ -501,14 +513,6 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
   const int64_t mtiles = p.R_max / kTile;
   const __nv_bfloat16* dOb = static_cast<const __nv_bfloat16*>(dO);
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
-  // dynamic-scheduler counters of the weight-gradient GEMMs, and the expert
-  // order (largest first) in which they take their tiles
-  MOE_TRY_CUDA(cudaMemsetAsync(w.sched, 0, 16 * sizeof(int), st));
-  {
-    ProfScope ps(st, "expert_order");
-    MOE_TRY_CUDA(launch_expert_order(p.E, rt->counts, w.expert_order, st));
-  }
-
   // dH kernel: dA' = dO[tok] W2[e]^T; epilogue: H -> A, dS partials, dSwiGLU, A_hat
   {
     GemmParams g = base_params(p, rt, status);
@@ -525,17 +529,31 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     ProfScope ps(st, "dh_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DH, p.bn_dh, p.epi_dh, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
-  // router path, dz = s * (dS - sum_j s_j dS_j), before dX~ which consumes it
-  if (rg) {
-    {
-      ProfScope ps(st, "router_bwd");
-      MOE_TRY_CUDA(launch_router_bwd((int)p.T, p.E, p.Epad, p.nds, rt->tok_ptr, rt->pair_row, rt->pair_expert,
-                                     rt->pair_gate, w.dS_part, w.dz_row, w.dz_split, st));
-    }
-    {
-      ProfScope ps(st, "router_wr_transpose");
-      MOE_TRY_CUDA(launch_transpose_wr(p.d, p.E, Wr, w.WrT, st));
-    }
+  // Router path, dz = s * (dS - sum_j s_j dS_j), and Wr^T, both consumed by
+  // the dX~ epilogue; the expert order (largest first) in which the
+  // weight-gradient GEMMs take their tiles, and their zeroed tile counters.
+  {
+    BwdPrepArgs a{};
+    a.T = (int)p.T;
+    a.d = p.d;
+    a.E = p.E;
+    a.Epad = p.Epad;
+    a.nds = p.nds;
+    a.router = rg ? 1 : 0;
+    a.tok_ptr = rt->tok_ptr;
+    a.pair_row = rt->pair_row;
+    a.pair_expert = rt->pair_expert;
+    a.pair_gate = rt->pair_gate;
+    a.dS_part = w.dS_part;
+    a.dz_row = w.dz_row;
+    a.dz_split = w.dz_split;
+    a.Wr = Wr;
+    a.WrT = w.WrT;
+    a.counts = rt->counts;
+    a.expert_order = w.expert_order;
+    a.sched = w.sched;
+    ProfScope ps(st, "bwd_prep");
+    MOE_TRY_CUDA(launch_bwd_prep(a, st));
   }
   // dW2[e] = A_hat^T dO[tok]
   {
@@ -550,7 +568,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, 4, g,
+    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, p.epi_dw, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
   record_ready(grad_ready, 0, st);  // dW2 final
@@ -567,7 +585,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, 4, g,
+    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, p.epi_dw, g,
                              grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
   }
   record_ready(grad_ready, 1, st);  // dW1 final
@@ -730,9 +748,11 @@ size_t carve_noalloc_route(const Plan& p, void* base, RouteWs* w) {
   w->hist = c.take<int>((size_t)p.nchunks * p.E);
   w->local_rank = c.take<int>((size_t)p.T * p.K);
   w->logits = nullptr;
-  w->member = nullptr;
-  w->final_ = nullptr;
-  w->cnt = nullptr;
+  w->memberT = nullptr;
+  w->finalT = nullptr;
+  w->probsT = nullptr;
+  w->local = nullptr;
+  w->blk = nullptr;
   return c.off;
 }
 }  // namespace

@@ -44,8 +44,12 @@ cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid
   MOE_CASE(G_DXT, 256, 8)
   MOE_CASE(G_DW1, 128, 4)
   MOE_CASE(G_DW1, 256, 4)
+  MOE_CASE(G_DW1, 128, 8)
+  MOE_CASE(G_DW1, 256, 8)
   MOE_CASE(G_DW2, 128, 4)
   MOE_CASE(G_DW2, 256, 4)
+  MOE_CASE(G_DW2, 128, 8)
+  MOE_CASE(G_DW2, 256, 8)
   MOE_CASE(G_RTR, 192, 4)
   MOE_CASE(G_DWR, 128, 4)
 #undef MOE_CASE

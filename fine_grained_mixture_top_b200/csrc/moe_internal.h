@@ -54,25 +54,40 @@ cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s);  // rank + scan 
 struct RoundArgs {
   int T, E, mode;
   unsigned long long seed;
-  const float* probs;
-  uint32_t* member;   // [T, Ew]
-  uint32_t* final_;   // [T, Ew]
-  int* cnt;           // [T]
-  int Ew;
+  const float* probs;   // [T, E]
+  float* probsT;        // [E, T]
+  uint32_t* memberT;    // [E, ceil(T/32)] routed tokens of each expert
+  uint32_t* finalT;     // [E, ceil(T/32)] tokens of each expert after rounding
+  int* local;           // [T] offset of each token's pairs inside its block of 256
+  int* blk;             // [ceil(T/256) + 1] block offsets, total last
+  int* sync;            // [1] blocks done
 };
 cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStream_t s);
 
 // ---- aggregation and router backward (moe_agg.cu)
 cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pair_row, const float* pair_gate,
                                  const __nv_bfloat16* Y, __nv_bfloat16* O, cudaStream_t s);
-cudaError_t launch_router_bwd(int T, int E, int Epad, int nts, const int* tok_ptr, const int* pair_row,
-                              const int* pair_expert, const float* pair_gate, const float* dS_part,
-                              float* dz_row, __nv_bfloat16* dz_split, cudaStream_t s);
-cudaError_t launch_transpose_wr(int d, int E, const float* Wr, float* WrT, cudaStream_t s);
+// Backward preparation (router backward, Wr^T, expert order), one launch.
+struct BwdPrepArgs {
+  int T, d, E, Epad, nds;  // nds: dS partials per row
+  int router;              // router path on: dz, dz split and Wr^T
+  const int* tok_ptr;
+  const int* pair_row;
+  const int* pair_expert;
+  const float* pair_gate;
+  const float* dS_part;
+  float* dz_row;               // [R_max]
+  __nv_bfloat16* dz_split;     // [T, 2 Epad]
+  const float* Wr;             // [d, E]
+  float* WrT;                  // [E, d]
+  const int* counts;           // [E]
+  int* expert_order;           // [E]
+  int* sched;                  // [16] weight-gradient tile counters, zeroed here
+  int tok_blocks, tr_blocks;   // set by the launcher
+};
+cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t s);
 cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s);
 cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const __nv_bfloat16* dXt,
                                  __nv_bfloat16* dX, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
-cudaError_t launch_expert_order(int E, const int* counts, int* order, cudaStream_t s);
-
 }  // namespace moe

@@ -30,33 +30,6 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Exclusive scan over a 1024-thread block; *total receives the block sum.
-__device__ int block_exclusive_scan_1024(int v, int* sh /*[33]*/, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = sh[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    sh[lane] = w;
-  }
-  __syncthreads();
-  const int prefix = warp > 0 ? sh[warp - 1] : 0;
-  *total = sh[31];
-  __syncthreads();
-  return prefix + x - v;
-}
-
 // ---------------------------------------------------------------- Wr split
 // Wr (fp32) = hi + mid + lo with each part a bf16; X is exactly bf16, so the
 // three tensor-core products accumulated in fp32 give fp32-accurate logits.
@@ -351,148 +324,291 @@ __device__ __forceinline__ unsigned long long splitmix64_dev(unsigned long long 
   return z ^ (z >> 31);
 }
 
-__global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int Ew, uint32_t* member) {
+// Token rounding works on per-expert rows: memberT[e][w] holds bit t & 31 of
+// word w = t / 32 for each token t routed to e, probsT[e][t] = p[t, e].  One
+// block per expert then reads its row contiguously.
+__global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int W, uint32_t* memberT,
+                                 int* sync) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t == 0) *sync = 0;  // for tr_count_kernel's last block
   if (t >= T) return;
-  for (int p = tok_ptr[t]; p < tok_ptr[t + 1]; ++p) {
-    const int e = pair_expert[p];
-    atomicOr(&member[(size_t)t * Ew + (e >> 5)], 1u << (e & 31));
+  for (int p = tok_ptr[t]; p < tok_ptr[t + 1]; ++p)
+    atomicOr(&memberT[(size_t)pair_expert[p] * W + (t >> 5)], 1u << (t & 31));
+}
+
+// probsT[e, t] = probs[t, e], 32 x 32 tiles through shared memory
+__global__ void tr_transpose_kernel(const float* __restrict__ probs, float* __restrict__ probsT, int T, int E) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.x * 32, t0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int t = t0 + i, e = e0 + threadIdx.x;
+    if (t < T && e < E) tile[i][threadIdx.x] = probs[(size_t)t * E + e];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int e = e0 + i, t = t0 + threadIdx.x;
+    if (t < T && e < E) probsT[(size_t)e * T + t] = tile[threadIdx.x][i];
   }
 }
 
 // One block per expert: radix select (8 passes of 8 bits) of the k extreme
-// 64-bit keys (p bits << 32 | ~t) among the candidate tokens.
-__global__ void __launch_bounds__(1024) tr_select_kernel(int T, int E, int Ew, int mode, unsigned long long seed,
-                                                         const int* counts, const float* probs,
-                                                         const uint32_t* member, uint32_t* final_) {
+// 64-bit keys (p bits << 32 | ~t) among the candidate tokens, then the
+// expert's final row finalT[e] = memberT[e] with the selected tokens added
+// (rounding up) or removed (rounding down).  With STAGED the expert's p row
+// and candidate mask are first copied into shared memory; histogram updates
+// are aggregated per warp over lanes with the same digit.
+template <bool STAGED>
+__global__ void __launch_bounds__(1024) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
+                                                         const int* counts, const float* probsT,
+                                                         const uint32_t* memberT, uint32_t* finalT) {
+  extern __shared__ uint32_t stage[];  // STAGED: p bits [T], then the candidate mask [W]
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ int s_k;
   const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const uint32_t* mrow = memberT + (size_t)e * W;
+  uint32_t* frow = finalT + (size_t)e * W;
+  const float* prow = probsT + (size_t)e * T;
   const int c = counts[e];
   const int rem = c % kTile;
-  if (rem == 0) return;
+  if (rem == 0) {  // already a multiple of the tile: keep the routed set
+    for (int w = threadIdx.x; w < W; w += blockDim.x) frow[w] = mrow[w];
+    return;
+  }
   bool up;
   if (mode == 1) up = rem >= kTile / 2;
   else up = (int)(splitmix64_dev(seed ^ (unsigned long long)e) % (unsigned long long)kTile) < rem;
   if (up && c - rem + kTile > T) up = false;
   const int k = up ? kTile - rem : rem;
-  const uint32_t wmask = 1u << (e & 31);
-  const int wi = e >> 5;
+  // candidates: unrouted tokens when rounding up, routed ones when rounding down
+  const uint32_t tail = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xFFFFFFFFu;
+  auto cand_word = [&](int w) -> uint32_t {
+    const uint32_t m = mrow[w];
+    const uint32_t valid = (w == W - 1) ? tail : 0xFFFFFFFFu;
+    return (up ? ~m : m) & valid;
+  };
+  uint32_t* s_p = stage;
+  uint32_t* s_cand = stage + T;
+  if constexpr (STAGED) {
+    for (int t = threadIdx.x; t < T; t += blockDim.x) s_p[t] = __float_as_uint(prow[t]);
+    for (int w = threadIdx.x; w < W; w += blockDim.x) s_cand[w] = cand_word(w);
+    __syncthreads();
+  }
   auto is_cand = [&](int t) -> bool {
-    const bool m = (member[(size_t)t * Ew + wi] & wmask) != 0u;
-    return up ? !m : m;
+    const uint32_t cw = STAGED ? s_cand[t >> 5] : cand_word(t >> 5);
+    return (cw >> (t & 31)) & 1u;
   };
   auto key_of = [&](int t) -> unsigned long long {
-    const unsigned long long kk =
-        ((unsigned long long)__float_as_uint(probs[(size_t)t * E + e]) << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)t);
+    const uint32_t pb = STAGED ? s_p[t] : __float_as_uint(prow[t]);
+    const unsigned long long kk = ((unsigned long long)pb << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)t);
     return up ? ~kk : kk;   // select the k smallest of this key
   };
+  __shared__ int s_done;
   unsigned long long prefix = 0ull, mask = 0ull;
   int kk = k;
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
-      if (!is_cand(t)) continue;
-      const unsigned long long key = key_of(t);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255ull], 1u);
+    for (int t0 = 0; t0 < T; t0 += blockDim.x) {  // warp-uniform trip count
+      const int t = t0 + threadIdx.x;
+      bool hit = false;
+      uint32_t digit = 0u;
+      if (t < T && is_cand(t)) {
+        const unsigned long long key = key_of(t);
+        hit = (key & mask) == prefix;
+        digit = (uint32_t)((key >> shift) & 255ull);
+      }
+      const uint32_t active = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        const uint32_t peers = __match_any_sync(active, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+      }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int cum = 0, dg = 0;
-      for (; dg < 256; ++dg) {
-        if (cum + (int)hist[dg] >= kk) break;
-        cum += (int)hist[dg];
+    if (threadIdx.x < 32) {  // warp 0: first digit whose running count reaches kk
+      int loc[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        loc[i] = (int)hist[8 * lane + i];
+        sum += loc[i];
       }
-      s_prefix = prefix | ((unsigned long long)dg << shift);
-      s_k = kk - cum;
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t reach = __ballot_sync(0xffffffffu, incl >= kk);
+      const int owner = __ffs(reach) - 1;  // kk <= number of matching candidates, so some lane reaches it
+      if (lane == owner) {
+        int cum = incl - sum, dg = 8 * lane;
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i, ++dg) {
+          if (cum + loc[i] >= kk) break;
+          cum += loc[i];
+        }
+        const int left = kk - cum;
+        s_prefix = prefix | ((unsigned long long)dg << shift);
+        s_k = left;
+        // once the p bits are fixed (after 4 passes), stop if every candidate
+        // with that p is selected: the token bits only break ties
+        s_done = (shift == 32 && left == (int)hist[dg]) ? 1 : 0;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
     kk = s_k;
     mask |= 255ull << shift;
+    const bool done = s_done != 0 && shift == 32;
     __syncthreads();
-  }
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    if (!is_cand(t)) continue;
-    if (key_of(t) <= prefix) {
-      if (up) atomicOr(&final_[(size_t)t * Ew + wi], wmask);
-      else atomicAnd(&final_[(size_t)t * Ew + wi], ~wmask);
+    if (done) {
+      prefix |= 0xFFFFFFFFull;  // select every candidate whose p bits are <= the k-th one's
+      break;
     }
+  }
+  // the selected candidates are those with key <= prefix (exactly k of them)
+  for (int w = threadIdx.x; w < W; w += blockDim.x) {
+    uint32_t sel = 0u;
+    const uint32_t cw = STAGED ? s_cand[w] : cand_word(w);
+    for (uint32_t m = cw; m; m &= m - 1u) {
+      const int b = __ffs(m) - 1;
+      if (key_of(w * 32 + b) <= prefix) sel |= 1u << b;
+    }
+    const uint32_t mem = mrow[w];
+    frow[w] = up ? (mem | sel) : (mem & ~sel);
   }
 }
 
-__global__ void tr_count_kernel(const uint32_t* final_, int T, int Ew, int* cnt) {
+// A warp holds 32 consecutive tokens (one word column w of finalT).  For each
+// group of 32 experts, lane j loads expert (32 c + j)'s word and 32 ballots
+// transpose the 32 x 32 bit block, so that lane i ends with the group's
+// expert mask of token 32 w + i.
+__device__ __forceinline__ uint32_t tr_token_mask(const uint32_t* finalT, int E, int W, int w, int c, int lane) {
+  const int e = 32 * c + lane;
+  const uint32_t x = (e < E && w < W) ? finalT[(size_t)e * W + w] : 0u;
+  uint32_t mine = 0u;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (x >> i) & 1u);
+    if (lane == i) mine = b;
+  }
+  return mine;
+}
+
+// Per token: its expert count after rounding; a block-wide exclusive scan
+// gives its offset inside the block, and the last block to finish scans the
+// block totals (exclusive, total at [nblocks]).
+__global__ void __launch_bounds__(256) tr_count_kernel(const uint32_t* finalT, int T, int E, int W, int* local,
+                                                       int* blk, int* sync) {
+  __shared__ int sh[8];
+  __shared__ int is_last;
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
   int c = 0;
-  for (int w = 0; w < Ew; ++w) c += __popc(final_[(size_t)t * Ew + w]);
-  cnt[t] = c;
-}
-
-__global__ void __launch_bounds__(1024) tr_ptr_scan_kernel(const int* cnt, int T, int* tok_ptr) {
-  __shared__ int sh[33];
-  const int per = (T + 1023) / 1024;
-  const int t0 = threadIdx.x * per;
-  int local = 0;
-  for (int t = t0; t < t0 + per && t < T; ++t) local += cnt[t];
+  for (int g = 0; g < (E + 31) / 32; ++g) c += __popc(tr_token_mask(finalT, E, W, t >> 5, g, lane));
+  if (t >= T) c = 0;
   int total;
-  int run = block_exclusive_scan_1024(local, sh, &total);
-  for (int t = t0; t < t0 + per && t < T; ++t) {
-    tok_ptr[t] = run;
-    run += cnt[t];
+  const int ex = block_exclusive_scan_256(c, sh, &total);
+  if (t < T) local[t] = ex;
+  if (threadIdx.x == 0) blk[blockIdx.x] = total;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(sync, 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int nb = gridDim.x;
+  int carry = 0;
+  for (int b0 = 0; b0 < nb; b0 += blockDim.x) {
+    const int b = b0 + threadIdx.x;
+    const int v = b < nb ? __ldcg(blk + b) : 0;
+    int tot;
+    const int bex = block_exclusive_scan_256(v, sh, &tot);
+    if (b < nb) blk[b] = carry + bex;
+    carry += tot;
   }
-  if (threadIdx.x == 0) tok_ptr[T] = total;
+  if (threadIdx.x == 0) blk[nb] = carry;
 }
 
-__global__ void tr_write_kernel(const uint32_t* final_, const float* probs, int T, int E, int Ew,
-                                const int* tok_ptr, int* pair_expert, float* pair_gate) {
+// Per token: tok_ptr and its pairs in ascending expert order, gates = p
+// renormalised over the token's final expert set.
+__global__ void __launch_bounds__(256) tr_write_kernel(const uint32_t* finalT, const float* probs, int T, int E,
+                                                       int W, const int* local, const int* blk, int* tok_ptr,
+                                                       int* pair_expert, float* pair_gate) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  const uint32_t* f = final_ + (size_t)t * Ew;
-  const float* pr = probs + (size_t)t * E;
+  const int lane = threadIdx.x & 31;
+  const bool live = t < T;
+  int p = live ? blk[blockIdx.x] + local[t] : 0;
+  if (live) {
+    tok_ptr[t] = p;
+    if (t == T - 1) tok_ptr[T] = blk[gridDim.x];
+  }
+  const float* pr = probs + (size_t)(live ? t : 0) * E;
+  const int groups = (E + 31) / 32;
   float sum = 0.f;
-  for (int w = 0; w < Ew; ++w)
-    for (uint32_t m = f[w]; m; m &= m - 1u) sum += pr[w * 32 + __ffs(m) - 1];
+  for (int g = 0; g < groups; ++g) {
+    const uint32_t m = tr_token_mask(finalT, E, W, t >> 5, g, lane);
+    if (live)
+      for (uint32_t r = m; r; r &= r - 1u) sum += pr[32 * g + __ffs(r) - 1];
+  }
   const float inv = sum > 0.f ? 1.0f / sum : 0.f;
-  int p = tok_ptr[t];
-  for (int w = 0; w < Ew; ++w)
-    for (uint32_t m = f[w]; m; m &= m - 1u) {
-      const int e = w * 32 + __ffs(m) - 1;
-      pair_expert[p] = e;
-      pair_gate[p] = pr[e] * inv;
-      ++p;
-    }
+  for (int g = 0; g < groups; ++g) {
+    const uint32_t m = tr_token_mask(finalT, E, W, t >> 5, g, lane);
+    if (live)
+      for (uint32_t r = m; r; r &= r - 1u) {
+        const int e = 32 * g + __ffs(r) - 1;
+        pair_expert[p] = e;
+        pair_gate[p] = pr[e] * inv;
+        ++p;
+      }
+  }
 }
+
+constexpr size_t kTrStageMax = 200 * 1024;  // dynamic shared memory of the staged select
 
 cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStream_t s) {
-  const size_t mbytes = (size_t)r.T * r.Ew * sizeof(uint32_t);
-  cudaError_t err = cudaMemsetAsync(r.member, 0, mbytes, s);
+  const int W = (r.T + 31) / 32;
+  cudaError_t err = cudaMemsetAsync(r.memberT, 0, (size_t)r.E * W * sizeof(uint32_t), s);
   if (err != cudaSuccess) return err;
   const int tb = (r.T + 255) / 256;
   {
     ProfScope ps(s, "round_member");
-    tr_member_kernel<<<tb, 256, 0, s>>>(a.tok_ptr, a.pair_expert, r.T, r.Ew, r.member);
+    tr_member_kernel<<<tb, 256, 0, s>>>(a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.sync);
   }
-  err = cudaMemcpyAsync(r.final_, r.member, mbytes, cudaMemcpyDeviceToDevice, s);
-  if (err != cudaSuccess) return err;
+  {
+    ProfScope ps(s, "round_transpose");
+    dim3 grid((r.E + 31) / 32, (r.T + 31) / 32), block(32, 8);
+    tr_transpose_kernel<<<grid, block, 0, s>>>(r.probs, r.probsT, r.T, r.E);
+  }
   {
     ProfScope ps(s, "round_select");
-    tr_select_kernel<<<r.E, 1024, 0, s>>>(r.T, r.E, r.Ew, r.mode, r.seed, a.counts, r.probs, r.member, r.final_);
+    // stage the expert's p row and candidate mask when they fit in shared memory
+    const size_t staged = ((size_t)r.T + (size_t)W) * sizeof(uint32_t);
+    if (staged <= kTrStageMax) {
+      static bool configured = false;  // one device per process, as for the GEMM kernels
+      if (!configured) {
+        err = cudaFuncSetAttribute(tr_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kTrStageMax);
+        if (err != cudaSuccess) return err;
+        configured = true;
+      }
+      tr_select_kernel<true><<<r.E, 1024, staged, s>>>(r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
+                                                        r.finalT);
+    } else {
+      tr_select_kernel<false><<<r.E, 1024, 0, s>>>(r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
+                                                    r.finalT);
+    }
   }
   {
     ProfScope ps(s, "round_count");
-    tr_count_kernel<<<tb, 256, 0, s>>>(r.final_, r.T, r.Ew, r.cnt);
-  }
-  {
-    ProfScope ps(s, "round_scan");
-    tr_ptr_scan_kernel<<<1, 1024, 0, s>>>(r.cnt, r.T, a.tok_ptr);
+    tr_count_kernel<<<tb, 256, 0, s>>>(r.finalT, r.T, r.E, W, r.local, r.blk, r.sync);
   }
   {
     ProfScope ps(s, "round_write");
-    tr_write_kernel<<<tb, 256, 0, s>>>(r.final_, r.probs, r.T, r.E, r.Ew, a.tok_ptr, a.pair_expert, a.pair_gate);
+    tr_write_kernel<<<tb, 256, 0, s>>>(r.finalT, r.probs, r.T, r.E, W, r.local, r.blk, a.tok_ptr, a.pair_expert,
+                                       a.pair_gate);
   }
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;

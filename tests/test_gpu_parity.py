@@ -74,9 +74,11 @@ def test_expert_only_gradient_without_router_path():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("mode", [1, 2])
-def test_token_rounding_parity(mode):
-    cfg = MoEConfig("tr", T=2048, d=128, E=16, n=64, K=2, w_std=0.05, bias="normal", seed=21)
+@pytest.mark.parametrize("mode,T", [(1, 2048), (2, 2048), (2, 53248)])
+def test_token_rounding_parity(mode, T):
+    """T = 53248: an expert's column of p no longer fits in shared memory, so
+    the selection reads it from global memory in every pass."""
+    cfg = MoEConfig("tr", T=T, d=128, E=16, n=64, K=2, w_std=0.05, bias="normal", seed=21)
     seed = 1234
     inp = make_inputs(cfg, "cuda")
     layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=mode, seed=seed)
