@@ -300,7 +300,10 @@ def main():
     per = {}
     for name, t in recs_all:
         per.setdefault(name, []).append(t)
-    dom = max(per, key=lambda k: sum(per[k]))
+    # the dominant kernel among those whose algorithmic work is known (the
+    # roofline needs it); every kernel still appears in the breakdown
+    work0 = kernel_work(cfg, R)
+    dom = max((k for k in per if k in work0), key=lambda k: sum(per[k]))
 
     # ---- device-timed region
     vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
