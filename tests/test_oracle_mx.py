@@ -1,0 +1,128 @@
+"""Pins of the MXFP8 oracle against the format's definition (OCP Microscaling
+formats: E4M3 elements, E8M0 block scales of 32) and plain mathematics --
+nothing here re-derives a value through the function under test."""
+import numpy as np
+
+from oracle import moe_oracle as mo
+from oracle import mx_oracle as mx
+
+
+def test_e4m3_table_matches_the_closed_form():
+    # hand-computed values from the bit layout S.EEEE.MMM, bias 7
+    known = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5, 0x38: 1.0,
+             0x39: 1.125, 0x40: 2.0, 0x4E: 4 * 1.75, 0x7E: 448.0, 0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0}
+    for c, v in known.items():
+        assert mx.e4m3_decode(c) == v, hex(c)
+    assert np.isnan(mx.e4m3_decode(0x7F)) and np.isnan(mx.e4m3_decode(0xFF))
+    mags = mx.e4m3_decode(np.arange(0x7F))
+    assert np.all(np.diff(mags) > 0)                      # strictly increasing magnitudes
+    # normals: consecutive codes inside a binade differ by 2^(e-7)/8
+    for ex in range(1, 16):
+        codes = np.arange(ex * 8, min(ex * 8 + 8, 0x7F))
+        assert np.allclose(np.diff(mx.e4m3_decode(codes)), 2.0 ** (ex - 7) / 8)
+
+
+def test_every_finite_code_round_trips():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F])
+    np.testing.assert_array_equal(mx.e4m3_encode(mx.e4m3_decode(codes)), codes)
+
+
+def test_rounding_is_to_nearest_with_ties_to_even():
+    mags = mx.e4m3_decode(np.arange(0x7F))
+    mid = (mags[:-1] + mags[1:]) / 2                      # exact midpoints
+    got = mx.e4m3_encode(mid)
+    even = np.where(np.arange(1, 0x7F) % 2 == 0, np.arange(1, 0x7F), np.arange(0, 0x7E))
+    np.testing.assert_array_equal(got, even)
+    # a hair off the midpoint goes to the nearer neighbour
+    np.testing.assert_array_equal(mx.e4m3_encode(mid * (1 + 1e-9)), np.arange(1, 0x7F))
+    np.testing.assert_array_equal(mx.e4m3_encode(mid[1:] * (1 - 1e-9)), np.arange(1, 0x7E))
+    # saturation and signed zero
+    np.testing.assert_array_equal(mx.e4m3_encode([449.0, 1e30, -1e30]), [0x7E, 0x7E, 0xFE])
+    np.testing.assert_array_equal(mx.e4m3_encode([-(2.0 ** -11), 0.0, -0.0]), [0x80, 0x00, 0x80])
+
+
+def test_scale_rule_is_the_smallest_non_saturating_exponent():
+    rng = np.random.default_rng(1)
+    amax = np.concatenate([rng.lognormal(0, 6, 2000), [448.0, 449.0, 1.0, 1.75, 1.7500001, 2.0 ** -120]])
+    e = mx.scale_exponent(amax)
+    # brute force over exponents: amax <= 448 2^e and not amax <= 448 2^(e-1)
+    assert np.all(amax <= 448.0 * np.exp2(e.astype(float)))
+    assert np.all(amax > 448.0 * np.exp2(e.astype(float) - 1))
+    assert mx.scale_exponent(0.0) == -127 and mx.scale_code(0.0) == 0
+
+
+def test_block_quantization_error_bound():
+    rng = np.random.default_rng(2)
+    M = rng.standard_normal((64, 256)) * np.exp2(rng.integers(-20, 20, (64, 1)))
+    codes, sc = mx.mx_quantize(M)
+    D = mx.mx_dequantize(codes, sc)
+    X = np.repeat(mx.scale_value(sc), mx.BLOCK, axis=-1)
+    # half a unit in the last place: 2^-4 relative for normals, 2^-10 X below 2^-6 X
+    bound = np.maximum(np.abs(M) * 2.0 ** -4, X * 2.0 ** -10)
+    assert np.all(np.abs(D - M) <= bound)
+    assert np.all(np.abs(M) <= 448.0 * X)                 # nothing saturates
+
+
+def test_power_of_two_scaling_moves_only_the_scales():
+    rng = np.random.default_rng(3)
+    M = rng.standard_normal((8, 128))
+    c0, s0 = mx.mx_quantize(M)
+    for k in (-5, 3, 17):
+        c1, s1 = mx.mx_quantize(M * 2.0 ** k)
+        np.testing.assert_array_equal(c1, c0)
+        np.testing.assert_array_equal(s1.astype(int), s0.astype(int) + k)
+
+
+def _layer(T, d, E, n, K, seed, integer=False):
+    rng = np.random.default_rng(seed)
+    if integer:   # every 32-block holds +-15 and integers: quantization is exact
+        X = rng.integers(-15, 16, (T, d)).astype(float)
+        X[:, ::32] = 15
+        W1 = rng.integers(-15, 16, (E, d, 2 * n)).astype(float)
+        W1[:, ::32, :] = -15
+    else:
+        X = rng.standard_normal((T, d))
+        W1 = rng.standard_normal((E, d, 2 * n)) * 0.05
+    W2 = rng.standard_normal((E, n, d)) * 0.05
+    Wr = rng.standard_normal((d, E)) * 0.05
+    return X, Wr, W1, W2
+
+
+def test_representable_inputs_give_the_exact_up_projection():
+    X, Wr, W1, W2 = _layer(40, 64, 4, 32, 2, 4, integer=True)
+    np.testing.assert_array_equal(mx.mx_round(X), X)
+    fw = mo.forward(X, Wr, None, W1, W2, 2)
+    fq = mx.forward_mxfp8(X, Wr, None, W1, W2, 2)
+    np.testing.assert_array_equal(fq["H"], fw["H"])
+    np.testing.assert_array_equal(fq["A"], fw["A"])
+
+
+def test_dense_case_matches_plain_matmuls():
+    # E = 1, K = 1: one expert with gate 1, so the layer is a dense MLP on the
+    # quantized operands, written out here with numpy alone
+    X, Wr, W1, W2 = _layer(33, 64, 1, 64, 1, 5)
+    fq = mx.forward_mxfp8(X, Wr, None, W1, W2, 1)
+
+    def q(M, axis):   # quantize along `axis` in blocks of 32, then back
+        Mt = np.moveaxis(M, axis, -1)
+        B = Mt.reshape(Mt.shape[:-1] + (-1, 32))
+        am = np.abs(B).max(-1)
+        f, Ex = np.frexp(am)
+        e = (Ex - 1) - 8 + (2 * f > 1.75)
+        S = np.exp2(e)[..., None]
+        return np.moveaxis((mx.e4m3_decode(mx.e4m3_encode(B / S)) * S).reshape(Mt.shape), -1, axis)
+
+    H = q(X, 1) @ q(W1[0], 0)
+    g, u = H[:, :64], H[:, 64:]
+    A = g / (1 + np.exp(-g)) * u
+    O = q(A, 1) @ q(W2[0], 0)
+    np.testing.assert_allclose(fq["O"], O, rtol=1e-12, atol=1e-12)
+
+
+def test_quantized_forward_stays_near_the_exact_forward():
+    X, Wr, W1, W2 = _layer(64, 128, 8, 64, 2, 6)
+    fw = mo.forward(X, Wr, None, W1, W2, 2)
+    fq = mx.forward_mxfp8(X, Wr, None, W1, W2, 2)
+    rel = np.abs(fq["O"] - fw["O"]).max() / np.abs(fw["O"]).max()
+    # three 3-bit-mantissa roundings on the path to O: a few percent, not more
+    assert 1e-4 < rel < 0.1, rel
