@@ -645,6 +645,27 @@ moe_status moe_get_status(void* stream, int32_t* where) {
   return static_cast<moe_status>(h[0]);
 }
 
+moe_status moe_mx_quantize_rows(const void* in, int64_t rows, int32_t K, void* codes, void* scales, void* stream) {
+  if (rows < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (K % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes) || !aligned16(scales))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY_CUDA(launch_mx_quant_rows(static_cast<const __nv_bfloat16*>(in), rows, K, static_cast<uint8_t*>(codes),
+                                    static_cast<uint8_t*>(scales), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_mx_quantize_cols(const void* in, int32_t E, int32_t K, int32_t N, void* codes, void* scales,
+                                void* stream) {
+  if (E < 0 || K <= 0 || N < 0) return MOE_ERR_INVALID_ARG;
+  if (K % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes) || !aligned16(scales))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(in), E, K, N, static_cast<uint8_t*>(codes),
+                                    static_cast<uint8_t*>(scales), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_set_sm_budget(int32_t sms) {
   if (sms < 0) return MOE_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);

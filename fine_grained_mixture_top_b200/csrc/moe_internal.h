@@ -90,4 +90,12 @@ cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* p
 cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const __nv_bfloat16* dXt,
                                  __nv_bfloat16* dX, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
+
+// ---- MXFP8 quantization (moe_mx.cu)
+cudaError_t launch_mx_quant_rows(const __nv_bfloat16* in, int64_t rows, int K, uint8_t* codes, uint8_t* scales,
+                                 cudaStream_t s);
+cudaError_t launch_mx_quant_cols(const __nv_bfloat16* in, int E, int K, int N, uint8_t* codes, uint8_t* scales,
+                                 cudaStream_t s);
+cudaError_t launch_mx_scale_tiles(const uint8_t* scales, int E, int K, int N, int split_half, uint8_t* tiles,
+                                  cudaStream_t s);
 }  // namespace moe

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
                                       P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       ctypes.c_size_t, P(c_void_p), c_void_p]
         L.moe_set_sm_budget.argtypes = [c_int32]
+        L.moe_mx_quantize_rows.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
+        L.moe_mx_quantize_cols.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
         L.moe_get_status.argtypes = [c_void_p, P(c_int32)]
         L.moe_set_spin_limit.argtypes = [c_int64]
         L.moe_selftest_wait_timeout.argtypes = [c_void_p, c_void_p]
@@ -96,7 +98,7 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
                   "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout", "moe_backward_ev",
-                  "moe_set_sm_budget"):
+                  "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols"):
             getattr(L, f).restype = c_int32
         _lib = L
     return _lib
@@ -210,6 +212,30 @@ def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW
             e.record()
     evs = (c_void_p * 3)(*[None if e is None else e.cuda_event for e in grad_events])
     _check(lib().moe_backward_ev(*args, evs, _stream(stream)), "moe_backward_ev")
+
+
+def mx_quantize_rows(x, stream=None):
+    """x [rows, K] bf16 (device) -> (codes [rows, K] uint8, scales [rows, K/32]
+    uint8): MXFP8 along each row."""
+    import torch
+    rows, K = x.shape
+    codes = torch.empty(rows, K, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(rows, K // 32, dtype=torch.uint8, device=x.device)
+    _check(lib().moe_mx_quantize_rows(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_mx_quantize_rows")
+    return codes, scales
+
+
+def mx_quantize_cols(w, stream=None):
+    """w [E, K, N] bf16 (device) -> (codes [E, N, K] uint8, scales [E, N, K/32]
+    uint8): MXFP8 along K for each column, transposed so that K is contiguous."""
+    import torch
+    E, K, N = w.shape
+    codes = torch.empty(E, N, K, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(E, N, K // 32, dtype=torch.uint8, device=w.device)
+    _check(lib().moe_mx_quantize_cols(_ptr(w), E, K, N, _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_mx_quantize_cols")
+    return codes, scales
 
 
 def moe_set_sm_budget(sms: int):

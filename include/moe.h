@@ -192,6 +192,26 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
 moe_status moe_set_sm_budget(int32_t sms);
 
 /*
+ * MXFP8 quantization (the pages list MXFP8 precision as future work of the
+ * method, page "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE", closing
+ * paragraph; the format is the OCP Microscaling definition): E4M3 codes with
+ * one E8M0 scale per 32 consecutive elements along K, the scale being the
+ * smallest power of two at which no element of the block saturates.
+ *
+ * moe_mx_quantize_rows: in[rows, K] bf16 -> codes[rows, K] u8 and
+ *   scales[rows, K/32] u8, quantized along each row.
+ * moe_mx_quantize_cols: in[E, K, N] bf16 (an expert weight stack, K rows) ->
+ *   codes[E, N, K] u8 (transposed: K contiguous) and scales[E, N, K/32] u8,
+ *   quantized along K for each column.
+ * K must be a multiple of 32 (MOE_ERR_UNSUPPORTED otherwise); pointers must
+ * be 16-byte aligned device pointers (MOE_ERR_INVALID_ARG).  Asynchronous on
+ * `stream`.
+ */
+moe_status moe_mx_quantize_rows(const void* in, int64_t rows, int32_t K, void* codes, void* scales, void* stream);
+moe_status moe_mx_quantize_cols(const void* in, int32_t E, int32_t K, int32_t N, void* codes, void* scales,
+                                void* stream);
+
+/*
  * Synchronises `stream`, returns the device status word (MOE_OK if no kernel
  * reported an error since the last call) and clears it.  *where (nullable)
  * receives the code of the wait or check that failed.

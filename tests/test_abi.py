@@ -86,6 +86,9 @@ def test_invalid_options_and_null_arguments(moe):
     assert L.moe_set_sm_budget(0) == 0
     assert L.moe_backward_ev(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, None, None,
                              ctypes.byref(rt), None, None, None, None, None, None, 0, None, None) == 1
+    assert L.moe_mx_quantize_rows(None, 4, 32, None, None, None) == 1
+    assert L.moe_mx_quantize_rows(None, 4, 48, None, None, None) == 2     # K not a multiple of 32
+    assert L.moe_mx_quantize_cols(None, 1, 64, 8, None, None, None) == 1
     assert moe.last_error() == ""  # no CUDA error on this thread
 
 
