@@ -13,6 +13,9 @@
 //   DW2  dW2[e] = A_hat^T dO[tok] (K runs over the rows of expert e; gather on B)
 //   RTR  router logits X Wr with Wr split into three bf16 parts (hi+mid+lo)
 //   DWR  router weight gradient X^T dz, dz split into two bf16 parts, split-K
+//   UPQ  UP with MXFP8 operands (E4M3 codes, one E8M0 scale per 32 K): the
+//        epilogue stores H (bf16) and A quantized to MXFP8 with its scales
+//   DOWNQ DOWN with MXFP8 operands
 //
 // Sources: page "SonicMoE：突破细粒度MoE硬件效率瓶颈，实现高稀疏性下的极致训练加速"
 // (implementation paragraph: grouped GEMMs with modular fusion, eight kernels);
@@ -31,11 +34,12 @@
 
 #include <type_traits>
 
+#include "mx.cuh"
 #include "ptx.cuh"
 
 namespace moe {
 
-enum GemmKind : int { G_UP = 0, G_DOWN, G_DH, G_DXT, G_DW1, G_DW2, G_RTR, G_DWR };
+enum GemmKind : int { G_UP = 0, G_DOWN, G_DH, G_DXT, G_DW1, G_DW2, G_RTR, G_DWR, G_UPQ, G_DOWNQ };
 
 struct GemmParams {
   CUtensorMap tmA;   // TMA map of A (kinds whose A is not gathered)
@@ -64,17 +68,25 @@ struct GemmParams {
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
+  // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
+  // K block of 128), the scale of row m, sub-block j at 16 (m % 32) + 4 (m / 32) + j.
+  const uint8_t* sfa_src;    // UPQ: X scales [T, d/32] (gathered per row); DOWNQ: A scale tiles [R_max/128][n/128]
+  const uint8_t* sfb_src;    // weight scale tiles [E][N tiles][K/128]
+  uint8_t* aq_out;           // UPQ: A codes [R_max, n]
+  uint8_t* sa_out;           // UPQ: A scale tiles [R_max/128][n/128]
 };
 
 template <int KIND>
 struct KindTraits {
-  static constexpr bool kGroupedM = (KIND == G_UP || KIND == G_DOWN || KIND == G_DH || KIND == G_DXT);
+  static constexpr bool kGroupedM =
+      (KIND == G_UP || KIND == G_DOWN || KIND == G_DH || KIND == G_DXT || KIND == G_UPQ || KIND == G_DOWNQ);
+  static constexpr bool kFp8 = (KIND == G_UPQ || KIND == G_DOWNQ);
   static constexpr bool kGroupedK = (KIND == G_DW1 || KIND == G_DW2);
-  static constexpr bool kAGather = (KIND == G_UP || KIND == G_DH || KIND == G_DW1);
+  static constexpr bool kAGather = (KIND == G_UP || KIND == G_DH || KIND == G_DW1 || KIND == G_UPQ);
   static constexpr bool kBGather = (KIND == G_DW2);
   static constexpr bool kGather = kAGather || kBGather;
   static constexpr bool kAMN = (KIND == G_DW1 || KIND == G_DW2 || KIND == G_DWR);
-  static constexpr bool kBMN = !(KIND == G_DH || KIND == G_DXT);
+  static constexpr bool kBMN = !(KIND == G_DH || KIND == G_DXT || KIND == G_UPQ || KIND == G_DOWNQ);
 };
 
 // Epilogue configuration: EPI = 4 or 8 epilogue warps.  With 8, two warps
@@ -91,7 +103,7 @@ struct EpiCfg {
   // dX~ kernel keeps 2 (so that its stage ring keeps its depth), while the
   // weight-gradient kinds, which get 8 warps when their tiles are store-bound
   // (few rows per expert), keep 4 bulk stores in flight per warp.
-  static constexpr int kBufs = (KIND == G_UP || KIND == G_DH)
+  static constexpr int kBufs = (KIND == G_UP || KIND == G_DH || KIND == G_UPQ)
                                    ? 3
                                    : (EPI == 8 ? (KindTraits<KIND>::kGroupedK ? 4 : 2) : 3);
   static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
@@ -120,15 +132,21 @@ constexpr int kTileQ = 4;        // depth of the dynamic scheduler's tile queue
 template <int KIND, int BN, int NBUF = 12>
 struct GemmShape {
   using KT = KindTraits<KIND>;
-  static constexpr bool kSplit = (KIND == G_UP || KIND == G_DH);
+  static constexpr bool kSplit = (KIND == G_UP || KIND == G_DH || KIND == G_UPQ);
+  // B slot: BN rows of 128 bytes (64 bf16 or 128 fp8 K elements)
   static constexpr int kBBytes = BN * kBK * 2;
+  // MXFP8 kinds: one 512-byte scale tile per A slot and per 128 rows of a B slot
+  static constexpr int kSFABytes = KT::kFp8 ? 512 : 0;
+  static constexpr int kSFBBytes = KT::kFp8 ? 512 * (BN / 128) : 0;
+  static constexpr int kASlot = kABytes + kSFABytes;  // budget per A slot
+  static constexpr int kBSlot = kBBytes + kSFBBytes;  // budget per B slot
   static constexpr int kStoreBytes = NBUF * kStoreBuf;  // epilogue staging: NBUF buffers of 2 KB
   static constexpr int kBudget = (kSmemLimit - 2048 - kStoreBytes) < kStageBudget
                                      ? (kSmemLimit - 2048 - kStoreBytes) : kStageBudget;
   static constexpr int cap8(int x) { return x > 8 ? 8 : x; }
-  static constexpr int kStages = cap8(kBudget / (kABytes + kBBytes));  // one (A, B) ring
-  static constexpr int kSBs = (kBudget - 3 * kBBytes >= 5 * kABytes) ? (kBBytes >= 32768 ? 3 : 4) : 2;
-  static constexpr int kSA = kSplit ? cap8((kBudget - kSBs * kBBytes) / kABytes) : kStages;
+  static constexpr int kStages = cap8(kBudget / (kASlot + kBSlot));  // one (A, B) ring
+  static constexpr int kSBs = (kBudget - 3 * kBSlot >= 5 * kASlot) ? (kBBytes >= 32768 ? 3 : 4) : 2;
+  static constexpr int kSA = kSplit ? cap8((kBudget - kSBs * kBSlot) / kASlot) : kStages;
   static constexpr int kSB = kSplit ? kSBs : kStages;
   // cp.async publication lag of a gathered operand (k-blocks in flight per
   // thread = lag + 1; the MMA keeps ring - lag - 1 published k-blocks queued)
@@ -137,11 +155,17 @@ struct GemmShape {
   static constexpr int kBOffset = kSA * kABytes;
   // accumulator buffers start at power-of-two column offsets
   static constexpr int kAccStride = BN <= 64 ? 64 : (BN <= 128 ? 128 : 256);
-  static constexpr int kTmemCols = 2 * kAccStride;
-  static constexpr int kStoreOffset = kBOffset + kSB * kBBytes;  // epilogue staging
+  // MXFP8: the scale factors live in TMEM after the two accumulators
+  static constexpr int kSFACol = 2 * kAccStride;      // 4 columns
+  static constexpr int kSFBCol = 2 * kAccStride + 4;  // 4 columns per 128 B rows
+  static constexpr int kTmemCols = KT::kFp8 ? 512 : 2 * kAccStride;
+  static constexpr int kSFAOffset = kBOffset + kSB * kBBytes;      // MXFP8 scale-tile rings
+  static constexpr int kSFBOffset = kSFAOffset + kSA * kSFABytes;
+  static constexpr int kStoreOffset = kSFBOffset + kSB * kSFBBytes;  // epilogue staging
   static constexpr int kBarOffset = kStoreOffset + kStoreBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;  // barriers + alignment slack
   static_assert(kSA >= 2 && kSB >= 2 && kSA <= 8 && kSB <= 8, "ring depths");
+  static_assert(!KT::kFp8 || (BN == 128 && kSFBCol + 4 * (BN / 128) <= kTmemCols), "MXFP8 tiles are 128 wide");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
@@ -174,10 +198,11 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
     t.nt = tile - t.mt * p.num_n_tiles;
     t.e = __ldg(p.tile_expert + t.mt);
     t.m0 = t.mt * kBM;
-    if constexpr (KIND == G_UP) t.n0 = t.nt * (BN / 2);
+    if constexpr (KIND == G_UP || KIND == G_UPQ) t.n0 = t.nt * (BN / 2);
     else t.n0 = t.nt * BN;
-    const int K = (KIND == G_UP || KIND == G_DH) ? p.d : (KIND == G_DOWN ? p.n : 2 * p.n);
-    t.nkb = K / kBK;
+    const int K = (KIND == G_UP || KIND == G_DH || KIND == G_UPQ) ? p.d
+                  : ((KIND == G_DOWN || KIND == G_DOWNQ) ? p.n : 2 * p.n);
+    t.nkb = KT::kFp8 ? K / 128 : K / kBK;  // a k-block is 128 bytes of K per row
   } else if constexpr (KT::kGroupedK) {
     const int per_e = p.num_m_tiles * p.num_n_tiles;
     const int ei = tile / per_e;
@@ -223,15 +248,20 @@ __device__ __forceinline__ uint32_t sw128(int line, int chunk) {
 // (completing on bar_b); an operand the gather warps stream is skipped.
 template <int KIND, int BN>
 __device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t, int kb, uint32_t a_s,
-                                          uint32_t bar_a, uint32_t b_s, uint32_t bar_b) {
+                                          uint32_t bar_a, uint32_t b_s, uint32_t bar_b, uint32_t sfa_s,
+                                          uint32_t sfb_s) {
   const void* tA = &p.tmA;
   const void* tB = &p.tmB;
   const int k0 = kb * kBK;
   constexpr int nb = BN / 64;
+  using SHp = GemmShape<KIND, BN>;
   // one ring: a single arrive.expect_tx covers both operands' bytes
-  constexpr bool kOne = !GemmShape<KIND, BN>::kSplit;
-  constexpr uint32_t kTxA = (KIND == G_UP || KIND == G_DH || KIND == G_DW1) ? 0u : (uint32_t)kABytes;
-  constexpr uint32_t kTxB = (KIND == G_DW2) ? 0u : (uint32_t)(nb * kBoxBytes);
+  constexpr bool kOne = !SHp::kSplit;
+  constexpr uint32_t kTxA = (KIND == G_UP || KIND == G_DH || KIND == G_DW1 || KIND == G_UPQ)
+                                ? 0u : (uint32_t)(kABytes + SHp::kSFABytes);
+  constexpr uint32_t kTxB = (KIND == G_DW2) ? 0u : (uint32_t)(nb * kBoxBytes + SHp::kSFBBytes);
+  (void)sfa_s;
+  (void)sfb_s;
   if constexpr (kOne) {
     mbar_arrive_expect_tx(bar_a, kTxA + kTxB);
     bar_b = bar_a;
@@ -269,6 +299,22 @@ __device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t
   } else if constexpr (KIND == G_DW2) {
     expect_a(2 * kBoxBytes);
     for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar_a, t.m0 + 64 * h, t.krow0 + k0);
+  } else if constexpr (KIND == G_UPQ) {
+    // W1 codes transposed [E * 2n rows, d bytes]: 64 gate rows, then the
+    // same 64 up rows; the scale tile of (expert, N tile, K block)
+    const int x = kb * 128;
+    expect_b((uint32_t)(BN * 128 + SHp::kSFBBytes));
+    tma_load_2d(b_s, tB, bar_b, x, t.e * 2 * p.n + t.n0);
+    tma_load_2d(b_s + 64 * 128, tB, bar_b, x, t.e * 2 * p.n + p.n + t.n0);
+    bulk_load(sfb_s, p.sfb_src + ((size_t)(t.e * p.num_n_tiles + t.nt) * (p.d / 128) + kb) * 512, 512, bar_b);
+  } else if constexpr (KIND == G_DOWNQ) {
+    // A codes [R_max, n bytes] and its scale tiles; W2 codes transposed
+    // [E * d rows, n bytes] and their scale tiles
+    const int x = kb * 128;
+    tma_load_2d(a_s, tA, bar_a, x, t.m0);
+    bulk_load(sfa_s, p.sfa_src + ((size_t)t.mt * (p.n / 128) + kb) * 512, 512, bar_a);
+    tma_load_2d(b_s, tB, bar_a, x, t.e * p.d + t.n0);
+    bulk_load(sfb_s, p.sfb_src + ((size_t)(t.e * (p.d / 128) + t.nt) * (p.n / 128) + kb) * 512, 512, bar_a);
   } else if constexpr (KIND == G_RTR) {
     expect_a(kABytes);
     tma_load_2d(a_s, tA, bar_a, k0, t.m0);
@@ -404,7 +450,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    if constexpr (!(KIND == G_UP || KIND == G_DH || KIND == G_DW1)) tma_prefetch_desc(&p.tmA);
+    if constexpr (!KT::kAGather) tma_prefetch_desc(&p.tmA);
     if constexpr (!KT::kBGather) tma_prefetch_desc(&p.tmB);
   }
   if (warp == 1) {
@@ -476,7 +522,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
               break;
             }
           }
-          issue_tma<KIND, BN>(p, t, kb, a_slot(sa), smem_u32(&full_a[sa]), b_slot(sb), smem_u32(&full_b[sb]));
+          issue_tma<KIND, BN>(p, t, kb, a_slot(sa), smem_u32(&full_a[sa]), b_slot(sb), smem_u32(&full_b[sb]),
+                              base + SH::kSFAOffset + (uint32_t)(sa * SH::kSFABytes),
+                              base + SH::kSFBOffset + (uint32_t)(sb * SH::kSFBBytes));
         }
       }
     }
@@ -569,13 +617,30 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         if (lane == 0) {
           const uint32_t a_s = a_slot(sa);
           const uint32_t b_s = b_slot(sb);
+          if constexpr (KT::kFp8) {
+            // scale tiles into TMEM (in issue order with the MMAs that read them),
+            // then 4 MMAs of K = 32 fp8 elements, each with its scale byte
+            const uint32_t sfa_t = tmem_base + (uint32_t)SH::kSFACol;
+            const uint32_t sfb_t = tmem_base + (uint32_t)SH::kSFBCol;
+            tc_cp_32x128b_x4(sfa_t, smem_desc_rows16(base + SH::kSFAOffset + (uint32_t)(sa * SH::kSFABytes)));
+            tc_cp_32x128b_x4(sfb_t, smem_desc_rows16(base + SH::kSFBOffset + (uint32_t)(sb * SH::kSFBBytes)));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = KT::kAMN ? smem_desc_sw128(a_s + kk * 2048, kBoxBytes, 1024)
-                                         : smem_desc_sw128(a_s + kk * 32, 16, 1024);
-            const uint64_t bd = KT::kBMN ? smem_desc_sw128(b_s + kk * 2048, kBoxBytes, 1024)
-                                         : smem_desc_sw128(b_s + kk * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc_sw128(a_s + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(b_s + kk * 32, 16, 1024);
+              const uint32_t sel = (uint32_t)kk << 30;
+              tc_mma_mxf8(d_tmem, ad, bd, idesc_mxf8(BN, (uint32_t)kk, (uint32_t)kk), sfa_t | sel, sfb_t | sel,
+                          (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = KT::kAMN ? smem_desc_sw128(a_s + kk * 2048, kBoxBytes, 1024)
+                                           : smem_desc_sw128(a_s + kk * 32, 16, 1024);
+              const uint64_t bd = KT::kBMN ? smem_desc_sw128(b_s + kk * 2048, kBoxBytes, 1024)
+                                           : smem_desc_sw128(b_s + kk * 32, 16, 1024);
+              tc_mma_bf16(d_tmem, ad, bd, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit(smem_u32(&empty_a[sa]));
           if (kSplit) tc_commit(smem_u32(&empty_b[sb]));
@@ -770,7 +835,54 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
             bulk_commit();
           }
         }
-      } else if constexpr (KIND == G_DOWN || KIND == G_DXT || KT::kGroupedK) {
+      } else if constexpr (KIND == G_UPQ) {
+        // H (bf16, kept for the backward) through the staging boxes; A
+        // quantized per row in blocks of 32 to E4M3 codes with an E8M0 scale
+        // (the smallest exponent at which nothing saturates), the codes
+        // stored straight from registers, the two scales of this tile's 64
+        // columns into the scale tile of (M tile, K block t.n0 / 128)
+        constexpr int BNh = BN / 2;  // gate columns [0, BNh), up columns [BNh, BN)
+        const int r = t.m0 + rloc;
+        uint32_t sc2 = 0u;
+#pragma unroll 1
+        for (int c = 0; c < BNh; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tacc + c, g);
+          tmem_ld32(tacc + BNh + c, u);
+          tc_wait_ld();
+          float gv[32], uv[32], av[32];
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            gv[i] = bf16_round(__uint_as_float(g[i]));
+            uv[i] = bf16_round(__uint_as_float(u[i]));
+            av[i] = gv[i] * sigmoidf_(gv[i]) * uv[i];
+            amax = fmaxf(amax, fabsf(av[i]));
+          }
+          stage_wait(std::integral_constant<int, 0>{});
+          stage_row32(stg, lane, gv);
+          stage_row32(stg + kStoreBuf, lane, uv);
+          stage_publish();
+          if (lane == 0) {
+            tma_store_2d(&p.tmC0, stg, t.n0 + c, row0);
+            tma_store_2d(&p.tmC0, stg + kStoreBuf, p.n + t.n0 + c, row0);
+            bulk_commit();
+          }
+          const uint32_t code = mx_scale_code(amax);
+          const float sinv = mx_inv_scale(code);
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            w[i] = mx_e4m3x2(av[4 * i] * sinv, av[4 * i + 1] * sinv) |
+                   (mx_e4m3x2(av[4 * i + 2] * sinv, av[4 * i + 3] * sinv) << 16);
+          uint4* dst = reinterpret_cast<uint4*>(p.aq_out + (size_t)r * p.n + t.n0 + c);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          sc2 |= code << (8 * (c / 32));
+        }
+        *reinterpret_cast<uint16_t*>(p.sa_out + ((size_t)t.mt * (p.n / 128) + t.n0 / 128) * 512 +
+                                     16 * (rloc & 31) + 4 * (rloc >> 5) + (t.n0 % 128) / 32) = (uint16_t)sc2;
+      } else if constexpr (KIND == G_DOWN || KIND == G_DXT || KIND == G_DOWNQ || KT::kGroupedK) {
         int orow = row0;
         bool live = true;
         if constexpr (KT::kGroupedK) {
@@ -933,13 +1045,18 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       const int tile = consume_tile(ti, ok);
       if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
-      if constexpr (KIND == G_UP || KIND == G_DH) {
-        // A tile = 128 gathered rows x 64 columns; this thread: lines line0 + 16 j
+      if constexpr (KIND == G_UP || KIND == G_DH || KIND == G_UPQ) {
+        // A tile = 128 gathered rows x 128 bytes of K; this thread: lines
+        // line0 + 16 j (MXFP8: the codes are read as pairs of bytes, so the
+        // same 16-byte chunks apply; the chunk-0 threads also copy each row's
+        // 4 scale bytes of the k-block into the scale tile)
         const __nv_bfloat16* src[8];
         uint32_t nbytes[8];
+        int toks[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int tok = __ldg(p.row_tok + t.m0 + line0 + 16 * j);
+          toks[j] = tok;
           src[j] = p.gsrc + (size_t)(tok < 0 ? 0 : tok) * p.gld + chunk * 8;
           nbytes[j] = tok < 0 ? 0u : 16u;
         }
@@ -952,6 +1069,18 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           const uint32_t a_s = a_slot(s);
 #pragma unroll
           for (int j = 0; j < 8; ++j) cp_async_16(a_s + sw128(line0 + 16 * j, chunk), src[j] + kb * kBK, nbytes[j]);
+          if constexpr (KIND == G_UPQ) {
+            if (chunk == 0) {
+              const uint32_t sf_s = base + SH::kSFAOffset + (uint32_t)(s * SH::kSFABytes);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int r = line0 + 16 * j;
+                const int tok = toks[j];
+                const uint8_t* ssrc = p.sfa_src + (size_t)(tok < 0 ? 0 : tok) * (p.d / 32) + kb * 4;
+                cp_async_4(sf_s + 16 * (r & 31) + 4 * (r >> 5), ssrc, tok < 0 ? 0u : 4u);
+              }
+            }
+          }
           cp_async_commit();
           if (pending == kLag) {
             cp_async_wait<kLag>();

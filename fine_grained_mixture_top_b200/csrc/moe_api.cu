@@ -86,6 +86,18 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+// Byte matrix [rows, cols] (MXFP8 codes), 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                  uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 bool make_store_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return make_tmap(m, base, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
@@ -201,10 +213,37 @@ struct FwdWs {
   __nv_bfloat16* A;
   __nv_bfloat16* Y;
 };
+// MXFP8 forward: codes and scales of X, W1, W2 and A, and Y
+struct MxFwdWs {
+  uint8_t *Xq, *SX;            // [T, d], [T, d/32]
+  uint8_t *W1q, *SW1, *SW1t;   // [E, 2n, d], [E, 2n, d/32], scale tiles [E][n/64][d/128]
+  uint8_t *W2q, *SW2, *SW2t;   // [E, d, n], [E, d, n/32], scale tiles [E][d/128][n/128]
+  uint8_t *Aq, *SA;            // [R_max, n], scale tiles [R_max/128][n/128]
+  __nv_bfloat16* Y;            // [R_max, d]
+};
 size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
   Carve c{static_cast<char*>(ws)};
   w->A = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
   w->Y = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
+  return c.off;
+}
+
+bool mx_supported(const Plan& p) { return p.n % 128 == 0; }
+
+size_t carve_fwd_mx(const Plan& p, void* ws, MxFwdWs* w) {
+  Carve c{static_cast<char*>(ws)};
+  const size_t T = (size_t)p.T, d = p.d, n = p.n, E = p.E, R = (size_t)p.R_max;
+  w->Xq = c.take<uint8_t>(T * d);
+  w->SX = c.take<uint8_t>(T * (d / 32));
+  w->W1q = c.take<uint8_t>(E * 2 * n * d);
+  w->SW1 = c.take<uint8_t>(E * 2 * n * (d / 32));
+  w->SW1t = c.take<uint8_t>(E * (n / 64) * (d / 128) * 512);
+  w->W2q = c.take<uint8_t>(E * d * n);
+  w->SW2 = c.take<uint8_t>(E * d * (n / 32));
+  w->SW2t = c.take<uint8_t>(E * (d / 128) * (n / 128) * 512);
+  w->Aq = c.take<uint8_t>(R * n);
+  w->SA = c.take<uint8_t>((R / 128) * (n / 128) * 512);
+  w->Y = c.take<__nv_bfloat16>(R * d);
   return c.off;
 }
 
@@ -352,6 +391,8 @@ moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes
   out->fwd_ws = carve_fwd(p, nullptr, &fw);
   out->bwd_ws = carve_bwd(p, nullptr, &bw);
   out->h_elems = p.R_max * 2 * p.n;
+  MxFwdWs mw;
+  out->fwd_mx_ws = mx_supported(p) ? carve_fwd_mx(p, nullptr, &mw) : 0;
   return MOE_OK;
 }
 
@@ -478,6 +519,80 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
   {
     ProfScope ps(st, "aggregate_fwd");
     MOE_TRY_CUDA(launch_aggregate_fwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, rt->pair_gate, w.Y,
+                                      static_cast<__nv_bfloat16*>(O), st));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
+                             const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
+                             void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!mx_supported(p)) return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {X, W1, W2, O, H};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  MxFwdWs w;
+  if (!ws || ws_bytes < carve_fwd_mx(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_fwd_mx(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t mtiles = p.R_max / kTile;
+  const int E = p.E, d = p.d, n = p.n;
+
+  // operands to MXFP8: X along d per row; W1 along d and W2 along n per
+  // output column, transposed so that K is contiguous, with their scales
+  // rearranged into the MMA's 512-byte scale tiles
+  {
+    ProfScope ps(st, "mx_quant_x");
+    MOE_TRY_CUDA(launch_mx_quant_rows(static_cast<const __nv_bfloat16*>(X), p.T, d, w.Xq, w.SX, st));
+  }
+  {
+    ProfScope ps(st, "mx_quant_w");
+    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W1), E, d, 2 * n, w.W1q, w.SW1, st));
+    MOE_TRY_CUDA(launch_mx_scale_tiles(w.SW1, E, d, 2 * n, 1, w.SW1t, st));
+    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W2), E, n, d, w.W2q, w.SW2, st));
+    MOE_TRY_CUDA(launch_mx_scale_tiles(w.SW2, E, n, d, 0, w.SW2t, st));
+  }
+  // up-projection on MXFP8 operands: H = X[tok] W1[e] (bf16 out), A = SwiGLU(H)
+  // quantized to MXFP8 with its scale tiles
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap_u8(&g.tmB, w.W1q, (uint64_t)E * 2 * n, (uint64_t)d, 128, 64));
+    g.gsrc = reinterpret_cast<const __nv_bfloat16*>(w.Xq);  // rows of d bytes, gathered in 16-byte chunks
+    g.gld = d / 2;
+    g.sfa_src = w.SX;
+    g.sfb_src = w.SW1t;
+    g.num_n_tiles = n / 64;
+    g.out0 = static_cast<__nv_bfloat16*>(H);
+    g.aq_out = w.Aq;
+    g.sa_out = w.SA;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, H, (uint64_t)p.R_max, (uint64_t)2 * n));
+    ProfScope ps(st, "up_proj_gemm_mx");
+    MOE_TRY_CUDA(launch_gemm(G_UPQ, 128, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  // down-projection on MXFP8 operands: Y = A W2[e]
+  {
+    GemmParams g = base_params(p, rt, status);
+    MOE_TRY_MAP(make_tmap_u8(&g.tmA, w.Aq, (uint64_t)p.R_max, (uint64_t)n, 128, 128));
+    MOE_TRY_MAP(make_tmap_u8(&g.tmB, w.W2q, (uint64_t)E * d, (uint64_t)n, 128, 128));
+    g.sfa_src = w.SA;
+    g.sfb_src = w.SW2t;
+    g.num_n_tiles = d / 128;
+    g.out0 = w.Y;
+    MOE_TRY_MAP(make_store_map(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)d));
+    ProfScope ps(st, "down_proj_gemm_mx");
+    MOE_TRY_CUDA(launch_gemm(G_DOWNQ, 128, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+  }
+  {
+    ProfScope ps(st, "aggregate_fwd");
+    MOE_TRY_CUDA(launch_aggregate_fwd((int)p.T, d, rt->tok_ptr, rt->pair_row, rt->pair_gate, w.Y,
                                       static_cast<__nv_bfloat16*>(O), st));
   }
   return MOE_OK;

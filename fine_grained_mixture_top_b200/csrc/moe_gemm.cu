@@ -50,6 +50,8 @@ cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid
   MOE_CASE(G_DW2, 256, 4)
   MOE_CASE(G_DW2, 128, 8)
   MOE_CASE(G_DW2, 256, 8)
+  MOE_CASE(G_UPQ, 128, 4)
+  MOE_CASE(G_DOWNQ, 128, 4)
   MOE_CASE(G_RTR, 192, 4)
   MOE_CASE(G_DWR, 128, 4)
 #undef MOE_CASE

@@ -83,6 +83,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// Untiled bulk copy global -> shared completing on an mbarrier (addresses
+// 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // TMA tensor store of a shared-memory box (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap), "r"(src),
@@ -178,6 +186,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 
+// 4-byte async copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// MXFP8 MMA: D[tmem] (+)= A * B with E4M3 operands and E8M0 block scales read
+// from TMEM (sfa, sfb: TMEM addresses whose top two bits select the byte of
+// the 32-bit column, matching the scale ids in the instruction descriptor).
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Copy 32 rows x 16 bytes of shared memory (descriptor) into TMEM columns
+// [taddr, taddr + 4) of lanes 0-31, repeated in each of the four lane quarters.
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and
 // stride byte offsets (16-byte units), version 1, 128-byte swizzle.
@@ -189,6 +220,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1 << 46;   // version
   d |= (uint64_t)2 << 61;   // SWIZZLE_128B
   return d;
+}
+
+// Shared-memory descriptor of rows of 16 bytes packed one after another (no
+// swizzle; 8-row core matrices 128 bytes apart), the source of a scale copy.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)(128 >> 4) << 32;  // stride between 8-row groups
+  d |= (uint64_t)1 << 46;           // version
+  return d;                         // layout type 0: no swizzle
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with E4M3 A/B (K-major), E8M0
+// scales, fp32 D, M = 128; a_sf / b_sf select the scale byte of the column.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int N, uint32_t a_sf, uint32_t b_sf) {
+  return (b_sf << 4)                      // B scale id
+         | (0u << 7) | (0u << 10)         // A, B format E4M3
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | (1u << 23)                     // scale format E8M0
+         | ((uint32_t)(128 >> 4) << 24)   // M / 16
+         | (a_sf << 29);                  // A scale id
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, M = 128.

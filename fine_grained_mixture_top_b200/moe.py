@@ -39,7 +39,8 @@ class MoeRouting(ctypes.Structure):
 
 class MoeSizes(ctypes.Structure):
     _fields_ = [("P_max", c_int64), ("R_max", c_int64), ("route_ws", ctypes.c_size_t),
-                ("fwd_ws", ctypes.c_size_t), ("bwd_ws", ctypes.c_size_t), ("h_elems", c_int64)]
+                ("fwd_ws", ctypes.c_size_t), ("bwd_ws", ctypes.c_size_t), ("h_elems", c_int64),
+                ("fwd_mx_ws", ctypes.c_size_t)]
 
 
 class MoEError(RuntimeError):
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.moe_token_round.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, ctypes.c_size_t, c_void_p]
         L.moe_forward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
                                   c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
+        L.moe_forward_mxfp8.argtypes = L.moe_forward.argtypes
         L.moe_backward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    ctypes.c_size_t, c_void_p]
@@ -98,7 +100,7 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
                   "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout", "moe_backward_ev",
-                  "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols"):
+                  "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols", "moe_forward_mxfp8"):
             getattr(L, f).restype = c_int32
         _lib = L
     return _lib
@@ -195,6 +197,12 @@ def moe_forward(dims, opts, X, W1, W2, routing: Routing, O, H, ws, stream=None):
     _check(lib().moe_forward(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(W1), _ptr(W2),
                              ctypes.byref(routing.struct), _ptr(O), _ptr(H), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_forward_mxfp8(dims, opts, X, W1, W2, routing: Routing, O, H, ws, stream=None):
+    _check(lib().moe_forward_mxfp8(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(W1), _ptr(W2),
+                                   ctypes.byref(routing.struct), _ptr(O), _ptr(H), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "moe_forward_mxfp8")
 
 
 def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW2, dWr, ws, stream=None,
@@ -294,6 +302,7 @@ class MoELayer:
         self.ws_route = torch.empty(self.sizes.route_ws, dtype=u8, device=device)
         self.ws_fwd = torch.empty(self.sizes.fwd_ws, dtype=u8, device=device)
         self.ws_bwd = torch.empty(self.sizes.bwd_ws, dtype=u8, device=device)
+        self.ws_fwd_mx = None   # MXFP8 forward workspace, allocated on first use
         self.H = torch.empty(self.sizes.R_max, 2 * n, dtype=bf, device=device)
         self.O = torch.empty(T, d, dtype=bf, device=device)
         self.dX = torch.empty(T, d, dtype=bf, device=device)
@@ -306,9 +315,17 @@ class MoELayer:
         if self.opts.round_mode:
             moe_token_round(self.dims, self.opts, self.routing, self.ws_route, stream)
 
-    def forward(self, X, W1, W2, stream=None, O=None):
+    def forward(self, X, W1, W2, stream=None, O=None, mxfp8=False):
         O = self.O if O is None else O
-        moe_forward(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd, stream)
+        if mxfp8:
+            if self.ws_fwd_mx is None:
+                import torch
+                if self.sizes.fwd_mx_ws == 0:
+                    raise MoEError(2, "moe_forward_mxfp8 (needs n % 128 == 0)")
+                self.ws_fwd_mx = torch.empty(self.sizes.fwd_mx_ws, dtype=torch.uint8, device=self.device)
+            moe_forward_mxfp8(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd_mx, stream)
+        else:
+            moe_forward(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd, stream)
         return O
 
     def backward(self, dO, X, Wr, W1, W2, stream=None, grad_events=None):

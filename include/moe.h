@@ -110,6 +110,7 @@ typedef struct {
   size_t fwd_ws;        /* bytes of ws for moe_forward */
   size_t bwd_ws;        /* bytes of ws for moe_backward */
   int64_t h_elems;      /* elements of the saved activation H = R_max * 2n (bf16) */
+  size_t fwd_mx_ws;     /* bytes of ws for moe_forward_mxfp8; 0 where that shape is unsupported */
 } moe_sizes;
 
 /* Capacities and workspace sizes for a shape.  Host only; no GPU work. */
@@ -150,6 +151,22 @@ moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe
  */
 moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1, const void* W2,
                        const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Forward with MXFP8 GEMM operands (MXFP8 precision is named as future work
+ * of the method, page "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE",
+ * closing paragraph; format: OCP Microscaling, as for moe_mx_quantize_rows).
+ * X is quantized along d per row, W1 along d and W2 along n per output
+ * column, A = SwiGLU(H) along n per row; the GEMMs multiply E4M3 codes with
+ * their E8M0 block scales on the tensor cores (kind::mxf8f6f4) and
+ * accumulate in fp32.  Same arguments and outputs as moe_forward (O bf16;
+ * H bf16 kept for moe_backward, which is unchanged); ws of
+ * moe_sizes.fwd_mx_ws bytes.  Needs n % 128 == 0 (MOE_ERR_UNSUPPORTED
+ * otherwise).
+ */
+moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
+                             const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
+                             void* stream);
 
 /*
  * Backward given dO[T,d] bf16 ([P2] implementation and algorithm paragraphs;

@@ -26,8 +26,12 @@ notes):
      A along n per row, W2[e] along n per output column -- the K dimension
      of each forward GEMM.  H and Y stay bf16 outputs of fp32 accumulation;
      the backward is unchanged (bf16).
-  M4 The quantized forward computes A = SwiGLU(H) from H as accumulated, then
-     quantizes A per row in blocks of 32 along n.
+  M4 The quantized forward computes A = SwiGLU(H) from H rounded to bf16 --
+     the activation the layer stores for its backward -- then quantizes A per
+     row in blocks of 32 along n.  The A codes are integer decisions taken
+     from floating-point values, so both sides take them from the same bf16
+     H (H itself is returned unrounded, the exact product of the quantized
+     operands).
 
 Parity status: pinned by tests/test_oracle_mx.py (the E4M3 table against the
 format's closed form, round trips of every code, ties to even, the scale
@@ -126,6 +130,15 @@ def mx_dequantize(codes, scales):
     return (B * scale_value(scales)[..., None]).reshape(c.shape)
 
 
+def bf16_round(x):
+    """Nearest bfloat16 value of each fp64 value (8 significant bits, ties to
+    even; below 2^-126 the spacing stays 2^-133)."""
+    x = np.asarray(x, F64)
+    _, E = np.frexp(x)                                   # |x| in [2^(E-1), 2^E)
+    ulp = np.exp2(np.maximum(E.astype(F64) - 8.0, -133.0))
+    return np.round(x / ulp) * ulp                       # np.round: half to even
+
+
 def mx_round(M):
     """M through quantization and back (the values the 8-bit GEMM multiplies)."""
     return mx_dequantize(*mx_quantize(M))
@@ -157,7 +170,7 @@ def forward_mxfp8(X, Wr, bias, W1, W2, K, topk_idx=None, routing=None):
         W1q = mx_round(np.asarray(W1[e], F64).T).T       # along d, per output column
         W2q = mx_round(np.asarray(W2[e], F64).T).T       # along n, per output column
         H[a:b] = Xq[perm["row_tok"][a:b]] @ W1q
-        A[a:b] = mo.swiglu(H[a:b], n)
+        A[a:b] = mo.swiglu(bf16_round(H[a:b]), n)         # M4
         Aq[a:b] = mx_round(A[a:b])                       # A along n, per row
         Y[a:b] = Aq[a:b] @ W2q
     O = mo.aggregate(Y, rt["pair_gate"], perm["pair_row"], rt["tok_ptr"], T)

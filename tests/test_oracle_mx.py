@@ -73,6 +73,23 @@ def test_power_of_two_scaling_moves_only_the_scales():
         np.testing.assert_array_equal(s1.astype(int), s0.astype(int) + k)
 
 
+def _bf16_torch(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, np.float64)).float().to(torch.bfloat16).double().numpy()
+
+
+def test_bf16_rounding_matches_the_format():
+    # ties to even at 1: spacing 2^-7 above 1, 2^-8 below
+    v = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 - 2.0 ** -9, 1 - 3 * 2.0 ** -9, -(1 + 2.0 ** -8),
+                  3 * 2.0 ** -134, 2.0 ** -134, 0.0])
+    np.testing.assert_array_equal(mx.bf16_round(v), [1.0, 1 + 2.0 ** -6, 1.0, 1 - 2.0 ** -7, -1.0,
+                                                     2.0 ** -132, 0.0, 0.0])
+    # fp32 inputs (no double rounding through fp32): the library conversion
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-60, 60, 20000))).astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(mx.bf16_round(x), _bf16_torch(x))
+
+
 def _layer(T, d, E, n, K, seed, integer=False):
     rng = np.random.default_rng(seed)
     if integer:   # every 32-block holds +-15 and integers: quantization is exact
@@ -94,7 +111,8 @@ def test_representable_inputs_give_the_exact_up_projection():
     fw = mo.forward(X, Wr, None, W1, W2, 2)
     fq = mx.forward_mxfp8(X, Wr, None, W1, W2, 2)
     np.testing.assert_array_equal(fq["H"], fw["H"])
-    np.testing.assert_array_equal(fq["A"], fw["A"])
+    # A from the stored (bf16) H
+    np.testing.assert_array_equal(fq["A"], mo.swiglu(_bf16_torch(fw["H"]), 32))
 
 
 def test_dense_case_matches_plain_matmuls():
@@ -113,7 +131,9 @@ def test_dense_case_matches_plain_matmuls():
         return np.moveaxis((mx.e4m3_decode(mx.e4m3_encode(B / S)) * S).reshape(Mt.shape), -1, axis)
 
     H = q(X, 1) @ q(W1[0], 0)
-    g, u = H[:, :64], H[:, 64:]
+    np.testing.assert_allclose(fq["H"], H, rtol=1e-12, atol=1e-12)
+    Hb = _bf16_torch(H)
+    g, u = Hb[:, :64], Hb[:, 64:]
     A = g / (1 + np.exp(-g)) * u
     O = q(A, 1) @ q(W2[0], 0)
     np.testing.assert_allclose(fq["O"], O, rtol=1e-12, atol=1e-12)
