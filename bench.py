@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--ref-sample-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mxfp8-forward", action="store_true",
+                    help="forward GEMMs on MXFP8 operands (moe_forward_mxfp8); backward unchanged")
     ap.add_argument("--comm-sms", type=int, default=16,
                     help="N>1: SMs left to NCCL while the gradient all-reduces overlap the backward "
                          "(0: all-reduce after the step, no overlap)")
@@ -77,6 +79,12 @@ def kernel_work(cfg, R):
         "aggregate_bwd": (R * d, 2 * R * d + 2 * T * d + 4 * R + 4 * T),
         "router_logits_gemm": (2 * T * d * E, 2 * T * d + 4 * d * E + 4 * T * E),
         "router_dwr_gemm": (2 * T * d * E, 2 * T * d + 4 * T * E + 4 * d * E),
+        # MXFP8 forward: 1-byte codes plus one scale byte per 32
+        "up_proj_gemm_mx": (4 * R * d * n, T * d * 33 // 32 + 2 * E * d * n * 33 // 32 + 4 * R * n + R * n * 33 // 32),
+        "down_proj_gemm_mx": (2 * R * d * n, R * n * 33 // 32 + E * d * n * 33 // 32 + 2 * R * d),
+        "mx_quant_x": (0, 2 * T * d + T * d * 33 // 32),
+        # W1 and W2 read (bf16), codes and their scale tiles written
+        "mx_quant_w": (0, 6 * E * d * n + 3 * E * d * n * 33 // 32),
     }
     return w
 
@@ -260,6 +268,9 @@ def main():
     layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=cfg.round_mode, router_grad=1,
                          seed=cfg.seed, device=dev)
     X, Wr, b, W1, W2, dO = (inp[k] for k in ("X", "Wr", "bias", "W1", "W2", "dO"))
+    layer.mxfp8 = args.mxfp8_forward
+    if args.mxfp8_forward:
+        workload += "; forward GEMMs on MXFP8 operands (E4M3, E8M0 scale per 32 along K)"
     stream = torch.cuda.current_stream()
     if overlap:
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -358,7 +369,8 @@ def main():
             entry["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
         breakdown[name] = entry
     # forward / backward split of the breakdown pass (routing counted apart)
-    fwd_k = {"up_proj_gemm", "down_proj_gemm", "aggregate_fwd"}
+    fwd_k = {"up_proj_gemm", "down_proj_gemm", "aggregate_fwd", "up_proj_gemm_mx", "down_proj_gemm_mx",
+             "mx_quant_x", "mx_quant_w"}
     route_us = fwd_us = bwd_us = 0.0
     for name, ts in per.items():
         us = 1e3 * sum(ts) / n_breakdown
@@ -448,7 +460,7 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16+mxfp8" if args.mxfp8_forward else "bf16", "data": "synthetic",
             "config": {"workload": workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
                        "router_bias": cfg.bias, "round_mode": cfg.round_mode,
                        "parallelism": f"dp{world}" + ((" (NCCL all-reduce of dW2, dW1, dWr overlapping the backward, "

@@ -216,8 +216,8 @@ struct FwdWs {
 // MXFP8 forward: codes and scales of X, W1, W2 and A, and Y
 struct MxFwdWs {
   uint8_t *Xq, *SX;            // [T, d], [T, d/32]
-  uint8_t *W1q, *SW1, *SW1t;   // [E, 2n, d], [E, 2n, d/32], scale tiles [E][n/64][d/128]
-  uint8_t *W2q, *SW2, *SW2t;   // [E, d, n], [E, d, n/32], scale tiles [E][d/128][n/128]
+  uint8_t *W1q, *SW1t;         // [E, 2n, d], scale tiles [E][n/64][d/128]
+  uint8_t *W2q, *SW2t;         // [E, d, n], scale tiles [E][d/128][n/128]
   uint8_t *Aq, *SA;            // [R_max, n], scale tiles [R_max/128][n/128]
   __nv_bfloat16* Y;            // [R_max, d]
 };
@@ -236,10 +236,8 @@ size_t carve_fwd_mx(const Plan& p, void* ws, MxFwdWs* w) {
   w->Xq = c.take<uint8_t>(T * d);
   w->SX = c.take<uint8_t>(T * (d / 32));
   w->W1q = c.take<uint8_t>(E * 2 * n * d);
-  w->SW1 = c.take<uint8_t>(E * 2 * n * (d / 32));
   w->SW1t = c.take<uint8_t>(E * (n / 64) * (d / 128) * 512);
   w->W2q = c.take<uint8_t>(E * d * n);
-  w->SW2 = c.take<uint8_t>(E * d * (n / 32));
   w->SW2t = c.take<uint8_t>(E * (d / 128) * (n / 128) * 512);
   w->Aq = c.take<uint8_t>(R * n);
   w->SA = c.take<uint8_t>((R / 128) * (n / 128) * 512);
@@ -555,10 +553,10 @@ moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const v
   }
   {
     ProfScope ps(st, "mx_quant_w");
-    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W1), E, d, 2 * n, w.W1q, w.SW1, st));
-    MOE_TRY_CUDA(launch_mx_scale_tiles(w.SW1, E, d, 2 * n, 1, w.SW1t, st));
-    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W2), E, n, d, w.W2q, w.SW2, st));
-    MOE_TRY_CUDA(launch_mx_scale_tiles(w.SW2, E, n, d, 0, w.SW2t, st));
+    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W1), E, d, 2 * n, w.W1q, nullptr, w.SW1t,
+                                      1, st));
+    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W2), E, n, d, w.W2q, nullptr, w.SW2t, 0,
+                                      st));
   }
   // up-projection on MXFP8 operands: H = X[tok] W1[e] (bf16 out), A = SwiGLU(H)
   // quantized to MXFP8 with its scale tiles
@@ -777,7 +775,7 @@ moe_status moe_mx_quantize_cols(const void* in, int32_t E, int32_t K, int32_t N,
   if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes) || !aligned16(scales))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(in), E, K, N, static_cast<uint8_t*>(codes),
-                                    static_cast<uint8_t*>(scales), static_cast<cudaStream_t>(stream)));
+                                    static_cast<uint8_t*>(scales), nullptr, 0, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

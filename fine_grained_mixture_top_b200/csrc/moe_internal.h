@@ -94,8 +94,8 @@ cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
 // ---- MXFP8 quantization (moe_mx.cu)
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16* in, int64_t rows, int K, uint8_t* codes, uint8_t* scales,
                                  cudaStream_t s);
+// codes [E][N][K] (K-major); scales linear [E][N][K/32] and/or (tiles != null,
+// K % 128 == 0, N % 128 == 0) the block-scaled GEMM's 512-byte scale tiles
 cudaError_t launch_mx_quant_cols(const __nv_bfloat16* in, int E, int K, int N, uint8_t* codes, uint8_t* scales,
-                                 cudaStream_t s);
-cudaError_t launch_mx_scale_tiles(const uint8_t* scales, int E, int K, int N, int split_half, uint8_t* tiles,
-                                  cudaStream_t s);
+                                 uint8_t* tiles, int split_half, cudaStream_t s);
 }  // namespace moe

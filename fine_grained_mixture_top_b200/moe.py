@@ -303,6 +303,7 @@ class MoELayer:
         self.ws_fwd = torch.empty(self.sizes.fwd_ws, dtype=u8, device=device)
         self.ws_bwd = torch.empty(self.sizes.bwd_ws, dtype=u8, device=device)
         self.ws_fwd_mx = None   # MXFP8 forward workspace, allocated on first use
+        self.mxfp8 = False      # default precision of forward(): MXFP8 GEMM operands when True
         self.H = torch.empty(self.sizes.R_max, 2 * n, dtype=bf, device=device)
         self.O = torch.empty(T, d, dtype=bf, device=device)
         self.dX = torch.empty(T, d, dtype=bf, device=device)
@@ -315,9 +316,9 @@ class MoELayer:
         if self.opts.round_mode:
             moe_token_round(self.dims, self.opts, self.routing, self.ws_route, stream)
 
-    def forward(self, X, W1, W2, stream=None, O=None, mxfp8=False):
+    def forward(self, X, W1, W2, stream=None, O=None, mxfp8=None):
         O = self.O if O is None else O
-        if mxfp8:
+        if self.mxfp8 if mxfp8 is None else mxfp8:
             if self.ws_fwd_mx is None:
                 import torch
                 if self.sizes.fwd_mx_ws == 0:
