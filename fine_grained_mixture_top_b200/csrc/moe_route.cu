@@ -61,16 +61,21 @@ cudaError_t launch_split_wr(const RouteArgs& a, cudaStream_t s) {
 // One warp per token; lane l holds the logits of experts l, l + 32, ... in
 // registers (PER of them).  p = softmax(z) over all E.  The K largest logits
 // are selected in K rounds (ties to the lower expert index, slots in
-// descending order): each lane offers its best unselected logit, one
-// warp-wide max over order-preserving integer keys finds the value and one
-// warp-wide min finds the lowest expert holding it.  The gates are a softmax
-// over the selected logits (= p renormalised).
+// descending order): each lane keeps its best unselected logit as an
+// order-preserving integer key; one warp-wide max finds the round's value and
+// one warp-wide min the lowest expert holding it.  Only the lane that gave up
+// its logit looks for its next best.  The gates are a softmax over the
+// selected logits (= p renormalised).
 constexpr int kTopkWarps = 8;
 
-// Unsigned key with the order of the float (no NaNs among logits).
+// Unsigned key with the order of the float (no NaNs among logits); 0 is
+// below the key of every float.
 __device__ __forceinline__ uint32_t order_key(float v) {
   const uint32_t u = __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 template <int PER>
@@ -88,53 +93,59 @@ __global__ void __launch_bounds__(256) softmax_topk_kernel(RouteArgs a) {
     if (e < a.E) m = fmaxf(m, z[j]);
   }
   m = warp_max(m);
+  float ex[PER];
   float sum = 0.f;
 #pragma unroll
-  for (int j = 0; j < PER; ++j)
-    if (lane + 32 * j < a.E) sum += expf(z[j] - m);
+  for (int j = 0; j < PER; ++j) {
+    ex[j] = expf(z[j] - m);
+    if (lane + 32 * j < a.E) sum += ex[j];
+  }
   sum = warp_sum(sum);
   const float inv = 1.0f / sum;
   float* pr = a.probs + (size_t)t * a.E;
 #pragma unroll
   for (int j = 0; j < PER; ++j)
-    if (lane + 32 * j < a.E) pr[lane + 32 * j] = expf(z[j] - m) * inv;
+    if (lane + 32 * j < a.E) pr[lane + 32 * j] = ex[j] * inv;
 
-  uint32_t taken = 0u;  // bit j: expert lane + 32 j already selected
-  float my_v = 0.f;
-  int my_e = 0;
-  for (int k = 0; k < a.K; ++k) {
-    uint32_t best = 0u;   // 0: nothing left on this lane (below every real key)
-    uint32_t best_e = 0xFFFFFFFFu;
+  // keys of this lane's unselected logits (0: none); -0 keys like +0
+  uint32_t key[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int e = lane + 32 * j;
-      if (e < a.E && !((taken >> j) & 1u)) {
-        const uint32_t key = order_key(z[j] == 0.f ? 0.f : z[j]);  // -0 ties with +0
-        if (key > best) {  // strict: the lower expert of a lane wins a tie
-          best = key;
-          best_e = (uint32_t)e;
-        }
-      }
-    }
-    const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
-    const uint32_t win = __reduce_min_sync(0xffffffffu, best == kmax ? best_e : 0xFFFFFFFFu);
-    const int owner = (int)(win & 31u);
-    if (lane == owner) taken |= 1u << (win >> 5);
-    float v_win = 0.f;
+  for (int j = 0; j < PER; ++j) key[j] = (lane + 32 * j < a.E) ? order_key(z[j] == 0.f ? 0.f : z[j]) : 0u;
+  uint32_t best = 0u;
+  int bj = 0;
+  auto local_best = [&]() {  // strict >: the lower expert of a lane wins a tie
+    best = 0u;
+    bj = 0;
 #pragma unroll
     for (int j = 0; j < PER; ++j)
-      if ((int)(win >> 5) == j) v_win = z[j];
-    v_win = __shfl_sync(0xffffffffu, v_win, owner);
+      if (key[j] > best) {
+        best = key[j];
+        bj = j;
+      }
+  };
+  local_best();
+  uint32_t my_key = 0u;
+  int my_e = 0;
+  for (int k = 0; k < a.K; ++k) {
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, best == kmax ? (uint32_t)(lane + 32 * bj) : 0xFFFFFFFFu);
+    if (lane == (int)(win & 31u)) {
+#pragma unroll
+      for (int j = 0; j < PER; ++j)
+        if (j == bj) key[j] = 0u;
+      local_best();
+    }
     if (lane == k) {
-      my_v = v_win;
+      my_key = kmax;
       my_e = (int)win;
     }
   }
+  const float my_v = key_value(my_key);
   const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-  const float ex = lane < a.K ? expf(my_v - vmax) : 0.f;
-  const float den = warp_sum(ex);
+  const float g_ex = lane < a.K ? expf(my_v - vmax) : 0.f;
+  const float den = warp_sum(g_ex);
   if (lane < a.K) {
-    const float g = ex / den;
+    const float g = g_ex / den;
     const size_t o = (size_t)t * a.K + lane;
     a.topk_idx[o] = my_e;
     a.topk_gate[o] = g;
