@@ -689,25 +689,30 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       if (!ok) break;
       if (!mbar_wait(smem_u32(&acc_full[0]), tcount & 1, abort_flag, p.st, KIND * 16 + 4)) break;
       tc_fence_after();
-      const int trow = t.m0 + rloc;
-      float* dst = p.outf + (size_t)trow * p.E;
+      // each warp's 32 rows x 32 logits go through shared memory (padded
+      // rows, conflict-free both ways) and leave as 128-byte row pieces
+      float* stg = reinterpret_cast<float*>(smem + SH::kStoreOffset + (warp - 2) * (EC::kBufs * kStoreBuf));
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
         uint32_t mid[32], lo[32];
         tmem_ld32(lane_addr + 128 + c, mid);
         tmem_ld32(lane_addr + 192 + c, lo);
         tc_wait_ld();
-        if (trow < p.T) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = t.nt * 64 + c + i;
-            if (e < p.E) {
-              float z = (c == 0 ? hs[i] : hs[32 + i]) + (__uint_as_float(mid[i]) + __uint_as_float(lo[i]));
-              if (p.bias) z += __ldg(p.bias + e);
-              dst[e] = z;
-            }
-          }
+        for (int i = 0; i < 32; ++i) {
+          const int e = t.nt * 64 + c + i;
+          float z = (c == 0 ? hs[i] : hs[32 + i]) + (__uint_as_float(mid[i]) + __uint_as_float(lo[i]));
+          if (p.bias && e < p.E) z += __ldg(p.bias + e);
+          stg[lane * 33 + i] = z;
         }
+        __syncwarp();
+        const int e = t.nt * 64 + c + lane;
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+          const int trow = t.m0 + q * 32 + r;
+          if (trow < p.T && e < p.E) p.outf[(size_t)trow * p.E + e] = stg[r * 33 + lane];
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[0]));
