@@ -461,6 +461,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above touched only shared memory, TMEM and the kernel's own
+  // parameters; global reads and writes start once the predecessor is done
+  pdl_wait();
 
   const int num_tiles = gemm_num_tiles<KIND, BN>(p);
 

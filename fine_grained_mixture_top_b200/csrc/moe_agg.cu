@@ -35,6 +35,7 @@ __global__ void __launch_bounds__(256) aggregate_fwd_kernel(int T, int d8, const
                                                             const int* __restrict__ pair_row,
                                                             const float* __restrict__ pair_gate,
                                                             const uint4* __restrict__ Y, uint4* __restrict__ O) {
+  pdl_wait();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)T * d8) return;
   const int t = (int)(idx / d8), c = (int)(idx - (int64_t)t * d8);
@@ -60,7 +61,7 @@ cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pa
                                  const __nv_bfloat16* Y, __nv_bfloat16* O, cudaStream_t s) {
   const int d8 = d / 8;
   const int64_t n = (int64_t)T * d8;
-  aggregate_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+  launch_pdl(aggregate_fwd_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 
       T, d8, tok_ptr, pair_row, pair_gate, reinterpret_cast<const uint4*>(Y), reinterpret_cast<uint4*>(O));
   return cudaGetLastError();
 }
@@ -134,6 +135,7 @@ __device__ __forceinline__ void transpose_tile(const float* __restrict__ in, flo
 // dWr[i, e] = sum over K splits of the split-K partials, in split order
 __global__ void dwr_reduce_kernel(int d, int E, int Epad, int splits, const float* __restrict__ part,
                                   float* __restrict__ dWr) {
+  pdl_wait();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)d * E) return;
   const int i = (int)(idx / E), e = (int)(idx - (int64_t)i * E);
@@ -144,7 +146,7 @@ __global__ void dwr_reduce_kernel(int d, int E, int Epad, int splits, const floa
 
 cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s) {
   const int64_t n = (int64_t)d * E;
-  dwr_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d, E, Epad, splits, part, dWr);
+  launch_pdl(dwr_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d, E, Epad, splits, part, dWr);
   return cudaGetLastError();
 }
 
@@ -154,6 +156,7 @@ __global__ void __launch_bounds__(256) aggregate_bwd_kernel(int T, int d8, const
                                                             const int* __restrict__ pair_row,
                                                             const uint4* __restrict__ dXt,
                                                             uint4* __restrict__ dX) {
+  pdl_wait();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)T * d8) return;
   const int t = (int)(idx / d8), c = (int)(idx - (int64_t)t * d8);
@@ -175,7 +178,7 @@ cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pa
                                  __nv_bfloat16* dX, cudaStream_t s) {
   const int d8 = d / 8;
   const int64_t n = (int64_t)T * d8;
-  aggregate_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+  launch_pdl(aggregate_bwd_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 
       T, d8, tok_ptr, pair_row, reinterpret_cast<const uint4*>(dXt), reinterpret_cast<uint4*>(dX));
   return cudaGetLastError();
 }
@@ -202,6 +205,7 @@ __device__ __forceinline__ void expert_order_block(int E, const int* __restrict_
 //                                       weight-gradient scheduler; zeroes its
 //                                       tile counters
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
+  pdl_wait();
   const int b = blockIdx.x;
   if (b < a.tok_blocks) {
     router_bwd_token(a, b * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
@@ -221,7 +225,7 @@ cudaError_t launch_bwd_prep(const BwdPrepArgs& a0, cudaStream_t s) {
   BwdPrepArgs a = a0;
   a.tok_blocks = a.router ? (a.T + 7) / 8 : 0;
   a.tr_blocks = a.router ? ((a.E + 31) / 32) * ((a.d + 31) / 32) : 0;
-  bwd_prep_kernel<<<a.tok_blocks + a.tr_blocks + 1, 256, 0, s>>>(a);
+  launch_pdl(bwd_prep_kernel, dim3(a.tok_blocks + a.tr_blocks + 1), dim3(256), 0, s, a);
   return cudaGetLastError();
 }
 

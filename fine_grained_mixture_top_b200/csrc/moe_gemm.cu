@@ -21,8 +21,7 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
     configured_dev = dev;
   }
   if (grid <= 0) return cudaSuccess;
-  fn<<<grid, threads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(fn, dim3(grid), dim3(threads), (size_t)smem, stream, p);
 }
 
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s) {

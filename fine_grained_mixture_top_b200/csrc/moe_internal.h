@@ -3,10 +3,36 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 #include "gemm.cuh"
 
 namespace moe {
+
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+
+// Launch on `s` with programmatic stream serialization (see pdl_wait): the
+// kernel's blocks may be scheduled while the previous kernel of the stream
+// finishes.  Every kernel of this library calls pdl_wait() before touching
+// global memory.
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              A&&... args) {
+  cudaLaunchConfig_t c = {};
+  c.gridDim = grid;
+  c.blockDim = block;
+  c.dynamicSmemBytes = smem;
+  c.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  c.attrs = at;
+  c.numAttrs = 1;
+  return cudaLaunchKernelEx(&c, kernel, std::forward<A>(args)...);
+}
+
 
 constexpr int kTile = 128;        // rows per expert tile (segments are padded to it)
 constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation

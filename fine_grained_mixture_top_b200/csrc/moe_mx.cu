@@ -18,6 +18,7 @@ constexpr int kRowIters = 4;
 __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows,
                                                             int K, uint8_t* __restrict__ codes,
                                                             uint8_t* __restrict__ scales) {
+  pdl_wait();
   const int kblocks = K / kMxBlock;
   const int64_t slots = rows * kblocks * 4;  // 4 lanes per block
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const __nv_bfloat16*
 __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int E, int K,
                                                             int N, uint8_t* __restrict__ codes,
                                                             uint8_t* __restrict__ scales) {
+  pdl_wait();
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int kblocks = K / kMxBlock;
   if (g >= (int64_t)E * kblocks * N) return;
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(256) mx_quant_cols_tiled_kernel(const __nv_bfl
                                                                   int N, int split_half, uint8_t* __restrict__ codes,
                                                                   uint8_t* __restrict__ scales,
                                                                   uint8_t* __restrict__ tiles) {
+  pdl_wait();
   __shared__ __align__(16) __nv_bfloat16 tile[128][64];
   const int e = blockIdx.z;
   const int k0 = blockIdx.y * 128;
@@ -186,7 +189,7 @@ cudaError_t launch_mx_quant_rows(const __nv_bfloat16* in, int64_t rows, int K, u
   if (slots == 0) return cudaSuccess;
   const int64_t threads = (slots + kRowIters - 1) / kRowIters;
   const int64_t blocks = (threads + 255) / 256;  // grid stride = blocks * 256, a multiple of 4
-  mx_quant_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(in, rows, K, codes, scales);
+  launch_pdl(mx_quant_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, in, rows, K, codes, scales);
   return cudaGetLastError();
 }
 
@@ -196,12 +199,12 @@ cudaError_t launch_mx_quant_cols(const __nv_bfloat16* in, int E, int K, int N, u
   if (K % 128 == 0 && N % 64 == 0) {
     if (tiles && N % 128 != 0) return cudaErrorInvalidValue;
     dim3 grid((unsigned)(N / 64), (unsigned)(K / 128), (unsigned)E);
-    mx_quant_cols_tiled_kernel<<<grid, 256, 0, s>>>(in, K, N, split_half, codes, scales, tiles);
+    launch_pdl(mx_quant_cols_tiled_kernel, dim3(grid), dim3(256), 0, s, in, K, N, split_half, codes, scales, tiles);
     return cudaGetLastError();
   }
   if (tiles) return cudaErrorInvalidValue;
   const int64_t threads = (int64_t)E * (K / kMxBlock) * N;
-  mx_quant_cols_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(in, E, K, N, codes, scales);
+  launch_pdl(mx_quant_cols_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, in, E, K, N, codes, scales);
   return cudaGetLastError();
 }
 

@@ -37,6 +37,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // hi, mid, lo parts of experts 64 g .. 64 g + 63 (zero beyond E).
 __global__ void split_wr_kernel(const float* __restrict__ Wr, __nv_bfloat16* __restrict__ out, int d, int E,
                                 int Epad) {
+  pdl_wait();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)d * Epad) return;
   const int i = (int)(idx / Epad), e = (int)(idx % Epad);
@@ -53,7 +54,7 @@ __global__ void split_wr_kernel(const float* __restrict__ Wr, __nv_bfloat16* __r
 
 cudaError_t launch_split_wr(const RouteArgs& a, cudaStream_t s) {
   const int64_t n = (int64_t)a.d * a.Epad;
-  split_wr_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.Wr, a.Wr_split, a.d, a.E, a.Epad);
+  launch_pdl(split_wr_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, a.Wr, a.Wr_split, a.d, a.E, a.Epad);
   return cudaGetLastError();
 }
 
@@ -80,6 +81,7 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 
 template <int PER>
 __global__ void __launch_bounds__(256) softmax_topk_kernel(RouteArgs a) {
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= a.T) return;  // warp-uniform
@@ -161,12 +163,12 @@ __global__ void __launch_bounds__(256) softmax_topk_kernel(RouteArgs a) {
 cudaError_t launch_softmax_topk(const RouteArgs& a, cudaStream_t s) {
   const int blocks = (a.T + kTopkWarps - 1) / kTopkWarps;
   const int per = (a.E + 31) / 32;
-  if (per <= 1) softmax_topk_kernel<1><<<blocks, 256, 0, s>>>(a);
-  else if (per <= 2) softmax_topk_kernel<2><<<blocks, 256, 0, s>>>(a);
-  else if (per <= 4) softmax_topk_kernel<4><<<blocks, 256, 0, s>>>(a);
-  else if (per <= 8) softmax_topk_kernel<8><<<blocks, 256, 0, s>>>(a);
-  else if (per <= 16) softmax_topk_kernel<16><<<blocks, 256, 0, s>>>(a);
-  else if (per <= 32) softmax_topk_kernel<32><<<blocks, 256, 0, s>>>(a);
+  if (per <= 1) launch_pdl(softmax_topk_kernel<1>, dim3(blocks), dim3(256), 0, s, a);
+  else if (per <= 2) launch_pdl(softmax_topk_kernel<2>, dim3(blocks), dim3(256), 0, s, a);
+  else if (per <= 4) launch_pdl(softmax_topk_kernel<4>, dim3(blocks), dim3(256), 0, s, a);
+  else if (per <= 8) launch_pdl(softmax_topk_kernel<8>, dim3(blocks), dim3(256), 0, s, a);
+  else if (per <= 16) launch_pdl(softmax_topk_kernel<16>, dim3(blocks), dim3(256), 0, s, a);
+  else if (per <= 32) launch_pdl(softmax_topk_kernel<32>, dim3(blocks), dim3(256), 0, s, a);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
@@ -178,6 +180,7 @@ cudaError_t launch_softmax_topk(const RouteArgs& a, cudaStream_t s) {
 // per-expert bit mask, so the result does not depend on the order in which
 // threads run.
 __global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
+  pdl_wait();
   extern __shared__ uint32_t bits[];  // [E][8]
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.sync = 0;  // for chunk_scan_kernel's last block
   const int words = kChunk / 32;
@@ -235,6 +238,7 @@ __device__ int block_exclusive_scan_256(int v, int* sh /*[8]*/, int* total) {
 // the expert's total count.  The last block to finish then computes the
 // 128-padded segment offsets (exclusive scan over experts).
 __global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(RouteArgs a) {
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * (kScanThreads / 32) + warp;
   if (e < a.E) {
@@ -279,6 +283,7 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(RouteArgs a) {
 // The blocks after those: one warp per expert writes the tile -> expert list
 // and the padding rows (token -1, gate 0) of its segment.
 __global__ void __launch_bounds__(256) scatter_kernel(RouteArgs a, int token_blocks) {
+  pdl_wait();
   if ((int)blockIdx.x >= token_blocks) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = ((int)blockIdx.x - token_blocks) * 8 + warp;
@@ -307,16 +312,16 @@ __global__ void __launch_bounds__(256) scatter_kernel(RouteArgs a, int token_blo
 cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s) {
   {
     ProfScope ps(s, "permute_rank");
-    rank_kernel<<<a.nchunks, kChunk, (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s>>>(a);
+    launch_pdl(rank_kernel, dim3(a.nchunks), dim3(kChunk), (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s, a);
   }
   {
     ProfScope ps(s, "permute_scan");
-    chunk_scan_kernel<<<(a.E + 7) / 8, kScanThreads, 0, s>>>(a);
+    launch_pdl(chunk_scan_kernel, dim3((a.E + 7) / 8), dim3(kScanThreads), 0, s, a);
   }
   {
     ProfScope ps(s, "permute_scatter");
     const int token_blocks = (a.T + 255) / 256;
-    scatter_kernel<<<token_blocks + (a.E + 7) / 8, 256, 0, s>>>(a, token_blocks);
+    launch_pdl(scatter_kernel, dim3(token_blocks + (a.E + 7) / 8), dim3(256), 0, s, a, token_blocks);
   }
   return cudaGetLastError();
 }
@@ -340,6 +345,7 @@ __device__ __forceinline__ unsigned long long splitmix64_dev(unsigned long long 
 // block per expert then reads its row contiguously.
 __global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int W, uint32_t* memberT,
                                  int* sync) {
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t == 0) *sync = 0;  // for tr_count_kernel's last block
   if (t >= T) return;
@@ -349,6 +355,7 @@ __global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int
 
 // probsT[e, t] = probs[t, e], 32 x 32 tiles through shared memory
 __global__ void tr_transpose_kernel(const float* __restrict__ probs, float* __restrict__ probsT, int T, int E) {
+  pdl_wait();
   __shared__ float tile[32][33];
   const int e0 = blockIdx.x * 32, t0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -372,6 +379,7 @@ template <bool STAGED>
 __global__ void __launch_bounds__(1024) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
                                                          const int* counts, const float* probsT,
                                                          const uint32_t* memberT, uint32_t* finalT) {
+  pdl_wait();
   extern __shared__ uint32_t stage[];  // STAGED: p bits [T], then the candidate mask [W]
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
@@ -513,6 +521,7 @@ __device__ __forceinline__ uint32_t tr_token_mask(const uint32_t* finalT, int E,
 // block totals (exclusive, total at [nblocks]).
 __global__ void __launch_bounds__(256) tr_count_kernel(const uint32_t* finalT, int T, int E, int W, int* local,
                                                        int* blk, int* sync) {
+  pdl_wait();
   __shared__ int sh[8];
   __shared__ int is_last;
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -548,6 +557,7 @@ __global__ void __launch_bounds__(256) tr_count_kernel(const uint32_t* finalT, i
 __global__ void __launch_bounds__(256) tr_write_kernel(const uint32_t* finalT, const float* probs, int T, int E,
                                                        int W, const int* local, const int* blk, int* tok_ptr,
                                                        int* pair_expert, float* pair_gate) {
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const bool live = t < T;
@@ -586,12 +596,12 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
   const int tb = (r.T + 255) / 256;
   {
     ProfScope ps(s, "round_member");
-    tr_member_kernel<<<tb, 256, 0, s>>>(a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.sync);
+    launch_pdl(tr_member_kernel, dim3(tb), dim3(256), 0, s, a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.sync);
   }
   {
     ProfScope ps(s, "round_transpose");
     dim3 grid((r.E + 31) / 32, (r.T + 31) / 32), block(32, 8);
-    tr_transpose_kernel<<<grid, block, 0, s>>>(r.probs, r.probsT, r.T, r.E);
+    launch_pdl(tr_transpose_kernel, dim3(grid), dim3(block), 0, s, r.probs, r.probsT, r.T, r.E);
   }
   {
     ProfScope ps(s, "round_select");
@@ -605,20 +615,20 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
         if (err != cudaSuccess) return err;
         configured = true;
       }
-      tr_select_kernel<true><<<r.E, 1024, staged, s>>>(r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
+      launch_pdl(tr_select_kernel<true>, dim3(r.E), dim3(1024), staged, s, r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
                                                         r.finalT);
     } else {
-      tr_select_kernel<false><<<r.E, 1024, 0, s>>>(r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
+      launch_pdl(tr_select_kernel<false>, dim3(r.E), dim3(1024), 0, s, r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
                                                     r.finalT);
     }
   }
   {
     ProfScope ps(s, "round_count");
-    tr_count_kernel<<<tb, 256, 0, s>>>(r.finalT, r.T, r.E, W, r.local, r.blk, r.sync);
+    launch_pdl(tr_count_kernel, dim3(tb), dim3(256), 0, s, r.finalT, r.T, r.E, W, r.local, r.blk, r.sync);
   }
   {
     ProfScope ps(s, "round_write");
-    tr_write_kernel<<<tb, 256, 0, s>>>(r.finalT, r.probs, r.T, r.E, W, r.local, r.blk, a.tok_ptr, a.pair_expert,
+    launch_pdl(tr_write_kernel, dim3(tb), dim3(256), 0, s, r.finalT, r.probs, r.T, r.E, W, r.local, r.blk, a.tok_ptr, a.pair_expert,
                                        a.pair_gate);
   }
   err = cudaGetLastError();

@@ -71,6 +71,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Kernels of one stream are launched with programmatic stream serialization:
+// a kernel's blocks may be scheduled as its predecessor's last blocks exit,
+// run only what touches no global memory (barrier set-up, TMEM allocation,
+// descriptor prefetch), then wait here until the predecessor grid has
+// completed and its writes are visible.  (Without a programmatic predecessor
+// the wait returns at once.)  Every kernel waits before its first global
+// access, so each grid also completes after its predecessor and the ordering
+// is transitive down the stream.  No kernel triggers its dependents early:
+// letting the next grid's blocks in while a persistent GEMM still runs
+// measured slower (1.379 against 1.357 ms per 7B-class step).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
   asm volatile(
