@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 
-SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_route.cu", "moe_agg.cu", "moe_mx.cu"]
+SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_route.cu", "moe_agg.cu", "moe_mx.cu", "moe_ep.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xptxas", "-v", "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]

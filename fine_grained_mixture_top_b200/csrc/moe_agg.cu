@@ -88,9 +88,12 @@ __device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, in
     const float* part = dS_part + (size_t)pair_row[p] * nts;
     float ds = 0.f;
     for (int j = 0; j < nts; ++j) ds += part[j];
+    if (a.pair_dS) a.pair_dS[p] = ds;
+    if (!a.router) continue;
     dz_row[pair_row[p]] = ds;  // dS for now
     inner += pair_gate[p] * ds;
   }
+  if (!a.router) return;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) inner += __shfl_xor_sync(0xffffffffu, inner, o);
   __syncwarp();
@@ -131,6 +134,89 @@ __device__ __forceinline__ void transpose_tile(const float* __restrict__ in, flo
 }
 
 
+
+// Wr^T as a kernel of its own (the router backward from given dS).
+__global__ void __launch_bounds__(256) wr_transpose_kernel(const float* __restrict__ Wr, float* __restrict__ WrT,
+                                                           int d, int E) {
+  pdl_wait();
+  const int nbx = (E + 31) / 32;
+  transpose_tile(Wr, WrT, d, E, blockIdx.x % nbx, blockIdx.x / nbx);
+}
+
+// Router backward from caller-given dS per pair (dS[pos[p]], or dS[p] without
+// pos): one warp per token.  dz_p = s_p (dS_p - sum_q s_q dS_q) over the
+// token's pairs; the dense dz row split into bf16 hi + lo parts for the
+// dWr = X^T dz GEMM (layout as in router_bwd_token); dX_t += sum_p dz_p Wr[:, e_p]
+// (bf16 in and out, fp32 sums).
+__global__ void __launch_bounds__(256) router_bwd_given_kernel(int T, int d, int Epad, const int* __restrict__ tok_ptr,
+                                                               const int* __restrict__ pair_expert,
+                                                               const float* __restrict__ pair_gate,
+                                                               const float* __restrict__ dS,
+                                                               const int* __restrict__ pos,
+                                                               const float* __restrict__ WrT,
+                                                               __nv_bfloat16* __restrict__ dz_split,
+                                                               __nv_bfloat16* __restrict__ dX) {
+  pdl_wait();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
+  auto ds_of = [&](int p) { return dS[pos ? pos[p] : p]; };
+  float inner = 0.f;
+  for (int p = p0 + lane; p < p1; p += 32) inner += pair_gate[p] * ds_of(p);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) inner += __shfl_xor_sync(0xffffffffu, inner, o);
+  __nv_bfloat16* row = dz_split + (size_t)t * 2 * Epad;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+  for (int c = lane; c < 2 * Epad; c += 32) row[c] = zero;
+  __syncwarp();
+  for (int p = p0 + lane; p < p1; p += 32) {
+    const float dz = pair_gate[p] * (ds_of(p) - inner);
+    const int e = pair_expert[p];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(dz);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(dz - __bfloat162float(hi));
+    const int col = (e >> 6) * 128 + (e & 63);
+    row[col] = hi;
+    row[col + 64] = lo;
+  }
+  // dX row: 8 columns per lane per step
+  uint4* xr = reinterpret_cast<uint4*>(dX + (size_t)t * d);
+  for (int c8 = lane; c8 < d / 8; c8 += 32) {
+    float acc[8];
+    const uint4 v = xr[c8];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      acc[2 * i] = f.x;
+      acc[2 * i + 1] = f.y;
+    }
+    for (int p = p0; p < p1; ++p) {
+      const float dz = pair_gate[p] * (ds_of(p) - inner);
+      const float4* w = reinterpret_cast<const float4*>(WrT + (size_t)pair_expert[p] * d) + 2 * c8;
+      const float4 a = __ldg(w), b = __ldg(w + 1);
+      acc[0] = fmaf(dz, a.x, acc[0]);
+      acc[1] = fmaf(dz, a.y, acc[1]);
+      acc[2] = fmaf(dz, a.z, acc[2]);
+      acc[3] = fmaf(dz, a.w, acc[3]);
+      acc[4] = fmaf(dz, b.x, acc[4]);
+      acc[5] = fmaf(dz, b.y, acc[5]);
+      acc[6] = fmaf(dz, b.z, acc[6]);
+      acc[7] = fmaf(dz, b.w, acc[7]);
+    }
+    xr[c8] = pack8(acc);
+  }
+}
+
+cudaError_t launch_router_bwd_given(int T, int d, int E, int Epad, const int* tok_ptr, const int* pair_expert,
+                                    const float* pair_gate, const float* dS, const int* pos, const float* Wr,
+                                    float* WrT, __nv_bfloat16* dz_split, __nv_bfloat16* dX, cudaStream_t s) {
+  const int nb = ((E + 31) / 32) * ((d + 31) / 32);
+  launch_pdl(wr_transpose_kernel, dim3(nb), dim3(256), 0, s, Wr, WrT, d, E);
+  launch_pdl(router_bwd_given_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, s, T, d, Epad, tok_ptr,
+             pair_expert, pair_gate, dS, pos, (const float*)WrT, dz_split, dX);
+  return cudaGetLastError();
+}
 
 // dWr[i, e] = sum over K splits of the split-K partials, in split order
 __global__ void dwr_reduce_kernel(int d, int E, int Epad, int splits, const float* __restrict__ part,
@@ -223,7 +309,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
 
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a0, cudaStream_t s) {
   BwdPrepArgs a = a0;
-  a.tok_blocks = a.router ? (a.T + 7) / 8 : 0;
+  a.tok_blocks = (a.router || a.pair_dS) ? (a.T + 7) / 8 : 0;
   a.tr_blocks = a.router ? ((a.E + 31) / 32) * ((a.d + 31) / 32) : 0;
   launch_pdl(bwd_prep_kernel, dim3(a.tok_blocks + a.tr_blocks + 1), dim3(256), 0, s, a);
   return cudaGetLastError();

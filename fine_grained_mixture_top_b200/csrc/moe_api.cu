@@ -596,6 +596,36 @@ moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const v
   return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// dWr = X^T dz: the split-K tensor-core GEMM over the bf16 hi/lo split of dz
+// (w.dz_split, written before), then the reduction of the splits in order.
+// Returns the first failing CUDA status (tensor-map failures as
+// cudaErrorInvalidValue).
+cudaError_t run_dwr(const Plan& p, const moe_routing* rt, const BwdWs& w, const void* X, float* dWr, int* status,
+                    int sms, cudaStream_t st) {
+  GemmParams g = base_params(p, rt, status);
+  if (!make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 64) ||
+      !make_tmap(&g.tmB, w.dz_split, (uint64_t)p.T, (uint64_t)2 * p.Epad, 64, 64))
+    return cudaErrorInvalidValue;
+  g.num_m_tiles = (int)cdiv(p.d, 128);
+  g.num_n_tiles = p.Epad / 64;
+  g.ksplit = p.ksplit;
+  g.ksplit_rows = p.ksplit_rows;
+  g.outf = w.dWr_part;
+  {
+    ProfScope ps(st, "router_dwr_gemm");
+    cudaError_t e = launch_gemm(G_DWR, 128, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st);
+    if (e != cudaSuccess) return e;
+  }
+  ProfScope ps(st, "router_dwr_reduce");
+  return launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st);
+}
+}  // namespace
+
+extern "C" {
+
 moe_status moe_backward(const moe_dims* dims, const moe_opts* opts, const void* dO, const void* X, const float* Wr,
                         const void* W1, const void* W2, const moe_routing* rt, const void* H, void* dX, void* dW1,
                         void* dW2, float* dWr, void* ws, size_t ws_bytes, void* stream) {
@@ -665,6 +695,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     a.counts = rt->counts;
     a.expert_order = w.expert_order;
     a.sched = w.sched;
+    a.pair_dS = rt->pair_dS;
     ProfScope ps(st, "bwd_prep");
     MOE_TRY_CUDA(launch_bwd_prep(a, st));
   }
@@ -717,31 +748,108 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     ProfScope ps(st, "dxt_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
-  if (rg) {
-    GemmParams g = base_params(p, rt, status);
-    MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 64));
-    MOE_TRY_MAP(make_tmap(&g.tmB, w.dz_split, (uint64_t)p.T, (uint64_t)2 * p.Epad, 64, 64));
-    g.num_m_tiles = (int)cdiv(p.d, 128);
-    g.num_n_tiles = p.Epad / 64;
-    g.ksplit = p.ksplit;
-    g.ksplit_rows = p.ksplit_rows;
-    g.outf = w.dWr_part;
-    {
-      ProfScope ps(st, "router_dwr_gemm");
-      MOE_TRY_CUDA(launch_gemm(G_DWR, 128, 4, g,
-                               grid_for((int64_t)g.num_m_tiles * g.num_n_tiles * p.ksplit, sms), st));
-    }
-    {
-      ProfScope ps(st, "router_dwr_reduce");
-      MOE_TRY_CUDA(launch_dwr_reduce(p.d, p.E, p.Epad, p.ksplit, w.dWr_part, dWr, st));
-    }
-  }
+  if (rg) MOE_TRY_CUDA(run_dwr(p, rt, w, X, dWr, status, sms, st));
   record_ready(grad_ready, 2, st);  // dWr final (or nothing to wait for without the router path)
   {
     ProfScope ps(st, "aggregate_bwd");
     MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, rt->pair_row, w.dXt,
                                       static_cast<__nv_bfloat16*>(dX), st));
   }
+  return MOE_OK;
+}
+
+moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
+                           size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  RouteWs w;
+  if (!ws || ws_bytes < carve_route(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_route(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouteArgs a = route_args(p, rt, w);
+  a.st.word = status;
+  {
+    ProfScope ps(st, "given_pairs");
+    MOE_TRY_CUDA(launch_given_pairs((int)p.T, p.K, p.E, rt->topk_idx, rt->topk_gate, rt->tok_ptr, rt->pair_expert,
+                                    rt->pair_gate, a.st, st));
+  }
+  MOE_TRY_CUDA(launch_permute(a, st));
+  return MOE_OK;
+}
+
+moe_status moe_ep_pack(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const void* src,
+                       void* send_rows, float* send_gate, int32_t* pair_pos, void* ws, size_t ws_bytes,
+                       void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  if (send_rows && (!src || !aligned16(src) || !aligned16(send_rows))) return MOE_ERR_INVALID_ARG;
+  if ((send_gate && !aligned16(send_gate)) || (pair_pos && !aligned16(pair_pos))) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < (size_t)(p.E + 1) * sizeof(int)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope ps(st, "ep_pack");
+  MOE_TRY_CUDA(launch_ep_pack((int)p.T, p.d, p.E, p.R_max, p.P_max, rt->tok_ptr, rt->pair_expert, rt->pair_row,
+                              rt->counts, rt->offsets, rt->tile_expert, rt->row_tok, rt->row_gate,
+                              static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(send_rows),
+                              send_gate, pair_pos, static_cast<int*>(ws), st));
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const int32_t* pair_pos,
+                          const void* rows, void* out, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {pair_pos, rows, out};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope ps(st, "ep_combine");
+  MOE_TRY_CUDA(launch_aggregate_bwd((int)p.T, p.d, rt->tok_ptr, pair_pos, static_cast<const __nv_bfloat16*>(rows),
+                                    static_cast<__nv_bfloat16*>(out), st));
+  return MOE_OK;
+}
+
+moe_status moe_router_backward(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
+                               const moe_routing* rt, const float* dS, const int32_t* pair_pos, void* dX, float* dWr,
+                               void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  const void* ptrs[] = {X, Wr, dS, dX, dWr};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (pair_pos && !aligned16(pair_pos)) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
+  BwdWs w;
+  if (!ws || ws_bytes < carve_bwd(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_bwd(p, ws, &w);
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    ProfScope ps(st, "router_bwd_given");
+    MOE_TRY_CUDA(launch_router_bwd_given((int)p.T, p.d, p.E, p.Epad, rt->tok_ptr, rt->pair_expert, rt->pair_gate, dS,
+                                         pair_pos, Wr, w.WrT, w.dz_split, static_cast<__nv_bfloat16*>(dX), st));
+  }
+  MOE_TRY_CUDA(run_dwr(p, rt, w, X, dWr, status, sms, st));
   return MOE_OK;
 }
 

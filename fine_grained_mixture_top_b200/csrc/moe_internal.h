@@ -109,6 +109,7 @@ struct BwdPrepArgs {
   const int* counts;           // [E]
   int* expert_order;           // [E]
   int* sched;                  // [16] weight-gradient tile counters, zeroed here
+  float* pair_dS;              // [P] dS of each pair, or null
   int tok_blocks, tr_blocks;   // set by the launcher
 };
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t s);
@@ -116,6 +117,18 @@ cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* p
 cudaError_t launch_aggregate_bwd(int T, int d, const int* tok_ptr, const int* pair_row, const __nv_bfloat16* dXt,
                                  __nv_bfloat16* dX, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* flag, DevStatus st, cudaStream_t s);
+cudaError_t launch_router_bwd_given(int T, int d, int E, int Epad, const int* tok_ptr, const int* pair_expert,
+                                    const float* pair_gate, const float* dS, const int* pos, const float* Wr,
+                                    float* WrT, __nv_bfloat16* dz_split, __nv_bfloat16* dX, cudaStream_t s);
+
+// ---- caller-given routing and expert parallelism (moe_ep.cu)
+cudaError_t launch_given_pairs(int T, int K, int E, const int* topk_idx, const float* topk_gate, int* tok_ptr,
+                               int* pair_expert, float* pair_gate, DevStatus st, cudaStream_t s);
+cudaError_t launch_ep_pack(int T, int d, int E, int64_t R_max, int64_t P_max, const int* tok_ptr,
+                           const int* pair_expert, const int* pair_row, const int* counts, const int* offsets,
+                           const int* tile_expert, const int* row_tok, const float* row_gate,
+                           const __nv_bfloat16* src, __nv_bfloat16* send, float* send_gate, int* pair_pos, int* cum,
+                           cudaStream_t s);
 
 // ---- MXFP8 quantization (moe_mx.cu)
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16* in, int64_t rows, int K, uint8_t* codes, uint8_t* scales,

@@ -34,7 +34,8 @@ _ROUTING_PTRS = ["logits", "probs", "topk_idx", "topk_gate", "tok_ptr", "pair_ex
 
 
 class MoeRouting(ctypes.Structure):
-    _fields_ = [(name, c_void_p) for name in _ROUTING_PTRS] + [("P_max", c_int64), ("R_max", c_int64)]
+    _fields_ = [(name, c_void_p) for name in _ROUTING_PTRS] + [("P_max", c_int64), ("R_max", c_int64),
+                                                                ("pair_dS", c_void_p)]
 
 
 class MoeSizes(ctypes.Structure):
@@ -81,6 +82,12 @@ def lib() -> ctypes.CDLL:
                                       P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       ctypes.c_size_t, P(c_void_p), c_void_p]
         L.moe_set_sm_budget.argtypes = [c_int32]
+        L.moe_route_given.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, ctypes.c_size_t, c_void_p]
+        L.moe_ep_pack.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, ctypes.c_size_t, c_void_p]
+        L.moe_ep_combine.argtypes = [P(MoeDims), P(MoeOpts), P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p]
+        L.moe_router_backward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, P(MoeRouting), c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
         L.moe_mx_quantize_rows.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
         L.moe_mx_quantize_cols.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
         L.moe_get_status.argtypes = [c_void_p, P(c_int32)]
@@ -100,7 +107,8 @@ def lib() -> ctypes.CDLL:
         L.moe_last_error.restype = ctypes.c_char_p
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
                   "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout", "moe_backward_ev",
-                  "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols", "moe_forward_mxfp8"):
+                  "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols", "moe_forward_mxfp8",
+                  "moe_route_given", "moe_ep_pack", "moe_ep_combine", "moe_router_backward"):
             getattr(L, f).restype = c_int32
         _lib = L
     return _lib
@@ -155,7 +163,8 @@ class Routing:
         return self.tensors[k]
 
     @classmethod
-    def allocate(cls, dims: MoeDims, sizes: MoeSizes, device="cuda", with_logits: bool = True) -> "Routing":
+    def allocate(cls, dims: MoeDims, sizes: MoeSizes, device="cuda", with_logits: bool = True,
+                 with_pair_ds: bool = False) -> "Routing":
         import torch
         T, E, K = dims.T, dims.E, dims.K
         P, R = sizes.P_max, sizes.R_max
@@ -171,7 +180,8 @@ class Routing:
                 t[k] = None
                 continue
             t[k] = torch.empty(shape, dtype=dt, device=device)
-        st = MoeRouting(*[_ptr(t[k]) for k in _ROUTING_PTRS], P, R)
+        t["pair_dS"] = torch.empty((P,), dtype=f32, device=device) if with_pair_ds else None
+        st = MoeRouting(*[_ptr(t[k]) for k in _ROUTING_PTRS], P, R, _ptr(t["pair_dS"]))
         return cls(t, st)
 
 
@@ -179,6 +189,31 @@ def moe_route(dims, opts, X, Wr, bias, routing: Routing, ws, stream=None):
     _check(lib().moe_route(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(Wr), _ptr(bias),
                            ctypes.byref(routing.struct), _ptr(ws), ws.numel() * ws.element_size(),
                            _stream(stream)), "moe_route")
+
+
+def moe_route_given(dims, opts, routing: Routing, ws, stream=None):
+    """Permutation of a caller-given selection (routing['topk_idx'],
+    routing['topk_gate'] filled by the caller)."""
+    _check(lib().moe_route_given(ctypes.byref(dims), ctypes.byref(opts), ctypes.byref(routing.struct), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "moe_route_given")
+
+
+def moe_ep_pack(dims, opts, routing: Routing, src, send_rows, send_gate, pair_pos, ws, stream=None):
+    _check(lib().moe_ep_pack(ctypes.byref(dims), ctypes.byref(opts), ctypes.byref(routing.struct), _ptr(src),
+                             _ptr(send_rows), _ptr(send_gate), _ptr(pair_pos), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "moe_ep_pack")
+
+
+def moe_ep_combine(dims, opts, routing: Routing, pair_pos, rows, out, stream=None):
+    _check(lib().moe_ep_combine(ctypes.byref(dims), ctypes.byref(opts), ctypes.byref(routing.struct),
+                                _ptr(pair_pos), _ptr(rows), _ptr(out), _stream(stream)), "moe_ep_combine")
+
+
+def moe_router_backward(dims, opts, X, Wr, routing: Routing, dS, pair_pos, dX, dWr, ws, stream=None):
+    _check(lib().moe_router_backward(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(Wr),
+                                     ctypes.byref(routing.struct), _ptr(dS), _ptr(pair_pos), _ptr(dX), _ptr(dWr),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_router_backward")
 
 
 def moe_route_noalloc(dims, opts, X, Wr, bias, routing: Routing, stream=None):

@@ -84,6 +84,9 @@ typedef struct {
  *                                      rows hold token -1 and gate 0; inside a
  *                                      segment rows ascend in token order
  *   tile_expert[R_max/128]             expert of each 128-row tile
+ *   pair_dS[P_max] (nullable)          if set, moe_backward writes the router
+ *                                      score gradient dS of every pair there
+ *                                      (fp32), with or without router_grad
  */
 typedef struct {
   float* logits;
@@ -101,6 +104,7 @@ typedef struct {
   int32_t* tile_expert;
   int64_t P_max;
   int64_t R_max;
+  float* pair_dS;
 } moe_routing;
 
 typedef struct {
@@ -126,6 +130,21 @@ moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes
  */
 moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
                      const float* bias, const moe_routing* rt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Routing given by the caller: rt->topk_idx[T,K] (experts, distinct within a
+ * token, each in [0, E)) and rt->topk_gate[T,K] are inputs here.  Builds the
+ * pairs (token t's pairs are t*K .. t*K+K-1, in slot order) and the
+ * permutation exactly as moe_route does after its top-K; logits and probs
+ * are neither read nor written (so moe_token_round and the router path of
+ * moe_backward do not apply).  A token whose selection breaks the rules is
+ * replaced by experts 0..K-1 with gate 0 and reported as
+ * MOE_ERR_DEVICE_CHECK by moe_get_status.  ws of moe_sizes.route_ws bytes.
+ * Used by the expert ranks of expert parallelism, whose "tokens" are the
+ * rows they receive, each with one expert (K = 1) and its gate.
+ */
+moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /*
  * Token rounding ([P2] scheduling paragraph): rounds every expert's token
@@ -199,6 +218,45 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
                            const float* Wr, const void* W1, const void* W2, const moe_routing* rt, const void* H,
                            void* dX, void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes,
                            void* const* grad_ready, void* stream);
+
+/*
+ * Expert parallelism (named as future work of the method, page
+ * "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE", closing paragraph: a token
+ * all-to-all before the up-projection and after the down-projection).  The
+ * exchange is the caller's; these calls lay the rows out for it.  The send
+ * order is expert-major without padding: expert e's rows (its tokens in
+ * ascending order) start at sum_{e'<e} counts[e'], so experts owned by one
+ * rank form one contiguous block per destination.
+ *
+ * moe_ep_pack: send_rows[j] = src[token of row j] for the P routed rows
+ *   (src[T,d] bf16: X in the forward, dO in the backward; send_rows [P,d]
+ *   bf16, may be NULL), send_gate[j] = its gate (f32, may be NULL) and
+ *   pair_pos[p] = j for each pair p (i32, may be NULL).  ws: at least
+ *   4*(E+1) bytes (moe_sizes.route_ws is enough).
+ * moe_ep_combine: out[t] = sum over token t's pairs p of rows[pair_pos[p]]
+ *   (rows [P,d] bf16 in send order, as they come back; out [T,d] bf16,
+ *   overwritten; fp32 sums in pair order).  The expert ranks apply the gates.
+ */
+moe_status moe_ep_pack(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const void* src,
+                       void* send_rows, float* send_gate, int32_t* pair_pos, void* ws, size_t ws_bytes,
+                       void* stream);
+moe_status moe_ep_combine(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const int32_t* pair_pos,
+                          const void* rows, void* out, void* stream);
+
+/*
+ * The router path of the backward from router score gradients computed
+ * elsewhere (under expert parallelism, by the ranks that own the experts):
+ *   dS: fp32, dS of pair p at dS[pair_pos[p]] (pair_pos may be NULL: dS[p]);
+ *   dz = s (dS - sum s dS) over each token's experts ([P1] "MoE 与它的隐患";
+ *   [P2] algorithm paragraph: the router gradient from dS without Y);
+ *   dX[T,d] bf16 += dz Wr^T (read, updated, written back);
+ *   dWr[d,E] f32 = X^T dz (overwritten).
+ * X[T,d] bf16, Wr[d,E] f32, rt: the routing of moe_route.  ws of
+ * moe_sizes.bwd_ws bytes.
+ */
+moe_status moe_router_backward(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
+                               const moe_routing* rt, const float* dS, const int32_t* pair_pos, void* dX, float* dWr,
+                               void* ws, size_t ws_bytes, void* stream);
 
 /*
  * At most `sms` CTAs for each persistent GEMM kernel launched from now on by

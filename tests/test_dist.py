@@ -100,3 +100,66 @@ def test_rank_failing_before_exchange_is_reported_not_hung():
             p.kill()
     assert res != "no error"
     assert procs[1].exitcode == 3
+
+
+# ----------------------------------------------------------------------------
+# Expert parallelism: experts split over the ranks, routed rows exchanged by
+# all-to-all.  The plan and the exchanges are the product's
+# (fine_grained_mixture_top_b200.ep); the arithmetic is the oracle's.
+# ----------------------------------------------------------------------------
+def _ep_worker(rank, world, port, K, T, E, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from fine_grained_mixture_top_b200.ep import ExpertParallelMoE
+    from ep_oracle_engine import OracleEngine
+    X, W1, W2, Wr, b, dO = _layer(seed=5, T=T * world, E=E)
+    sl = slice(rank * T, (rank + 1) * T)
+    E_loc = E // world
+    es = slice(rank * E_loc, (rank + 1) * E_loc)
+    ep = ExpertParallelMoE(T, X.shape[1], E, W2.shape[1], K, OracleEngine(E, K, world))
+    t = torch.from_numpy
+    O = ep.forward(t(X[sl].copy()), t(Wr), t(b), t(W1[es].copy()), t(W2[es].copy()))
+    dX, dW1, dW2, dWr = ep.backward(t(dO[sl].copy()), t(X[sl].copy()), t(Wr), t(W1[es].copy()), t(W2[es].copy()))
+    out_q.put((rank, O.numpy(), dX.numpy(), dW1.numpy(), dW2.numpy(), dWr.numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E,K", [(2, 6, 2), (3, 6, 3), (2, 8, 1)])
+def test_expert_parallel_equals_full_batch(world, E, K):
+    """Each rank holds E/world experts and its own tokens; O, dX, its experts'
+    dW1/dW2 and the all-reduced dWr equal the single-process full batch."""
+    T = 40
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, K, T, E, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r[0], r[1:]) for r in (q.get(timeout=180) for _ in range(world)))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W1, W2, Wr, b, dO = _layer(seed=5, T=T * world, E=E)
+    fw = orc.forward(X, Wr, b, W1, W2, K)
+    bw = orc.backward(fw, dO, X, Wr, W1, W2)
+    E_loc = E // world
+    for r in range(world):
+        O, dX, dW1, dW2, dWr = got[r]
+        sl = slice(r * T, (r + 1) * T)
+        es = slice(r * E_loc, (r + 1) * E_loc)
+        np.testing.assert_allclose(O, fw["O"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dX, bw["dX"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dW1, bw["dW1"][es], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dW2, bw["dW2"][es], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dWr, bw["dWr"], rtol=1e-10, atol=1e-12)
+
+
+def test_exchange_plan_orders_rows_by_source_then_expert():
+    from fine_grained_mixture_top_b200.ep import exchange_plan
+    send = np.array([[3, 0], [1, 2], [0, 0]])        # this rank's rows for experts (g, l)
+    recv = np.array([[2, 1], [0, 4], [1, 0]])        # rows rank g sends for local expert l
+    ss, rs, le = exchange_plan(send, recv)
+    assert ss == [3, 3, 0] and rs == [3, 4, 1]
+    np.testing.assert_array_equal(le, [0, 0, 1, 1, 1, 1, 1, 0])
