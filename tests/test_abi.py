@@ -89,6 +89,24 @@ def test_invalid_options_and_null_arguments(moe):
     assert L.moe_mx_quantize_rows(None, 4, 32, None, None, None) == 1
     assert L.moe_mx_quantize_rows(None, 4, 48, None, None, None) == 2     # K not a multiple of 32
     assert L.moe_mx_quantize_cols(None, 1, 64, 8, None, None, None) == 1
+    # MXFP8 forward: unsupported n (% 128) before anything else; then arguments
+    assert L.moe_forward_mxfp8(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, ctypes.byref(rt),
+                               None, None, None, 0, None) == 2
+    dims128 = moe.dims_of(512, 128, 16, 128, 2)
+    assert L.moe_forward_mxfp8(ctypes.byref(dims128), ctypes.byref(moe.opts_of()), None, None, None,
+                               ctypes.byref(rt), None, None, None, 0, None) == 1
+    assert moe.query_sizes(dims128, moe.opts_of()).fwd_mx_ws > 0
+    assert moe.query_sizes(dims, moe.opts_of()).fwd_mx_ws == 0      # n = 64: no MXFP8 forward
+    # expert-parallel and given-routing entry points
+    assert L.moe_route_given(ctypes.byref(dims), ctypes.byref(moe.opts_of()), ctypes.byref(rt), None, 0, None) == 1
+    assert L.moe_ep_pack(ctypes.byref(dims), ctypes.byref(moe.opts_of()), ctypes.byref(rt), None, None, None, None,
+                         None, 0, None) == 1
+    assert L.moe_ep_combine(ctypes.byref(dims), ctypes.byref(moe.opts_of()), ctypes.byref(rt), None, None, None,
+                            None) == 1
+    assert L.moe_router_backward(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, ctypes.byref(rt),
+                                 None, None, None, None, None, 0, None) == 1
+    assert L.moe_route_given(ctypes.byref(moe.dims_of(512, 100, 16, 64, 2)), ctypes.byref(moe.opts_of()),
+                             ctypes.byref(rt), None, 0, None) == 2
     assert moe.last_error() == ""  # no CUDA error on this thread
 
 
