@@ -1147,10 +1147,15 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           }
         }
         if constexpr (kDyn) {
-          // Publish the tile's last k-blocks before taking the next tile from
-          // the queue: a stage held back across tiles would make the MMA wait
-          // on a tile the producer cannot publish while the queue is full.
-          if (ok && pending > 0) {
+          // Before blocking on the queue for the next tile, publish this
+          // tile's last k-blocks: a stage held back while this warp waits on
+          // the queue would make the MMA wait on it while the queue, full of
+          // tiles the MMA has not taken, cannot move.  When the next tile is
+          // already queued nothing blocks, and the held k-blocks are
+          // published as that tile's first copies go out, so the copy
+          // pipeline runs on across the tile boundary.
+          if (ok && pending > 0 &&
+              !mbar_test_wait(smem_u32(&tq_full[(ti + 1) % kTileQ]), ((ti + 1) / kTileQ) & 1)) {
             cp_async_wait<0>();
             fence_proxy_async_smem();
             for (int k = pending; k > 0; --k) mbar_arrive(smem_u32(&g_full[(it - k) % GS]));
