@@ -160,3 +160,27 @@ def test_mxfp8_forward_rejects_unsupported_n():
     layer.route(inp["X"], inp["Wr"], inp["bias"])
     with pytest.raises(moe.MoEError):
         layer.forward(inp["X"], inp["W1"], inp["W2"], mxfp8=True)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", [1, 2])
+def test_mxfp8_forward_after_token_rounding(mode):
+    """Token-rounded routing (every expert a multiple of 128 rows, tokens
+    with a varying number of experts) feeds the MXFP8 forward unchanged."""
+    from fine_grained_mixture_top_b200 import moe
+    cfg = MoEConfig("mx_tr", T=1500, d=256, E=16, n=128, K=2, w_std=0.05, bias="normal", seed=26,
+                    round_mode=mode)
+    inp = make_inputs(cfg, "cuda", need_grad_inputs=False)
+    layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=mode, seed=cfg.seed)
+    layer.route(inp["X"], inp["Wr"], inp["bias"])
+    layer.forward(inp["X"], inp["W1"], inp["W2"], mxfp8=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    g = P.gpu_routing(layer, cfg.T)
+    assert np.all(g["counts"] % 128 == 0)
+    X, Wr, W1, W2 = (P.f64(inp[k]) for k in ("X", "Wr", "W1", "W2"))
+    rt = {"tok_ptr": g["tok_ptr"], "pair_expert": g["pair_expert"], "pair_gate": g["pair_gate"]}
+    fq = mx.forward_mxfp8(X, Wr, None, W1, W2, cfg.K, routing=rt)
+    err = P.normwise(P.f64(layer.O), fq["O"])
+    print("mx_tr", mode, f"O {err:.2e}")
+    assert err <= P.TOL_BF16
