@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--ref-sample-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "ep"],
+                    help="dp: every rank holds all experts and its own tokens, weight gradients all-reduced; "
+                         "ep: rank r holds experts [rE/N, (r+1)E/N), routed rows exchanged by all-to-all")
     ap.add_argument("--mxfp8-forward", action="store_true",
                     help="forward GEMMs on MXFP8 operands (moe_forward_mxfp8); backward unchanged")
     ap.add_argument("--comm-sms", type=int, default=16,
@@ -237,6 +240,15 @@ def run_reference(args):
     return 0
 
 
+def _free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse_args()
@@ -274,12 +286,35 @@ def main():
     if args.mxfp8_forward:
         workload += "; forward GEMMs on MXFP8 operands (E4M3, E8M0 scale per 32 along K)"
     stream = torch.cuda.current_stream()
+    ep = None
+    if args.parallel == "ep":
+        if args.mxfp8_forward:
+            raise SystemExit("--parallel ep runs the bf16 forward")
+        if world == 1:  # the all-to-alls still need a (one-rank) group
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(_free_port()))
+            dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=180),
+                                    device_id=dev)
+        from fine_grained_mixture_top_b200.ep import CudaEngine, ExpertParallelMoE
+        E_loc = cfg.E // world
+        W1 = W1[rank * E_loc:(rank + 1) * E_loc].contiguous()
+        W2 = W2[rank * E_loc:(rank + 1) * E_loc].contiguous()
+        eng = CudaEngine(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, world, device=dev, seed=cfg.seed,
+                         round_mode=cfg.round_mode)
+        ep = ExpertParallelMoE(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, eng)
+        layer = eng  # routing statistics below
+        overlap = False
+        workload += f"; expert parallel over {world} rank(s), {E_loc} experts each, all-to-all of routed rows"
     if overlap:
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         moe.moe_set_sm_budget(sms - args.comm_sms)
         reducer = moe.OverlappedGradReduce(layer)
 
     def step():
+        if ep is not None:
+            ep.forward(X, Wr, b, W1, W2)
+            ep.backward(dO, X, Wr, W1, W2)
+            return
         if overlap:
             reducer.step(X, Wr, b, W1, W2, dO)
             return
@@ -414,13 +449,25 @@ def main():
         Xh = X.cpu().pin_memory()
         dOh = dO.cpu().pin_memory()
         Oh = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
-        runner = moe.HostFedRunner(layer)
+        if ep is None:
+            runner = moe.HostFedRunner(layer)
 
-        def e2e_step():
-            runner.step(Xh, dOh, Oh, Wr, b, W1, W2)
-            if world > 1:
-                for g in (layer.dW1, layer.dW2, layer.dWr):
-                    dist.all_reduce(g)
+            def e2e_step():
+                runner.step(Xh, dOh, Oh, Wr, b, W1, W2)
+                if world > 1:
+                    for g in (layer.dW1, layer.dW2, layer.dWr):
+                        dist.all_reduce(g)
+        else:
+            class _Copies:  # host copies in line with the expert-parallel step
+                def finish(self):
+                    pass
+            runner = _Copies()
+
+            def e2e_step():
+                X.copy_(Xh, non_blocking=True)
+                dO.copy_(dOh, non_blocking=True)
+                Oh.copy_(ep.forward(X, Wr, b, W1, W2), non_blocking=True)
+                ep.backward(dO, X, Wr, W1, W2)
 
         for _ in range(3):
             e2e_step()
@@ -469,9 +516,11 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16+mxfp8" if args.mxfp8_forward else "bf16", "data": "synthetic",
             "config": {"workload": workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
                        "router_bias": cfg.bias, "round_mode": cfg.round_mode,
-                       "parallelism": f"dp{world}" + ((" (NCCL all-reduce of dW2, dW1, dWr overlapping the backward, "
-                                                       f"{args.comm_sms} SMs left to NCCL)") if overlap else
-                                                      (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else "")),
+                       "parallelism": (f"ep{world} (NCCL all-to-all of routed rows and dS, all-reduce of dWr)"
+                                       if ep is not None else
+                                       f"dp{world}" + ((" (NCCL all-reduce of dW2, dW1, dWr overlapping the backward, "
+                                                        f"{args.comm_sms} SMs left to NCCL)") if overlap else
+                                                       (" (NCCL all-reduce of dW1, dW2, dWr)" if world > 1 else ""))),
                        "l2": "inputs larger than L2 (%d MB of X, dO, W1, W2 per step)" % (
                            (4 * cfg.T * cfg.d + 6 * cfg.E * cfg.d * cfg.n) // 2**20)},
             "tokens_per_s": round(cfg.T * world / (ms_step * 1e-3), 1),

@@ -121,16 +121,17 @@ class CudaEngine:
     E/G experts, K = 1): moe_route_given, moe_forward, moe_backward with the
     per-row dS written to the routing's pair_dS.  Buffers are allocated once
     for T tokens per rank; the expert side is sized for the most rows it can
-    receive, G * T * K."""
+    receive, G times this rank's pair capacity.  round_mode: token rounding
+    of this rank's routing before the exchange."""
 
-    def __init__(self, T, d, E, n, K, G, device="cuda", seed=0):
+    def __init__(self, T, d, E, n, K, G, device="cuda", seed=0, round_mode=0):
         import torch
         from . import moe
         self.moe = moe
         self.T, self.d, self.E, self.n, self.K, self.G = T, d, E, n, K, G
         self.E_loc = E // G
         self.dims = moe.dims_of(T, d, E, n, K)
-        self.opts = moe.opts_of(0, 1, seed)
+        self.opts = moe.opts_of(round_mode, 1, seed)
         self.sizes = moe.query_sizes(self.dims, self.opts)
         self.routing = moe.Routing.allocate(self.dims, self.sizes, device)
         u8, bf, f32, i32 = torch.uint8, torch.bfloat16, torch.float32, torch.int32
@@ -143,7 +144,7 @@ class CudaEngine:
         self.O = torch.empty(T, d, dtype=bf, device=device)
         self.dX = torch.empty(T, d, dtype=bf, device=device)
         self.dWr = torch.empty(d, E, dtype=f32, device=device)
-        cap = G * T * K
+        cap = G * self.sizes.P_max  # every rank may send all its routed rows here
         self.loc_opts = moe.opts_of(0, 0, 0)
         self.loc_sizes = moe.query_sizes(moe.dims_of(cap, d, self.E_loc, n, 1), self.loc_opts)
         self.loc_routing = moe.Routing.allocate(moe.dims_of(cap, d, self.E_loc, n, 1), self.loc_sizes, device,
@@ -161,6 +162,8 @@ class CudaEngine:
 
     def route(self, X, Wr, bias):
         self.moe.moe_route(self.dims, self.opts, X, Wr, bias, self.routing, self.ws_route)
+        if self.opts.round_mode:
+            self.moe.moe_token_round(self.dims, self.opts, self.routing, self.ws_route)
 
     def counts(self):
         return self.routing["counts"]
