@@ -62,9 +62,9 @@ __global__ void __launch_bounds__(1024) ep_scan_kernel(int E, const int* __restr
   if (i == 0) cum[0] = 0;
 }
 
-// One thread per (padded row, 16-byte chunk of d): the row's real position j
-// in expert-major order (padding rows are skipped), send[j] = src[token],
-// and the chunk-0 thread writes the gate.
+// One warp per padded row: the row's real position j in expert-major order
+// (padding rows are skipped), send[j] = src[token] in 16-byte pieces, four
+// loads in flight per lane, and lane 0 writes the gate.
 __global__ void __launch_bounds__(256) ep_pack_kernel(int64_t R_max, int d8, const int* __restrict__ offsets, int E,
                                                       const int* __restrict__ counts, const int* __restrict__ cum,
                                                       const int* __restrict__ tile_expert,
@@ -72,17 +72,25 @@ __global__ void __launch_bounds__(256) ep_pack_kernel(int64_t R_max, int d8, con
                                                       const uint4* __restrict__ src, uint4* __restrict__ send,
                                                       float* __restrict__ send_gate) {
   pdl_wait();
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= R_max * d8) return;
-  const int r = (int)(g / d8);
-  const int c = (int)(g - (int64_t)r * d8);
-  if (r >= __ldg(offsets + E)) return;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= R_max || r >= __ldg(offsets + E)) return;
   const int e = __ldg(tile_expert + (r >> 7));
-  const int i = r - __ldg(offsets + e);
+  const int i = (int)r - __ldg(offsets + e);
   if (i >= __ldg(counts + e)) return;  // padding row
   const int64_t j = (int64_t)__ldg(cum + e) + i;
-  send[j * d8 + c] = __ldg(src + (size_t)__ldg(row_tok + r) * d8 + c);
-  if (c == 0 && send_gate) send_gate[j] = __ldg(row_gate + r);
+  const uint4* s = src + (size_t)__ldg(row_tok + r) * d8;
+  uint4* o = send + j * d8;
+  for (int c = lane; c < d8; c += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c + 32 * u < d8) v[u] = __ldg(s + c + 32 * u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c + 32 * u < d8) o[c + 32 * u] = v[u];
+  }
+  if (lane == 0 && send_gate) send_gate[j] = __ldg(row_gate + r);
 }
 
 // pair_pos[p] = position of pair p's row in the send order.
@@ -112,8 +120,7 @@ cudaError_t launch_ep_pack(int T, int d, int E, int64_t R_max, int64_t P_max, co
   launch_pdl(ep_scan_kernel, dim3(1), dim3(1024), 0, s, E, counts, cum);
   const int d8 = d / 8;
   if (send) {
-    const int64_t n = R_max * d8;
-    launch_pdl(ep_pack_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, R_max, d8, offsets, E, counts,
+    launch_pdl(ep_pack_kernel, dim3((unsigned)((R_max + 7) / 8)), dim3(256), 0, s, R_max, d8, offsets, E, counts,
                (const int*)cum, tile_expert, row_tok, row_gate, reinterpret_cast<const uint4*>(src),
                reinterpret_cast<uint4*>(send), send_gate);
   }
