@@ -214,10 +214,14 @@ struct FwdWs {
   __nv_bfloat16* Y;
 };
 // MXFP8 forward: codes and scales of X, W1, W2 and A, and Y
-struct MxFwdWs {
-  uint8_t *Xq, *SX;            // [T, d], [T, d/32]
+// MXFP8 expert weights: codes K-major and scales in the MMA's tile layout
+struct MxWeights {
   uint8_t *W1q, *SW1t;         // [E, 2n, d], scale tiles [E][n/64][d/128]
   uint8_t *W2q, *SW2t;         // [E, d, n], scale tiles [E][d/128][n/128]
+};
+struct MxFwdWs {
+  MxWeights wt;                // filled by the quantizing forward; unused with pre-quantized weights
+  uint8_t *Xq, *SX;            // [T, d], [T, d/32]
   uint8_t *Aq, *SA;            // [R_max, n], scale tiles [R_max/128][n/128]
   __nv_bfloat16* Y;            // [R_max, d]
 };
@@ -230,15 +234,26 @@ size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
 
 bool mx_supported(const Plan& p) { return p.n % 128 == 0; }
 
-size_t carve_fwd_mx(const Plan& p, void* ws, MxFwdWs* w) {
-  Carve c{static_cast<char*>(ws)};
-  const size_t T = (size_t)p.T, d = p.d, n = p.n, E = p.E, R = (size_t)p.R_max;
-  w->Xq = c.take<uint8_t>(T * d);
-  w->SX = c.take<uint8_t>(T * (d / 32));
+size_t carve_mx_weights(const Plan& p, Carve& c, MxWeights* w) {
+  const size_t d = p.d, n = p.n, E = p.E;
   w->W1q = c.take<uint8_t>(E * 2 * n * d);
   w->SW1t = c.take<uint8_t>(E * (n / 64) * (d / 128) * 512);
   w->W2q = c.take<uint8_t>(E * d * n);
   w->SW2t = c.take<uint8_t>(E * (d / 128) * (n / 128) * 512);
+  return c.off;
+}
+size_t mx_weights_bytes(const Plan& p) {
+  Carve c{nullptr};
+  MxWeights w;
+  return carve_mx_weights(p, c, &w);
+}
+
+size_t carve_fwd_mx(const Plan& p, void* ws, MxFwdWs* w) {
+  Carve c{static_cast<char*>(ws)};
+  const size_t T = (size_t)p.T, d = p.d, n = p.n, R = (size_t)p.R_max;
+  carve_mx_weights(p, c, &w->wt);
+  w->Xq = c.take<uint8_t>(T * d);
+  w->SX = c.take<uint8_t>(T * (d / 32));
   w->Aq = c.take<uint8_t>(R * n);
   w->SA = c.take<uint8_t>((R / 128) * (n / 128) * 512);
   w->Y = c.take<__nv_bfloat16>(R * d);
@@ -391,6 +406,7 @@ moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes
   out->h_elems = p.R_max * 2 * p.n;
   MxFwdWs mw;
   out->fwd_mx_ws = mx_supported(p) ? carve_fwd_mx(p, nullptr, &mw) : 0;
+  out->mx_weights_bytes = mx_supported(p) ? mx_weights_bytes(p) : 0;
   return MOE_OK;
 }
 
@@ -522,51 +538,40 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
   return MOE_OK;
 }
 
-moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
-                             const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
-                             void* stream) {
-  Plan p;
-  moe_status s = make_plan(dims, opts, &p);
-  if (s != MOE_OK) return s;
-  if (!mx_supported(p)) return MOE_ERR_UNSUPPORTED;
-  const void* ptrs[] = {X, W1, W2, O, H};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
-  if (!routing_ok(rt, p, false)) return MOE_ERR_INVALID_ARG;
-  MxFwdWs w;
-  if (!ws || ws_bytes < carve_fwd_mx(p, nullptr, &w)) return MOE_ERR_WORKSPACE;
-  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
-  carve_fwd_mx(p, ws, &w);
-  int dev, sms;
-  int* status;
-  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace {
+// W1, W2 (bf16) to MXFP8 codes, K-major, with their scales in the MMA's tile
+// layout: W1 along d per output column (its tiles hold 64 gate and the same
+// 64 up columns), W2 along n per output column.
+cudaError_t quantize_mx_weights(const Plan& p, const void* W1, const void* W2, const MxWeights& wt, cudaStream_t st) {
+  ProfScope ps(st, "mx_quant_w");
+  cudaError_t e = launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W1), p.E, p.d, 2 * p.n, wt.W1q, nullptr,
+                                       wt.SW1t, 1, st);
+  if (e != cudaSuccess) return e;
+  return launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W2), p.E, p.n, p.d, wt.W2q, nullptr, wt.SW2t, 0, st);
+}
+
+// The MXFP8 forward on quantized weights: X to MXFP8 per row, then the
+// block-scaled up-projection (H bf16 out, A quantized in its epilogue), the
+// block-scaled down-projection and the aggregation.
+moe_status forward_mx(const Plan& p, const void* X, const MxWeights& wt, const moe_routing* rt, void* O, void* H,
+                      const MxFwdWs& w, int* status, int sms, cudaStream_t st) {
   const int64_t mtiles = p.R_max / kTile;
   const int E = p.E, d = p.d, n = p.n;
-
-  // operands to MXFP8: X along d per row; W1 along d and W2 along n per
-  // output column, transposed so that K is contiguous, with their scales
-  // rearranged into the MMA's 512-byte scale tiles
   {
     ProfScope ps(st, "mx_quant_x");
     MOE_TRY_CUDA(launch_mx_quant_rows(static_cast<const __nv_bfloat16*>(X), p.T, d, w.Xq, w.SX, st));
-  }
-  {
-    ProfScope ps(st, "mx_quant_w");
-    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W1), E, d, 2 * n, w.W1q, nullptr, w.SW1t,
-                                      1, st));
-    MOE_TRY_CUDA(launch_mx_quant_cols(static_cast<const __nv_bfloat16*>(W2), E, n, d, w.W2q, nullptr, w.SW2t, 0,
-                                      st));
   }
   // up-projection on MXFP8 operands: H = X[tok] W1[e] (bf16 out), A = SwiGLU(H)
   // quantized to MXFP8 with its scale tiles
   {
     GemmParams g = base_params(p, rt, status);
-    MOE_TRY_MAP(make_tmap_u8(&g.tmB, w.W1q, (uint64_t)E * 2 * n, (uint64_t)d, 128, 64));
+    MOE_TRY_MAP(make_tmap_u8(&g.tmB, wt.W1q, (uint64_t)E * 2 * n, (uint64_t)d, 128, 64));
     g.gsrc = reinterpret_cast<const __nv_bfloat16*>(w.Xq);  // rows of d bytes, gathered in 16-byte chunks
     g.gld = d / 2;
     g.sfa_src = w.SX;
-    g.sfb_src = w.SW1t;
+    g.sfb_src = wt.SW1t;
     g.num_n_tiles = n / 64;
     g.out0 = static_cast<__nv_bfloat16*>(H);
     g.aq_out = w.Aq;
@@ -579,9 +584,9 @@ moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const v
   {
     GemmParams g = base_params(p, rt, status);
     MOE_TRY_MAP(make_tmap_u8(&g.tmA, w.Aq, (uint64_t)p.R_max, (uint64_t)n, 128, 128));
-    MOE_TRY_MAP(make_tmap_u8(&g.tmB, w.W2q, (uint64_t)E * d, (uint64_t)n, 128, 128));
+    MOE_TRY_MAP(make_tmap_u8(&g.tmB, wt.W2q, (uint64_t)E * d, (uint64_t)n, 128, 128));
     g.sfa_src = w.SA;
-    g.sfb_src = w.SW2t;
+    g.sfb_src = wt.SW2t;
     g.num_n_tiles = d / 128;
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)d));
@@ -596,7 +601,90 @@ moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const v
   return MOE_OK;
 }
 
+// Shape, pointer and workspace checks shared by the MXFP8 forward entries.
+moe_status mx_forward_setup(const moe_dims* dims, const moe_opts* opts, const void* X, const moe_routing* rt,
+                            void* O, void* H, void* ws, size_t ws_bytes, Plan* p, MxFwdWs* w) {
+  moe_status s = make_plan(dims, opts, p);
+  if (s != MOE_OK) return s;
+  if (!mx_supported(*p)) return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {X, O, H};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!routing_ok(rt, *p, false)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < carve_fwd_mx(*p, nullptr, w)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  carve_fwd_mx(*p, ws, w);
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
+                             const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!W1 || !W2 || !aligned16(W1) || !aligned16(W2)) {
+    Plan p;
+    const moe_status s = make_plan(dims, opts, &p);
+    if (s != MOE_OK) return s;
+    return mx_supported(p) ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+  }
+  Plan p;
+  MxFwdWs w;
+  moe_status s = mx_forward_setup(dims, opts, X, rt, O, H, ws, ws_bytes, &p, &w);
+  if (s != MOE_OK) return s;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_TRY_CUDA(quantize_mx_weights(p, W1, W2, w.wt, st));
+  return forward_mx(p, X, w.wt, rt, O, H, w, status, sms, st);
+}
+
+moe_status moe_mx_quantize_weights(const moe_dims* dims, const moe_opts* opts, const void* W1, const void* W2,
+                                   void* wq, size_t wq_bytes, void* stream) {
+  Plan p;
+  moe_status s = make_plan(dims, opts, &p);
+  if (s != MOE_OK) return s;
+  if (!mx_supported(p)) return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {W1, W2, wq};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (wq_bytes < mx_weights_bytes(p)) return MOE_ERR_WORKSPACE;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms)) return MOE_ERR_CUDA;
+  Carve c{static_cast<char*>(wq)};
+  MxWeights wt;
+  carve_mx_weights(p, c, &wt);
+  MOE_TRY_CUDA(quantize_mx_weights(p, W1, W2, wt, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward_mxfp8_q(const moe_dims* dims, const moe_opts* opts, const void* X, const void* wq,
+                               const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream) {
+  if (!wq || !aligned16(wq)) {
+    Plan p;
+    const moe_status s = make_plan(dims, opts, &p);
+    if (s != MOE_OK) return s;
+    return mx_supported(p) ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+  }
+  Plan p;
+  MxFwdWs w;
+  moe_status s = mx_forward_setup(dims, opts, X, rt, O, H, ws, ws_bytes, &p, &w);
+  if (s != MOE_OK) return s;
+  int dev, sms;
+  int* status;
+  if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
+  Carve c{static_cast<char*>(const_cast<void*>(wq))};
+  MxWeights wt;
+  carve_mx_weights(p, c, &wt);
+  return forward_mx(p, X, wt, rt, O, H, w, status, sms, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"
+
+
 
 namespace {
 // dWr = X^T dz: the split-K tensor-core GEMM over the bf16 hi/lo split of dz

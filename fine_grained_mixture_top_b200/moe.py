@@ -41,7 +41,7 @@ class MoeRouting(ctypes.Structure):
 class MoeSizes(ctypes.Structure):
     _fields_ = [("P_max", c_int64), ("R_max", c_int64), ("route_ws", ctypes.c_size_t),
                 ("fwd_ws", ctypes.c_size_t), ("bwd_ws", ctypes.c_size_t), ("h_elems", c_int64),
-                ("fwd_mx_ws", ctypes.c_size_t)]
+                ("fwd_mx_ws", ctypes.c_size_t), ("mx_weights_bytes", ctypes.c_size_t)]
 
 
 class MoEError(RuntimeError):
@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.moe_forward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, P(MoeRouting), c_void_p,
                                   c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
         L.moe_forward_mxfp8.argtypes = L.moe_forward.argtypes
+        L.moe_mx_quantize_weights.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, ctypes.c_size_t,
+                                              c_void_p]
+        L.moe_forward_mxfp8_q.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, P(MoeRouting), c_void_p,
+                                          c_void_p, c_void_p, ctypes.c_size_t, c_void_p]
         L.moe_backward.argtypes = [P(MoeDims), P(MoeOpts), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    P(MoeRouting), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    ctypes.c_size_t, c_void_p]
@@ -108,7 +112,8 @@ def lib() -> ctypes.CDLL:
         for f in ("moe_query_sizes", "moe_route", "moe_token_round", "moe_forward", "moe_backward",
                   "moe_get_status", "moe_set_spin_limit", "moe_selftest_wait_timeout", "moe_backward_ev",
                   "moe_set_sm_budget", "moe_mx_quantize_rows", "moe_mx_quantize_cols", "moe_forward_mxfp8",
-                  "moe_route_given", "moe_ep_pack", "moe_ep_combine", "moe_router_backward"):
+                  "moe_route_given", "moe_ep_pack", "moe_ep_combine", "moe_router_backward",
+                  "moe_mx_quantize_weights", "moe_forward_mxfp8_q"):
             getattr(L, f).restype = c_int32
         _lib = L
     return _lib
@@ -240,6 +245,17 @@ def moe_forward_mxfp8(dims, opts, X, W1, W2, routing: Routing, O, H, ws, stream=
                                    ws.numel() * ws.element_size(), _stream(stream)), "moe_forward_mxfp8")
 
 
+def moe_mx_quantize_weights(dims, opts, W1, W2, wq, stream=None):
+    _check(lib().moe_mx_quantize_weights(ctypes.byref(dims), ctypes.byref(opts), _ptr(W1), _ptr(W2), _ptr(wq),
+                                         wq.numel() * wq.element_size(), _stream(stream)), "moe_mx_quantize_weights")
+
+
+def moe_forward_mxfp8_q(dims, opts, X, wq, routing: Routing, O, H, ws, stream=None):
+    _check(lib().moe_forward_mxfp8_q(ctypes.byref(dims), ctypes.byref(opts), _ptr(X), _ptr(wq),
+                                     ctypes.byref(routing.struct), _ptr(O), _ptr(H), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "moe_forward_mxfp8_q")
+
+
 def moe_backward(dims, opts, dO, X, Wr, W1, W2, routing: Routing, H, dX, dW1, dW2, dWr, ws, stream=None,
                  grad_events=None):
     """grad_events: None, or three torch.cuda.Event (or None) recorded once
@@ -362,6 +378,24 @@ class MoELayer:
             moe_forward_mxfp8(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd_mx, stream)
         else:
             moe_forward(self.dims, self.opts, X, W1, W2, self.routing, O, self.H, self.ws_fwd, stream)
+        return O
+
+    def quantize_weights_mxfp8(self, W1, W2, stream=None):
+        """MXFP8 copy of W1, W2 for forward_mxfp8_q (weights that stay fixed)."""
+        import torch
+        if self.sizes.mx_weights_bytes == 0:
+            raise MoEError(2, "moe_mx_quantize_weights (needs n % 128 == 0)")
+        wq = torch.empty(self.sizes.mx_weights_bytes, dtype=torch.uint8, device=self.device)
+        moe_mx_quantize_weights(self.dims, self.opts, W1, W2, wq, stream)
+        return wq
+
+    def forward_mxfp8_q(self, X, wq, stream=None, O=None):
+        """The MXFP8 forward on weights quantized once by quantize_weights_mxfp8."""
+        import torch
+        O = self.O if O is None else O
+        if self.ws_fwd_mx is None:
+            self.ws_fwd_mx = torch.empty(self.sizes.fwd_mx_ws, dtype=torch.uint8, device=self.device)
+        moe_forward_mxfp8_q(self.dims, self.opts, X, wq, self.routing, O, self.H, self.ws_fwd_mx, stream)
         return O
 
     def backward(self, dO, X, Wr, W1, W2, stream=None, grad_events=None):

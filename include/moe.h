@@ -114,7 +114,8 @@ typedef struct {
   size_t fwd_ws;        /* bytes of ws for moe_forward */
   size_t bwd_ws;        /* bytes of ws for moe_backward */
   int64_t h_elems;      /* elements of the saved activation H = R_max * 2n (bf16) */
-  size_t fwd_mx_ws;     /* bytes of ws for moe_forward_mxfp8; 0 where that shape is unsupported */
+  size_t fwd_mx_ws;     /* bytes of ws for moe_forward_mxfp8(_q); 0 where that shape is unsupported */
+  size_t mx_weights_bytes; /* bytes of the MXFP8 expert weights of moe_mx_quantize_weights; 0 if unsupported */
 } moe_sizes;
 
 /* Capacities and workspace sizes for a shape.  Host only; no GPU work. */
@@ -186,6 +187,21 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
 moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
                              const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
                              void* stream);
+
+/*
+ * The MXFP8 forward in two parts, for weights that stay fixed over many
+ * calls (inference): moe_mx_quantize_weights writes W1 and W2 as MXFP8 (E4M3
+ * codes, K-major, and their E8M0 scales in the layout the block-scaled MMA
+ * reads) into wq, moe_sizes.mx_weights_bytes bytes of caller memory;
+ * moe_forward_mxfp8_q is moe_forward_mxfp8 on those quantized weights (X
+ * is still quantized per call).  The results are those of moe_forward_mxfp8
+ * on the same W1, W2, bit for bit.  Same shape rule (n % 128 == 0) and
+ * errors; ws of moe_sizes.fwd_mx_ws bytes.
+ */
+moe_status moe_mx_quantize_weights(const moe_dims* dims, const moe_opts* opts, const void* W1, const void* W2,
+                                   void* wq, size_t wq_bytes, void* stream);
+moe_status moe_forward_mxfp8_q(const moe_dims* dims, const moe_opts* opts, const void* X, const void* wq,
+                               const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Backward given dO[T,d] bf16 ([P2] implementation and algorithm paragraphs;

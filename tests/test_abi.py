@@ -96,6 +96,12 @@ def test_invalid_options_and_null_arguments(moe):
     assert L.moe_forward_mxfp8(ctypes.byref(dims128), ctypes.byref(moe.opts_of()), None, None, None,
                                ctypes.byref(rt), None, None, None, 0, None) == 1
     assert moe.query_sizes(dims128, moe.opts_of()).fwd_mx_ws > 0
+    assert moe.query_sizes(dims128, moe.opts_of()).mx_weights_bytes >= 3 * 16 * 128 * 128
+    assert L.moe_mx_quantize_weights(ctypes.byref(dims), ctypes.byref(moe.opts_of()), None, None, None, 0, None) == 2
+    assert L.moe_mx_quantize_weights(ctypes.byref(dims128), ctypes.byref(moe.opts_of()), None, None, None, 0,
+                                     None) == 1
+    assert L.moe_forward_mxfp8_q(ctypes.byref(dims128), ctypes.byref(moe.opts_of()), None, None, ctypes.byref(rt),
+                                 None, None, None, 0, None) == 1
     assert moe.query_sizes(dims, moe.opts_of()).fwd_mx_ws == 0      # n = 64: no MXFP8 forward
     # expert-parallel and given-routing entry points
     assert L.moe_route_given(ctypes.byref(dims), ctypes.byref(moe.opts_of()), ctypes.byref(rt), None, 0, None) == 1

@@ -184,3 +184,23 @@ def test_mxfp8_forward_after_token_rounding(mode):
     err = P.normwise(P.f64(layer.O), fq["O"])
     print("mx_tr", mode, f"O {err:.2e}")
     assert err <= P.TOL_BF16
+
+
+@pytest.mark.gpu
+def test_prequantized_weights_give_the_same_forward():
+    """Weights quantized once (moe_mx_quantize_weights) then
+    moe_forward_mxfp8_q: bit for bit the forward that quantizes them itself."""
+    from fine_grained_mixture_top_b200 import moe
+    cfg = MX_SHAPES[1]
+    inp = make_inputs(cfg, "cuda", need_grad_inputs=False)
+    layer = _mx_layer(cfg, inp)
+    O1, H1 = layer.O.clone(), layer.H.clone()
+    wq = layer.quantize_weights_mxfp8(inp["W1"], inp["W2"])
+    layer.O.zero_()
+    layer.H.zero_()
+    layer.forward_mxfp8_q(inp["X"], wq)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    assert torch.equal(layer.O.view(torch.int16), O1.view(torch.int16))
+    R = int(layer.routing["offsets"][cfg.E].item())
+    assert torch.equal(layer.H[:R].view(torch.int16), H1[:R].view(torch.int16))
