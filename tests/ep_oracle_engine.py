@@ -13,14 +13,19 @@ from oracle import moe_oracle as orc
 
 
 class OracleEngine:
-    def __init__(self, E, K, G):
+    def __init__(self, E, K, G, round_mode=0, seed=0, tile=128):
         self.E, self.K, self.G = E, K, G
         self.E_loc = E // G
+        self.round_mode, self.seed, self.tile = round_mode, seed, tile
 
     # ---- source side (this rank's tokens, all E experts)
     def route(self, X, Wr, bias):
         b = None if bias is None else bias.numpy()
         self.rt = orc.route(X.numpy(), Wr.numpy(), b, self.K)
+        if self.round_mode:  # this rank's batch rounded on its own
+            tr = orc.token_round(self.rt["probs"], self.rt["tok_ptr"], self.rt["pair_expert"], self.round_mode,
+                                 self.seed, self.tile)
+            self.rt.update({k: tr[k] for k in ("tok_ptr", "pair_expert", "pair_gate")})
         self.perm = orc.permute(self.rt["tok_ptr"], self.rt["pair_expert"], self.E)
 
     def counts(self):

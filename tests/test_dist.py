@@ -107,7 +107,7 @@ def test_rank_failing_before_exchange_is_reported_not_hung():
 # all-to-all.  The plan and the exchanges are the product's
 # (fine_grained_mixture_top_b200.ep); the arithmetic is the oracle's.
 # ----------------------------------------------------------------------------
-def _ep_worker(rank, world, port, K, T, E, out_q):
+def _ep_worker(rank, world, port, K, T, E, out_q, round_mode=0):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -117,7 +117,8 @@ def _ep_worker(rank, world, port, K, T, E, out_q):
     sl = slice(rank * T, (rank + 1) * T)
     E_loc = E // world
     es = slice(rank * E_loc, (rank + 1) * E_loc)
-    ep = ExpertParallelMoE(T, X.shape[1], E, W2.shape[1], K, OracleEngine(E, K, world))
+    ep = ExpertParallelMoE(T, X.shape[1], E, W2.shape[1], K,
+                           OracleEngine(E, K, world, round_mode=round_mode, seed=11, tile=8))
     t = torch.from_numpy
     O = ep.forward(t(X[sl].copy()), t(Wr), t(b), t(W1[es].copy()), t(W2[es].copy()))
     dX, dW1, dW2, dWr = ep.backward(t(dO[sl].copy()), t(X[sl].copy()), t(Wr), t(W1[es].copy()), t(W2[es].copy()))
@@ -163,3 +164,44 @@ def test_exchange_plan_orders_rows_by_source_then_expert():
     ss, rs, le = exchange_plan(send, recv)
     assert ss == [3, 3, 0] and rs == [3, 4, 1]
     np.testing.assert_array_equal(le, [0, 0, 1, 1, 1, 1, 1, 0])
+
+
+def test_expert_parallel_with_token_rounding():
+    """Each rank rounds its own batch's expert counts (tile 8 here) before the
+    exchange; the layer equals the single-process oracle run on the
+    concatenation of the ranks' rounded routings."""
+    world, E, K, T = 2, 6, 2, 40
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, K, T, E, q, 2)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r[0], r[1:]) for r in (q.get(timeout=180) for _ in range(world)))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W1, W2, Wr, b, dO = _layer(seed=5, T=T * world, E=E)
+    ptrs, exps, gates = [np.zeros(1, np.int64)], [], []
+    for r in range(world):
+        sl = slice(r * T, (r + 1) * T)
+        rt = orc.route(X[sl], Wr, b, K)
+        tr = orc.token_round(rt["probs"], rt["tok_ptr"], rt["pair_expert"], 2, 11, 8)
+        assert np.all(tr["counts"] % 8 == 0)
+        ptrs.append(tr["tok_ptr"][1:] + ptrs[-1][-1])
+        exps.append(tr["pair_expert"])
+        gates.append(tr["pair_gate"])
+    routing = {"tok_ptr": np.concatenate(ptrs), "pair_expert": np.concatenate(exps),
+               "pair_gate": np.concatenate(gates)}
+    fw = orc.forward(X, Wr, b, W1, W2, K, routing=routing)
+    bw = orc.backward(fw, dO, X, Wr, W1, W2)
+    E_loc = E // world
+    for r in range(world):
+        O, dX, dW1, dW2, dWr = got[r]
+        sl = slice(r * T, (r + 1) * T)
+        es = slice(r * E_loc, (r + 1) * E_loc)
+        np.testing.assert_allclose(O, fw["O"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dX, bw["dX"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dW1, bw["dW1"][es], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dW2, bw["dW2"][es], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dWr, bw["dWr"], rtol=1e-10, atol=1e-12)
