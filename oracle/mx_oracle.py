@@ -36,8 +36,8 @@ notes):
 Parity status: pinned by tests/test_oracle_mx.py (the E4M3 table against the
 format's closed form, round trips of every code, ties to even, the scale
 rule against brute force, the element error bound, power-of-two
-equivariance, exactness on representable inputs, and the E=1, K=1 dense
-case against plain numpy matmuls).
+equivariance, exactness on representable inputs, the E=1, K=1 dense case
+against plain numpy matmuls, and several experts against per-token loops).
 """
 from __future__ import annotations
 

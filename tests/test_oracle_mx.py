@@ -146,3 +146,39 @@ def test_quantized_forward_stays_near_the_exact_forward():
     rel = np.abs(fq["O"] - fw["O"]).max() / np.abs(fw["O"]).max()
     # three 3-bit-mantissa roundings on the path to O: a few percent, not more
     assert 1e-4 < rel < 0.1, rel
+
+
+def test_quantized_forward_equals_per_token_loops():
+    """Several experts, K = 2, skewed router: every token's output written out
+    as a loop over its experts (quantize X_t and the expert's weight columns,
+    SwiGLU of the bf16-rounded H, quantize A, multiply, gate), with numpy
+    alone for the arithmetic and the format's codec for the rounding."""
+    rng = np.random.default_rng(8)
+    T, d, E, n, K = 24, 64, 5, 32, 2
+    X = rng.standard_normal((T, d))
+    W1 = rng.standard_normal((E, d, 2 * n)) * 0.1
+    W2 = rng.standard_normal((E, n, d)) * 0.1
+    Wr = rng.standard_normal((d, E))
+    b = rng.standard_normal(E)
+    fq = mx.forward_mxfp8(X, Wr, b, W1, W2, K)
+
+    def q(v):   # blocks of 32 along the last axis
+        B = v.reshape(v.shape[:-1] + (-1, 32))
+        am = np.abs(B).max(-1)
+        f, Ex = np.frexp(am)
+        e = np.where(am > 0, (Ex - 1) - 8 + (2 * f > 1.75), -127)
+        S = np.exp2(e.astype(float))[..., None]
+        return (mx.e4m3_decode(mx.e4m3_encode(B / S)) * S).reshape(v.shape)
+
+    z = X @ Wr + b
+    O = np.zeros((T, d))
+    for t in range(T):
+        top = sorted(range(E), key=lambda e: (-z[t, e], e))[:K]
+        g = np.exp(z[t, top] - z[t, top].max())
+        g /= g.sum()
+        for s, e in zip(g, top):
+            h = q(X[t]) @ q(W1[e].T).T
+            hb = _bf16_torch(h)
+            a = hb[:n] / (1 + np.exp(-hb[:n])) * hb[n:]
+            O[t] += s * (q(a) @ q(W2[e].T).T)
+    np.testing.assert_allclose(fq["O"], O, rtol=1e-12, atol=1e-12)
