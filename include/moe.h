@@ -175,7 +175,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
 /*
  * Forward with MXFP8 GEMM operands (MXFP8 precision is named as future work
  * of the method, page "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE",
- * closing paragraph; format: OCP Microscaling, as for moe_mx_quantize_rows).
+ * closing paragraph; format and scale rule as for moe_mx_quantize_rows).
  * X is quantized along d per row, W1 along d and W2 along n per output
  * column, A = SwiGLU(H) along n per row; the GEMMs multiply E4M3 codes with
  * their E8M0 block scales on the tensor cores (kind::mxf8f6f4) and
@@ -285,9 +285,14 @@ moe_status moe_set_sm_budget(int32_t sms);
 /*
  * MXFP8 quantization (the pages list MXFP8 precision as future work of the
  * method, page "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE", closing
- * paragraph; the format is the OCP Microscaling definition): E4M3 codes with
- * one E8M0 scale per 32 consecutive elements along K, the scale being the
- * smallest power of two at which no element of the block saturates.
+ * paragraph; the element and scale encodings are those of the OCP
+ * Microscaling formats): E4M3 codes with one E8M0 scale per 32 consecutive
+ * elements along K.  The scale is the smallest power of two at which no
+ * element of the block saturates.  This departs from the OCP MX v1.0 scale
+ * rule (section 6.3: shared exponent floor(log2 amax) - 8, elements above 448
+ * clamped), which gives a scale half as large, and clamps the block maximum,
+ * whenever the block maximum's significand exceeds 1.75; here no element is
+ * ever clamped.
  *
  * moe_mx_quantize_rows: in[rows, K] bf16 -> codes[rows, K] u8 and
  *   scales[rows, K/32] u8, quantized along each row.

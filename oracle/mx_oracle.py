@@ -14,11 +14,21 @@ E8M0 (an 8-bit biased exponent, bias 127), and each element is an FP8 E4M3
 value (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; subnormals; no
 infinities; the one NaN pattern S.1111.111; largest finite 448).
 
-Readings where the definition leaves a choice (each listed in the design
-notes):
+Readings (each listed in the design notes):
   M1 Shared exponent: the smallest e with amax <= 448 * 2^e, so no element
      of a block saturates.  With amax = f * 2^E, 1 <= f < 2, that is
      e = E - 8, plus 1 when f > 1.75.  An all-zero block gets scale code 0.
+     This DEPARTS from the OCP MX v1.0 specification (section 6.3), whose
+     shared exponent is floor(log2 amax) - 8 (8 = the exponent of E4M3's
+     largest normal, 448 = 1.75 * 2^8) with the elements that then exceed 448
+     clamped to 448.  The two rules agree when f <= 1.75 and differ by one
+     when f > 1.75 (about one block in eight for Gaussian data): OCP's rule
+     clamps that block's largest element(s), by up to 12.5 %; M1 instead
+     doubles the block's scale, so no element is clamped and every element
+     keeps the half-ulp error bound, at the cost of one bit of resolution
+     for the block's smallest elements.  `scale_exponent_ocp` states OCP's
+     rule for comparison; the tests pin both and the cases where they
+     differ.
   M2 Elements: v / 2^e rounded to the nearest E4M3 value, ties to the even
      code; magnitudes above 448 (none, given M1) saturate to 448.  A value
      that rounds to zero keeps its sign (code 0x80 for negative).
@@ -96,6 +106,16 @@ def scale_exponent(amax):
     f = 2.0 * f                    # 1 <= f < 2
     E = E.astype(np.int64) - 1
     e = E - 8 + (f > 1.75)
+    return np.where(amax > 0, e, -127)
+
+
+def scale_exponent_ocp(amax):
+    """Shared exponent of the OCP MX v1.0 rule (section 6.3), for comparison
+    with M1: floor(log2 amax) - 8 for E4M3; -127 for 0.  Not used by the
+    quantized forward."""
+    amax = np.asarray(amax, F64)
+    _, E = np.frexp(amax)          # amax = f * 2^E with 0.5 <= f < 1
+    e = E.astype(np.int64) - 1 - 8
     return np.where(amax > 0, e, -127)
 
 

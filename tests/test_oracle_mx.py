@@ -1,6 +1,10 @@
 """Pins of the MXFP8 oracle against the format's definition (OCP Microscaling
 formats: E4M3 elements, E8M0 block scales of 32) and plain mathematics --
-nothing here re-derives a value through the function under test."""
+nothing here re-derives a value through the function under test.
+
+The scale rule is reading M1 (the smallest non-saturating power of two), a
+stated departure from OCP MX v1.0 section 6.3; both rules are pinned below,
+each by brute force, together with the blocks on which they differ."""
 import numpy as np
 
 from oracle import moe_oracle as mo
@@ -42,6 +46,7 @@ def test_rounding_is_to_nearest_with_ties_to_even():
 
 
 def test_scale_rule_is_the_smallest_non_saturating_exponent():
+    # reading M1, the rule the quantizers and the oracle use
     rng = np.random.default_rng(1)
     amax = np.concatenate([rng.lognormal(0, 6, 2000), [448.0, 449.0, 1.0, 1.75, 1.7500001, 2.0 ** -120]])
     e = mx.scale_exponent(amax)
@@ -49,6 +54,45 @@ def test_scale_rule_is_the_smallest_non_saturating_exponent():
     assert np.all(amax <= 448.0 * np.exp2(e.astype(float)))
     assert np.all(amax > 448.0 * np.exp2(e.astype(float) - 1))
     assert mx.scale_exponent(0.0) == -127 and mx.scale_code(0.0) == 0
+
+
+def _floor_log2_brute(a):
+    """Largest integer k with 2^k <= a, by walking k (no frexp, no log)."""
+    k = 0
+    while 2.0 ** k > a:
+        k -= 1
+    while 2.0 ** (k + 1) <= a:
+        k += 1
+    return k
+
+
+def test_ocp_rule_is_floor_log2_minus_8():
+    # OCP MX v1.0 section 6.3: shared exponent = floor(log2 amax) - emax_elem,
+    # emax_elem = 8 for E4M3 (448 = 1.75 * 2^8)
+    rng = np.random.default_rng(1)
+    amax = np.concatenate([rng.lognormal(0, 6, 2000), [448.0, 449.0, 1.0, 1.75, 1.7500001, 2.0 ** -120]])
+    brute = np.array([_floor_log2_brute(a) - 8 for a in amax])
+    np.testing.assert_array_equal(mx.scale_exponent_ocp(amax), brute)
+    assert mx.scale_exponent_ocp(0.0) == -127
+
+
+def test_m1_departs_from_ocp_exactly_where_ocp_clamps():
+    rng = np.random.default_rng(4)
+    amax = np.concatenate([rng.lognormal(0, 6, 2000), [1.75, 1.7500001, 1.999, 448.0, 449.0, 511.0]])
+    f = amax / np.exp2([_floor_log2_brute(a) for a in amax])      # significand in [1, 2)
+    e_m1 = mx.scale_exponent(amax)
+    e_ocp = mx.scale_exponent_ocp(amax)
+    np.testing.assert_array_equal(e_m1 - e_ocp, (f > 1.75).astype(int))
+    # under OCP's exponent the block maximum lands above 448 exactly on those
+    # blocks, and E4M3 encoding clamps it to 448; under M1 it never does
+    over = amax / np.exp2(e_ocp.astype(float)) > 448.0
+    np.testing.assert_array_equal(over, f > 1.75)
+    assert np.all(mx.e4m3_decode(mx.e4m3_encode(amax[over] / np.exp2(e_ocp[over].astype(float)))) == 448.0)
+    assert np.all(amax / np.exp2(e_m1.astype(float)) <= 448.0)
+    # about one block in eight for Gaussian blocks of 32
+    g = np.abs(rng.standard_normal((20000, 32))).max(axis=1)
+    frac = np.mean(mx.scale_exponent(g) != mx.scale_exponent_ocp(g))
+    assert 0.05 < frac < 0.25
 
 
 def test_block_quantization_error_bound():
