@@ -4,11 +4,12 @@
 One step = the whole path on one batch: routing (router logits, softmax, top-K,
 permutation), forward (up-proj + SwiGLU, down-proj, aggregation) and backward
 (dH + dS, dW2, dX~, dW1, router backward, dX aggregation), all through the
-library's C ABI.  Workload: the fine-grained 7B-class layer, T=16384 tokens,
-d=1536, E=128, n=256, top-8, skewed router (bias ~ N(0, 0.5)); synthetic seeded
-inputs (workloads package).  Multi-GPU: one process per GPU (torchrun), each
-with its own batch (weak scaling); the weight gradients are all-reduced over
-NCCL as the data-parallel exchange step.
+library's C ABI.  Default workload: the DeepSeek-V3-shaped layer, T=8192
+tokens, d=7168, E=256, n=2048, top-8, Zipf(1.1) expert popularity -- the
+largest of the workloads that fits one GPU; --config NAME runs another.
+Synthetic seeded inputs (workloads package).  Multi-GPU: one process per GPU
+(torchrun), each with its own batch (weak scaling); the weight gradients are
+all-reduced over NCCL as the data-parallel exchange step.
 
 Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle on
 a bounded sample of the same workload instead.
@@ -30,8 +31,25 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer fwd+bwd TFLOP/s (bf16) and % of B200 tensor peak; tokens/sec"
-WORKLOAD = ("fine-grained 7B-class MoE layer fwd+bwd: T=16384, d=1536, E=128, n=256, top-8, SwiGLU, "
-            "skewed router (bias ~N(0,0.5))")
+WORKLOADS = {
+    "dsv3": ("DeepSeek-V3-shaped MoE layer fwd+bwd: T=8192, d=7168, E=256, n=2048, top-8, SwiGLU, "
+             "Zipf(1.1) expert popularity (router bias -1.1 ln rank)"),
+    "7b": ("fine-grained 7B-class MoE layer fwd+bwd: T=16384, d=1536, E=128, n=256, top-8, SwiGLU, "
+           "skewed router (bias ~N(0,0.5))"),
+    "qwen3": ("Qwen3-MoE-shaped layer fwd+bwd: T=32768, d=2048, E=128, n=768, top-8, SwiGLU, balanced router"),
+    "olmoe": ("OLMoE-shaped layer fwd+bwd: T=32768, d=2048, E=64, n=1024, top-8, SwiGLU, balanced router"),
+    "tiny": ("tiny MoE layer fwd+bwd: T=512, d=128, E=16, n=64, top-2, SwiGLU"),
+}
+# a timed region at least this long runs under the power cap: its roofline
+# uses the sustained tensor peak; a shorter one uses the burst peak
+SUSTAINED_WINDOW_S = 2.0
+
+
+def workload_text(name, cfg):
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    return (f"{name} MoE layer fwd+bwd: T={cfg.T}, d={cfg.d}, E={cfg.E}, n={cfg.n}, top-{cfg.K}, SwiGLU, "
+            f"router bias {cfg.bias}, rounding mode {cfg.round_mode}")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -41,11 +59,14 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="7b")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
+    ap.add_argument("--config", default="dsv3",
+                    help="workload (default: the DeepSeek-V3-shaped layer, the largest that fits one GPU)")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=None,
+                    help="tokens of the CPU oracle's sample (default: about 10 s of fp64 work)")
     ap.add_argument("--cpu-min-seconds", type=float, default=10.0,
                     help="repeat the oracle step on the sample until this much CPU time has run (at most 4 times)")
-    ap.add_argument("--ref-sample-tokens", type=int, default=1024)
+    ap.add_argument("--ref-sample-tokens", type=int, default=None,
+                    help="tokens per reference-arm step (default: about 1 s of fp64 work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--parallel", default="dp", choices=["dp", "ep"],
@@ -172,22 +193,82 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
-def oracle_step_seconds(cfg, inp_cpu, tokens):
-    """Time the fp64 oracle (as it stands) on the first `tokens` tokens of the
-    batch: route, forward, backward.  Returns (seconds, threads)."""
+# fp64 bytes per expert the oracle holds: W1[e], W2[e] and their gradients
+def _expert_f64_bytes(cfg):
+    return 8 * 6 * cfg.d * cfg.n
+
+
+def oracle_sample_plan(cfg, X, Wr, bias, tokens, budget_bytes=8 << 30):
+    """The bounded sample the CPU oracle runs: the first `tokens` tokens, and
+    the experts their pairs go to, most-loaded first, as many as fit
+    `budget_bytes` of fp64 weights and weight gradients (all of them on the
+    smaller layers).  Returns the expert ids."""
     import numpy as np
     from oracle import moe_oracle as orc
-    X = inp_cpu["X"][:tokens].double().numpy()
-    dO = inp_cpu["dO"][:tokens].double().numpy()
-    W1 = inp_cpu["W1np"]
-    W2 = inp_cpu["W2np"]
-    Wr = inp_cpu["Wr"].double().numpy()
-    b = None if inp_cpu["bias"] is None else inp_cpu["bias"].double().numpy()
+    rt = orc.route(X[:tokens].double().numpy(), Wr.double().numpy(),
+                   None if bias is None else bias.double().numpy(), cfg.K)
+    counts = np.bincount(rt["pair_expert"], minlength=cfg.E)
+    cap = max(1, budget_bytes // _expert_f64_bytes(cfg))
+    used = [int(e) for e in np.argsort(-counts, kind="stable") if counts[e] > 0]
+    return sorted(used[:cap])
+
+
+def oracle_sample_step(cfg, smp):
+    """One step of the fp64 oracle (as it stands) on the sample `smp`: route
+    the sample's tokens over all E experts, keep the pairs that go to the
+    sample's experts (all pairs when every expert is in it), then forward and
+    backward with the router path.  Returns (seconds, pairs, threads)."""
+    import numpy as np
+    from oracle import moe_oracle as orc
+    X, dO, Wr, b, W1, W2, S = (smp[k] for k in ("X", "dO", "Wr", "bias", "W1", "W2", "experts"))
     t0 = time.perf_counter()
-    fw = orc.forward(X, Wr, b, W1, W2, cfg.K)
-    orc.backward(fw, dO, X, Wr, W1, W2)
+    rt = orc.route(X, Wr, b, cfg.K)
+    if len(S) == cfg.E:
+        sub, Wr_s = rt, Wr
+    else:
+        remap = -np.ones(cfg.E, np.int64)
+        remap[S] = np.arange(len(S))
+        keep = remap[rt["pair_expert"]] >= 0
+        pair_tok = np.repeat(np.arange(X.shape[0]), np.diff(rt["tok_ptr"]))
+        tok_ptr = np.concatenate([[0], np.cumsum(np.bincount(pair_tok[keep], minlength=X.shape[0]))])
+        sub = {"z": rt["z"][:, S], "probs": rt["probs"][:, S], "topk_idx": rt["topk_idx"], "tok_ptr": tok_ptr,
+               "pair_expert": remap[rt["pair_expert"][keep]], "pair_gate": rt["pair_gate"][keep]}
+        Wr_s = Wr[:, S]
+    fw = orc.forward(X, Wr_s, None, W1, W2, cfg.K, routing=sub)
+    orc.backward(fw, dO, X, Wr_s, W1, W2)
     dt = time.perf_counter() - t0
-    return dt, blas_threads()
+    return dt, int(sub["tok_ptr"][-1]), blas_threads()
+
+
+def oracle_sample(cfg, inp, tokens, experts):
+    """Host fp64 copies of the sample's tensors (`inp` may live on any device;
+    W1/W2 either full or already restricted to `experts`)."""
+    def f64(t):
+        return t.detach().to("cpu").double().numpy()
+    full = inp["W1"].shape[0] == cfg.E
+    idx = experts if full else list(range(len(experts)))
+    import torch
+    sel = torch.as_tensor(idx, device=inp["W1"].device)
+    return {"X": f64(inp["X"][:tokens]), "dO": f64(inp["dO"][:tokens]), "Wr": f64(inp["Wr"]),
+            "bias": None if inp["bias"] is None else f64(inp["bias"]),
+            "W1": f64(inp["W1"].index_select(0, sel)), "W2": f64(inp["W2"].index_select(0, sel)),
+            "experts": list(experts)}
+
+
+def default_sample_tokens(cfg, seconds):
+    """Tokens whose fp64 forward + backward (18 K d n flops each) take about
+    `seconds` at 0.15 TFLOP/s, the oracle's rate on a 16-thread host; at
+    least 16, a multiple of 16."""
+    per_tok = 18.0 * cfg.K * cfg.d * cfg.n
+    return int(max(16, min(cfg.T, seconds * 0.15e12 / per_tok)) // 16 * 16)
+
+
+def sample_text(cfg, tokens, experts, pairs):
+    if len(experts) == cfg.E:
+        return f"first {tokens} of {cfg.T} tokens of the batch with all {cfg.E} experts ({pairs} routed pairs)"
+    return (f"first {tokens} of {cfg.T} tokens of the batch, routed over all {cfg.E} experts; the {pairs} "
+            f"pairs that go to the {len(experts)} experts most loaded by them (the fp64 weights of all "
+            f"{cfg.E} would not fit the host), same per-pair work")
 
 
 def blas_threads():
@@ -199,40 +280,36 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_inputs(cfg):
-    from workloads import make_inputs
-    inp = make_inputs(cfg, "cpu")
-    inp["W1np"] = inp["W1"].double().numpy()
-    inp["W2np"] = inp["W2"].double().numpy()
-    return inp
-
-
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from workloads import CONFIGS
+    from workloads import CONFIGS, make_inputs
     cfg = CONFIGS[args.config]
-    inp = cpu_inputs(cfg)
-    tokens = min(args.ref_sample_tokens, cfg.T)
+    tokens = min(args.ref_sample_tokens or default_sample_tokens(cfg, 1.0), cfg.T)
+    base = make_inputs(cfg, "cpu", experts=[])
+    experts = oracle_sample_plan(cfg, base["X"], base["Wr"], base["bias"], tokens)
+    inp = make_inputs(cfg, "cpu", experts=experts)
+    smp = oracle_sample(cfg, inp, tokens, experts)
+    pairs = 0
     for _ in range(args.warmup):
-        oracle_step_seconds(cfg, inp, tokens)
+        oracle_sample_step(cfg, smp)
     times = []
     threads = 1
     for _ in range(args.steps):
-        dt, threads = oracle_step_seconds(cfg, inp, tokens)
+        dt, pairs, threads = oracle_sample_step(cfg, smp)
         times.append(dt)
     tot = sum(times)
-    flops = 18 * tokens * cfg.K * cfg.d * cfg.n
+    flops = 6 * 3 * pairs * cfg.d * cfg.n
     value = flops * args.steps / tot / 1e12
-    sample = f"first {tokens} of {cfg.T} tokens per step (full weights), fp64 numpy oracle"
+    sample = sample_text(cfg, tokens, experts, pairs) + " per step, fp64 numpy oracle"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n, "K": cfg.K,
-                   "parallelism": "single host process"},
-        "tokens_per_s": tokens * args.steps / tot,
+        "config": {"workload": workload_text(args.config, cfg), "T": cfg.T, "d": cfg.d, "E": cfg.E, "n": cfg.n,
+                   "K": cfg.K, "parallelism": "single host process"},
+        "tokens_per_s": pairs / cfg.K * args.steps / tot,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -273,11 +350,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
     cfg = CONFIGS[args.config]
-    if args.config != "7b":
-        workload = (f"{args.config} MoE layer fwd+bwd: T={cfg.T}, d={cfg.d}, E={cfg.E}, n={cfg.n}, "
-                    f"top-{cfg.K}, SwiGLU, router bias {cfg.bias}, rounding mode {cfg.round_mode}")
-    else:
-        workload = WORKLOAD
+    workload = workload_text(args.config, cfg)
     inp = make_inputs(cfg, dev, rank=rank)
     layer = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=cfg.round_mode, router_grad=1,
                          seed=cfg.seed, device=dev)
@@ -427,19 +500,28 @@ def main():
     avg_dom = sum(dom_times) / len(dom_times)
     fl, by = work.get(dom, (0, 0))
     intensity = fl / max(by, 1)
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    # The tensor peak that applies: the burst figure for a timed region
+    # shorter than SUSTAINED_WINDOW_S (the clocks have not settled under the
+    # power cap yet), the sustained one for a longer region.
+    window_s = ms_max * 1e-3
+    sustained = window_s >= SUSTAINED_WINDOW_S
+    tensor_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if intensity >= ridge:
         achieved = fl / (avg_dom * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tensor_peak, "unit": "TFLOP/s"}
+        roof["frac"] = round(achieved / tensor_peak, 4)
+        roof["frac_of_burst"] = round(achieved / peaks["bf16_tflops"], 4)
+        roof["frac_of_sustained"] = round(achieved / peaks["bf16_tflops_sustained"], 4)
     else:
         achieved = by / (avg_dom * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+        roof["frac"] = round(achieved / peaks["hbm_gbs"], 4)
     roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['bound'] == 'tensor' else 'copy bandwidth'})"
+    roof["peak_source"] = (f"{peak_src} " + (("sustained bf16" if sustained else "burst bf16") +
+                                             f" (timed region {window_s:.2f} s)"
+                                             if roof["bound"] == "tensor" else "copy bandwidth"))
     roof["traffic"] = measured_traffic(dom, args.config)
-    tensor_peak = peaks["bf16_tflops_sustained"]
 
     # ---- end-to-end through the public API with host buffers: every step
     # copies its X and dO from pinned host memory and its O back to pinned host
@@ -492,20 +574,24 @@ def main():
                "d2h_bytes_per_step": int(Oh.numel() * 2), "ms_per_step": round(e_ms_step, 4),
                "api": "HostFedRunner.step (pinned host X, dO in; O out)"}
 
-    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 only
+    # ---- CPU baseline: the oracle on a bounded sample of the same batch
+    # (the device's own input bytes), rank 0 at N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        inp_cpu = cpu_inputs(cfg)
-        tokens = min(args.cpu_sample_tokens, cfg.T)
-        dt, reps = 0.0, 0
+        tokens = min(args.cpu_sample_tokens or default_sample_tokens(cfg, args.cpu_min_seconds), cfg.T)
+        experts = oracle_sample_plan(cfg, X.cpu(), Wr.cpu(), None if b is None else b.cpu(), tokens)
+        smp = oracle_sample(cfg, inp, tokens, experts)
+        dt, reps, fl = 0.0, 0, 0
         while reps < 4 and (reps == 0 or dt < args.cpu_min_seconds):
-            step_s, threads = oracle_step_seconds(cfg, inp_cpu, tokens)
+            step_s, pairs, threads = oracle_sample_step(cfg, smp)
             dt += step_s
+            fl += 18 * pairs * cfg.d * cfg.n
             reps += 1
-        cpu = {"value": round(reps * 18 * tokens * cfg.K * cfg.d * cfg.n / dt / 1e12, 6), "unit": "TFLOP/s",
+        del smp
+        cpu = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s",
                "cores": threads, "kind": "oracle", "seconds": round(dt, 2),
-               "sample": f"first {tokens} of {cfg.T} tokens of the same batch and full weights, {reps} x "
-                         "route+forward+backward of the fp64 numpy oracle"}
+               "sample": sample_text(cfg, tokens, experts, pairs) + f", {reps} x route+forward+backward of the "
+                         "fp64 numpy oracle"}
 
     if world > 1:
         dist.barrier()

@@ -1,6 +1,10 @@
 // Instantiations and launcher of the tcgen05 grouped GEMM (see gemm.cuh).
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "gemm.cuh"
 #include "moe_internal.h"
 
@@ -12,16 +16,28 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
   constexpr int smem = GemmShape<KIND, BN, EPI * EC::kBufs>::kSmemBytes;
   constexpr int threads = EC::kThreads;
   auto fn = moe_gemm_kernel<KIND, BN, EPI>;
-  static int configured_dev = -1;  // per-process; the library serves one device at a time
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured_dev = dev;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
+  if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
   return launch_pdl(fn, dim3(grid), dim3(threads), (size_t)smem, stream, p);
+}
+
+// The dynamic shared-memory limit is a per-device property of a function: it
+// is set once for each (function, device), under a lock, so that host threads
+// driving different devices (or the same one) all see it set before they
+// launch.
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({fn, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done.insert({fn, dev});
+  return cudaSuccess;
 }
 
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s) {

@@ -37,6 +37,10 @@ inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_
 constexpr int kTile = 128;        // rows per expert tile (segments are padded to it)
 constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation
 
+// Sets `fn`'s dynamic shared-memory limit on the current device, once per
+// (function, device); thread-safe.
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
+
 // epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
 

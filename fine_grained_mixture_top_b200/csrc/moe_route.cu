@@ -608,13 +608,8 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
     // stage the expert's p row and candidate mask when they fit in shared memory
     const size_t staged = ((size_t)r.T + (size_t)W) * sizeof(uint32_t);
     if (staged <= kTrStageMax) {
-      static bool configured = false;  // one device per process, as for the GEMM kernels
-      if (!configured) {
-        err = cudaFuncSetAttribute(tr_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kTrStageMax);
-        if (err != cudaSuccess) return err;
-        configured = true;
-      }
+      err = set_max_dynamic_smem(reinterpret_cast<const void*>(tr_select_kernel<true>), (int)kTrStageMax);
+      if (err != cudaSuccess) return err;
       launch_pdl(tr_select_kernel<true>, dim3(r.E), dim3(1024), staged, s, r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
                                                         r.finalT);
     } else {

@@ -362,9 +362,12 @@ moe_status moe_profile_read(int32_t i, const char** name, float* ms);
  *     contents (each call writes every scratch byte it reads first).  Calls
  *     whose GPU work overlaps race on it: order them (one stream, or events).
  *   - Returns MOE_ERR_SCRATCH_LIMIT, without touching the GPU, when the shape
- *     needs more than 16 MiB of scratch:
- *       2*d*3*ceil(E/64)*64 + 4*ceil(T/256)*E + 4*T*K bytes (each part rounded
- *       up to 256 bytes).
+ *     needs more than 16 MiB (16777216 bytes) of scratch, namely the sum of
+ *       2*d*3*ceil(E/64)*64    (Wr split)
+ *       16                     (block-completion counters)
+ *       4*ceil(T/256)*E        (chunk histograms)
+ *       4*T*K                  (pair ranks)
+ *     bytes, each of the four parts rounded up to a multiple of 256.
  */
 moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
                              const float* bias, const moe_routing* rt, void* stream);

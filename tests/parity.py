@@ -30,6 +30,18 @@ def normwise(gpu, ref):
     return float(np.abs(gpu - ref).max() / scale)
 
 
+def elementwise(gpu, ref, floor=1e-2):
+    """Largest elementwise relative error |gpu - ref| / |ref| over the entries
+    with |ref| above `floor` times max |ref| (reported beside the normwise
+    error; bf16 storage alone puts it near 2^-9)."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    big = np.abs(ref) > floor * np.abs(ref).max()
+    if not big.any():
+        return 0.0
+    return float((np.abs(gpu - ref)[big] / np.abs(ref)[big]).max())
+
+
 def run_layer(inp, T, d, E, n, K, round_mode=0, router_grad=1, seed=0):
     import torch
     from fine_grained_mixture_top_b200 import moe
@@ -153,3 +165,28 @@ def tokens_of_expert(g, e):
     pe = g["pair_expert"]
     pair_tok = np.repeat(np.arange(len(g["tok_ptr"]) - 1), np.diff(g["tok_ptr"]))
     return np.unique(pair_tok[pe == e])
+
+
+def expert_columns_problem(g, z, e, te, J, W1, W2, n):
+    """The oracle's sub-problem for columns J of expert e's weight gradients.
+
+    SwiGLU acts column by column (A_j depends on g_j and u_j only), and
+    dW1[e][:, j], dW1[e][:, n + j] and dW2[e][j, :] depend only on column j of
+    the gate and up projections, on row j of W2[e] and on each row's gate s_r.
+    So a layer whose only expert has the weights W1[e][:, J | n + J] and
+    W2[e][J, :], fed the tokens of e with their full-set gates, has exactly the
+    weight gradients dW1[e][:, J | n + J] and dW2[e][J, :] of the full layer.
+    Returns (routing, W1 sub [1, d, 2|J|], W2 sub [1, |J|, d])."""
+    te = np.asarray(te, np.int64)
+    full = sub_routing(g, z, te)
+    sel = full["pair_expert"] == e
+    assert sel.sum() == len(te)
+    gate = full["pair_gate"][sel]
+    tok_ptr = np.arange(len(te) + 1, dtype=np.int64)
+    rt = {"z": None, "probs": None, "topk_idx": np.zeros((len(te), 1), np.int64), "tok_ptr": tok_ptr,
+          "pair_expert": np.zeros(len(te), np.int64), "pair_gate": gate}
+    J = np.asarray(J, np.int64)
+    cols = np.concatenate([J, n + J])
+    W1s = np.asarray(W1[e], np.float64)[:, cols][None]
+    W2s = np.asarray(W2[e], np.float64)[J, :][None]
+    return rt, W1s, W2s

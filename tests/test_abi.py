@@ -120,3 +120,56 @@ def test_status_strings(moe):
     assert moe.status_str(0) == "ok"
     assert "timed out" in moe.status_str(5)
     assert moe.status_str(99) == "unknown status"
+
+
+def _noalloc_bytes(T, d, E, K):
+    """Scratch of moe_route_noalloc by the formula its header documents."""
+    up = lambda x: -(-x // 256) * 256   # noqa: E731
+    return (up(2 * d * 3 * (-(-E // 64) * 64)) + up(16) + up(4 * (-(-T // 256)) * E) + up(4 * T * K))
+
+
+def test_route_noalloc_scratch_limit_follows_the_documented_formula():
+    """Shapes the formula puts within 16 MiB get past the scratch check (and
+    fail the null-pointer check); shapes just beyond it are refused."""
+    import ctypes
+    from fine_grained_mixture_top_b200 import moe
+    limit = 16 << 20
+    d, E, K = 1024, 64, 8
+    # largest T (multiple of 8) that fits, by the formula
+    T = 8
+    while _noalloc_bytes(T + 8, d, E, K) <= limit:
+        T += 8
+    for t, fits in ((T, True), (T + 8, False), (T + 4096, False), (1000, True)):
+        assert (_noalloc_bytes(t, d, E, K) <= limit) == fits
+        rt = moe.MoeRouting()
+        rc = moe.lib().moe_route_noalloc(ctypes.byref(moe.dims_of(t, d, E, 64, K)), ctypes.byref(moe.opts_of()),
+                                         None, None, None, ctypes.byref(rt), None)
+        assert rc == (moe.MOE_ERR_INVALID_ARG if fits else moe.MOE_ERR_SCRATCH_LIMIT), (t, rc)
+
+
+def test_saved_activation_is_constant_in_granularity():
+    """The only per-(token, expert) tensor kept from forward to backward is H
+    [R, 2n] (moe_sizes.h_elems); neither Y nor A is kept.  At a fixed activated
+    width K*n, making experts finer (E up, n down, K up) leaves it unchanged
+    up to the 128-row padding of each expert's segment, while a layer that
+    cached Y [T*K, d] would grow with K (page "DeepSeek做大→Mega MoE，Tri Dao团队
+    加快→SonicMoE", section "第一，激活内存与专家粒度解耦"; the activation
+    memory of the paper summary's results paragraph)."""
+    from fine_grained_mixture_top_b200 import moe
+    T, d = 16384, 1536
+    family = [(64, 512, 4), (128, 256, 8), (256, 128, 16), (512, 64, 32)]   # K * n = 2048
+    saved, y_cache = [], []
+    for E, n, K in family:
+        s = moe.query_sizes(moe.dims_of(T, d, E, n, K), moe.opts_of())
+        assert s.h_elems == s.R_max * 2 * n
+        # padding: at most 127 rows per expert, i.e. at most 127 E 2n = 254 E n elements
+        assert 2 * T * K * n <= s.h_elems <= 2 * T * K * n + 254 * E * n + 2 * 128 * n
+        saved.append(s.h_elems)
+        y_cache.append(T * K * d)
+    # 2 T K n = 2 T * 2048 on the whole family; padding adds at most 254 E n
+    # (E n = 32768 throughout) plus the final round-up to 128 rows, under 13 %
+    base = 2 * T * 2048
+    for (E, n, K), h in zip(family, saved):
+        assert base <= h <= base + 254 * E * n + 256 * n
+    assert max(saved) / min(saved) < 1.13
+    assert y_cache[-1] == 8 * y_cache[0]

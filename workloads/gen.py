@@ -93,12 +93,17 @@ def _gen(torch, device, seed: int):
     return g
 
 
-def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True, rank: int = 0) -> dict:
+def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True, rank: int = 0,
+                experts=None) -> dict:
     """Return the seeded input tensors of `cfg` on `device` (torch tensors).
 
-    Large weight tensors are produced one expert at a time so that the fp32
-    temporaries stay small.  `rank` selects a different batch of tokens (X and
-    dO) for data-parallel replica `rank`; the weights do not depend on it.
+    Large weight tensors are produced one expert at a time, each expert from
+    its own seed, so that the fp32 temporaries stay small and a subset of the
+    experts can be produced alone: with `experts` (a list of expert ids) W1
+    and W2 hold only those experts, in that order, with the same values the
+    full tensors hold for them.  `rank` selects a different batch of tokens
+    (X and dO) for data-parallel replica `rank`; the weights do not depend on
+    it.
     """
     import torch
 
@@ -109,11 +114,13 @@ def make_inputs(cfg: MoEConfig, device="cpu", need_grad_inputs: bool = True, ran
     g = _gen(torch, dev, data + 1)
     out["X"] = (torch.randn(cfg.T, cfg.d, generator=g, device=dev) * cfg.x_std).to(torch.bfloat16)
 
+    ids = list(range(cfg.E)) if experts is None else [int(e) for e in experts]
+
     def expert_weights(shape_e, seed):
-        w = torch.empty((cfg.E,) + shape_e, dtype=torch.bfloat16, device=dev)
-        g_ = _gen(torch, dev, seed)
-        for e in range(cfg.E):
-            w[e] = (torch.randn(shape_e, generator=g_, device=dev) * cfg.w_std).to(torch.bfloat16)
+        w = torch.empty((len(ids),) + shape_e, dtype=torch.bfloat16, device=dev)
+        for i, e in enumerate(ids):
+            g_ = _gen(torch, dev, seed * 1_000_003 + e)
+            w[i] = (torch.randn(shape_e, generator=g_, device=dev) * cfg.w_std).to(torch.bfloat16)
         return w
 
     out["W1"] = expert_weights((cfg.d, 2 * cfg.n), base + 2)
