@@ -17,7 +17,10 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 
-SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_route.cu", "moe_agg.cu", "moe_mx.cu", "moe_ep.cu"]
+SOURCES = ["moe_api.cu", "moe_gemm.cu", "moe_route.cu", "moe_agg.cu", "moe_mx.cu", "moe_ep.cu", "moe_debug.cu"]
+# the debug build: the same sources with the device-side routing checks on
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libmoe_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xptxas", "-v", "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]
@@ -38,12 +41,12 @@ def _deps_mtime() -> float:
     return newest
 
 
-def _compile(src: str, force: bool) -> tuple[str, str]:
-    obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+def _compile(src: str, force: bool, debug: bool = False) -> tuple[str, str]:
+    obj = os.path.join(BUILD_DEBUG if debug else BUILD, src.replace(".cu", ".o"))
     path = os.path.join(CSRC, src)
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= _deps_mtime():
         return obj, ""
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", path, "-o", obj]
+    cmd = [nvcc(), *ARCH, *FLAGS, *(["-DMOE_DEBUG=1"] if debug else []), "-c", path, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
@@ -52,20 +55,23 @@ def _compile(src: str, force: bool) -> tuple[str, str]:
     return obj, r.stderr
 
 
-def build(force: bool = False, jobs: int = 4, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int = 4, verbose: bool = False, debug: bool = False) -> str:
+    """Build libmoe.so, or with debug=True libmoe_debug.so (MOE_DEBUG=1:
+    device-side routing checks that report through the status word)."""
+    out_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    os.makedirs(out_dir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        results = list(ex.map(lambda s: _compile(s, force), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, force, debug), SOURCES))
     objs = [o for o, _ in results]
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs]
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", lib, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
@@ -73,5 +79,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-j", type=int, default=4)
     ap.add_argument("-v", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libmoe_debug.so (device-side routing checks)")
     a = ap.parse_args()
-    print(build(a.force, a.j, a.v))
+    print(build(a.force, a.j, a.v, a.debug))

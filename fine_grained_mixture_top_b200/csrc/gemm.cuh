@@ -238,6 +238,24 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
   return t;
 }
 
+// Token id of a gathered row.  The debug build (MOE_DEBUG=1) checks it and
+// turns an out-of-range id into a padding row (zero fill) after recording
+// the violation, so that no copy leaves the gathered tensor.
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+template <int KIND>
+__device__ __forceinline__ int gather_tok(const GemmParams& p, int r) {
+  int tok = __ldg(p.row_tok + r);
+#if MOE_DEBUG
+  if (tok < -1 || tok >= p.T) {
+    raise_status(p.st, ST_DEVICE_CHECK, 0x200 + KIND);
+    tok = -1;
+  }
+#endif
+  return tok;
+}
+
 // Byte offset of 16-byte chunk `c` of 128-byte line `i` in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(int line, int chunk) {
   return (uint32_t)(line * 128 + ((chunk ^ (line & 7)) << 4));
@@ -1063,7 +1081,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         int toks[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int tok = __ldg(p.row_tok + t.m0 + line0 + 16 * j);
+          const int tok = gather_tok<KIND>(p, t.m0 + line0 + 16 * j);
           toks[j] = tok;
           src[j] = p.gsrc + (size_t)(tok < 0 ? 0 : tok) * p.gld + chunk * 8;
           nbytes[j] = tok < 0 ? 0u : 16u;
@@ -1108,7 +1126,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         for (int q = 0; q < 2; ++q)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            tk[q + 1][j] = q < t.nkb ? __ldg(p.row_tok + t.krow0 + q * kBK + line0 + 16 * j) : -1;
+            tk[q + 1][j] = q < t.nkb ? gather_tok<KIND>(p, t.krow0 + q * kBK + line0 + 16 * j) : -1;
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % GS;
 #pragma unroll
@@ -1118,7 +1136,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           }
           if (kb + 2 < t.nkb) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tk[2][j] = __ldg(p.row_tok + t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
+            for (int j = 0; j < 4; ++j) tk[2][j] = gather_tok<KIND>(p, t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
           }
           if (!mbar_wait(smem_u32(&g_empty[s]), ((it / GS) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
             ok = false;

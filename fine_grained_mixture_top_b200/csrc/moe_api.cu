@@ -340,6 +340,44 @@ GemmParams base_params(const Plan& p, const moe_routing* rt, int* status) {
   return g;
 }
 
+// Debug build: check the routing's invariants on the device before (or
+// after) a step uses (or builds) it, wait for the check and report a
+// violation as cudaErrorInvalidValue (the caller returns MOE_ERR_DEVICE_CHECK
+// through moe_get_status, and launches nothing more).  Nothing is launched,
+// and nothing waits, in the release build.
+cudaError_t validate_routing(const Plan& p, const moe_routing* rt, int* status, cudaStream_t st) {
+  if (!MOE_DEBUG) return cudaSuccess;
+  RoutingView v;
+  v.T = p.T;
+  v.P_max = p.P_max;
+  v.R_max = p.R_max;
+  v.E = p.E;
+  v.tok_ptr = rt->tok_ptr;
+  v.pair_expert = rt->pair_expert;
+  v.pair_row = rt->pair_row;
+  v.counts = rt->counts;
+  v.offsets = rt->offsets;
+  v.row_tok = rt->row_tok;
+  v.tile_expert = rt->tile_expert;
+  {
+    ProfScope ps(st, "validate_routing");
+    cudaError_t e = launch_validate_routing(v, DevStatus{status, g_spin_limit}, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  int h = 0;
+  e = cudaMemcpy(&h, status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return e;
+  return h == 0 ? cudaSuccess : cudaErrorInvalidValue;
+}
+#define MOE_VALIDATE(p, rt, status, st)                              \
+  do {                                                               \
+    const cudaError_t moe_v_ = validate_routing(p, rt, status, st);  \
+    if (moe_v_ == cudaErrorInvalidValue) return MOE_ERR_DEVICE_CHECK; \
+    if (moe_v_ != cudaSuccess) return cuda_failed(moe_v_, __LINE__);  \
+  } while (0)
+
 // Records event grad_ready[i] (a cudaEvent_t, may be null) on the stream.
 // Recording cannot fail on a valid event; a failure surfaces at the next sync.
 inline void record_ready(void* const* grad_ready, int i, cudaStream_t st) {
@@ -451,6 +489,7 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
     MOE_TRY_CUDA(launch_softmax_topk(a, st));
   }
   MOE_TRY_CUDA(launch_permute(a, st));
+  MOE_VALIDATE(p, rt, status, st);
   return MOE_OK;
 }
 
@@ -483,6 +522,7 @@ moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe
   r.blk = w.blk;
   r.sync = w.sync + 1;
   MOE_TRY_CUDA(launch_token_round(a, r, static_cast<cudaStream_t>(stream)));
+  MOE_VALIDATE(p, rt, status, static_cast<cudaStream_t>(stream));
   return MOE_OK;
 }
 
@@ -504,6 +544,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
   if (!device_state(&dev, &status, &sms) || !get_encode()) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t mtiles = p.R_max / kTile;
+  MOE_VALIDATE(p, rt, status, st);
 
   // up-projection: H = X[tok] W1[e], A = SwiGLU(H)
   {
@@ -559,6 +600,7 @@ moe_status forward_mx(const Plan& p, const void* X, const MxWeights& wt, const m
                       const MxFwdWs& w, int* status, int sms, cudaStream_t st) {
   const int64_t mtiles = p.R_max / kTile;
   const int E = p.E, d = p.d, n = p.n;
+  MOE_VALIDATE(p, rt, status, st);
   {
     ProfScope ps(st, "mx_quant_x");
     MOE_TRY_CUDA(launch_mx_quant_rows(static_cast<const __nv_bfloat16*>(X), p.T, d, w.Xq, w.SX, st));
@@ -744,6 +786,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
   const int64_t mtiles = p.R_max / kTile;
   const __nv_bfloat16* dOb = static_cast<const __nv_bfloat16*>(dO);
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  MOE_VALIDATE(p, rt, status, st);
   // dH kernel: dA' = dO[tok] W2[e]^T; epilogue: H -> A, dS partials, dSwiGLU, A_hat
   {
     GemmParams g = base_params(p, rt, status);
@@ -868,6 +911,7 @@ moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe
                                     rt->pair_gate, a.st, st));
   }
   MOE_TRY_CUDA(launch_permute(a, st));
+  MOE_VALIDATE(p, rt, status, st);
   return MOE_OK;
 }
 
@@ -1119,5 +1163,6 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* op
   MOE_TRY_CUDA(launch_gemm(G_RTR, 192, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
   MOE_TRY_CUDA(launch_softmax_topk(a, st));
   MOE_TRY_CUDA(launch_permute(a, st));
+  MOE_VALIDATE(p, rt, status, st);
   return MOE_OK;
 }

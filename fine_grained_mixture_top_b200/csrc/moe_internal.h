@@ -134,6 +134,19 @@ cudaError_t launch_ep_pack(int T, int d, int E, int64_t R_max, int64_t P_max, co
                            const __nv_bfloat16* src, __nv_bfloat16* send, float* send_gate, int* pair_pos, int* cum,
                            cudaStream_t s);
 
+// ---- debug build only (moe_debug.cu): routing consistency checks
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+struct RoutingView {
+  int64_t T, P_max, R_max;
+  int E;
+  const int *tok_ptr, *pair_expert, *pair_row, *counts, *offsets, *row_tok, *tile_expert;
+};
+// Checks the routing's invariants; a violation sets MOE_ERR_DEVICE_CHECK in
+// the status word.  A no-op (no launch) unless built with MOE_DEBUG=1.
+cudaError_t launch_validate_routing(const RoutingView& v, DevStatus st, cudaStream_t s);
+
 // ---- MXFP8 quantization (moe_mx.cu)
 cudaError_t launch_mx_quant_rows(const __nv_bfloat16* in, int64_t rows, int K, uint8_t* codes, uint8_t* scales,
                                  cudaStream_t s);

@@ -11,7 +11,9 @@ import os
 from dataclasses import dataclass
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# MOE_DEBUG=1 in the environment loads the debug build instead (device-side
+# routing checks reported through moe_get_status; same results otherwise)
+LIB_PATH = os.path.join(_PKG, "libmoe_debug.so" if os.environ.get("MOE_DEBUG") == "1" else "libmoe.so")
 
 c_void_p = ctypes.c_void_p
 c_int32 = ctypes.c_int32
@@ -61,8 +63,9 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libmoe.so is not built ({LIB_PATH}); run python -m "
-                               "fine_grained_mixture_top_b200.build")
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run python -m "
+                               "fine_grained_mixture_top_b200.build" +
+                               (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.POINTER
         L.moe_query_sizes.argtypes = [P(MoeDims), P(MoeOpts), P(MoeSizes)]
