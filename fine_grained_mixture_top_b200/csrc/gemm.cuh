@@ -74,7 +74,30 @@ struct GemmParams {
   const uint8_t* sfb_src;    // weight scale tiles [E][N tiles][K/128]
   uint8_t* aq_out;           // UPQ: A codes [R_max, n]
   uint8_t* sa_out;           // UPQ: A scale tiles [R_max/128][n/128]
+  // Role timeline (moe_trace_gemm), null when off: per CTA and role, up to
+  // trace_cap records of (globaltimer ns, clock64 low bits, tile << 8 | event)
+  uint8_t* trace;
+  int trace_cap;
 };
+
+// One timeline record; roles: 0 TMA producer, 1 MMA issuer, 2 epilogue
+// (its first warp), 3 gather warps (their first thread).
+struct TraceRec {
+  unsigned long long ns;
+  uint32_t clk;
+  uint32_t info;  // tile << 8 | event
+};
+__device__ __forceinline__ void trace_ev(const GemmParams& p, int role, int& n, int tile, int ev) {
+  if (p.trace && n < p.trace_cap) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    TraceRec* r = reinterpret_cast<TraceRec*>(p.trace) + ((size_t)blockIdx.x * 4 + role) * p.trace_cap + n;
+    r->ns = t;
+    r->clk = (uint32_t)clock64();
+    r->info = ((uint32_t)tile << 8) | (uint32_t)ev;
+    ++n;
+  }
+}
 
 template <int KIND>
 struct KindTraits {
@@ -524,12 +547,13 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
-      int it = 0;
+      int it = 0, ntr = 0;
       bool ok = true;
       for (int ti = 0; ok; ++ti) {
         const int tile = produce_tile(ti, ok);
         if (!ok || tile >= num_tiles) break;
         const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+        trace_ev(p, 0, ntr, tile, 0);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
           if constexpr (!kSplit) {
@@ -547,6 +571,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
                               base + SH::kSFAOffset + (uint32_t)(sa * SH::kSFABytes),
                               base + SH::kSFBOffset + (uint32_t)(sb * SH::kSFBBytes));
         }
+        trace_ev(p, 0, ntr, tile, 1);
       }
     }
   } else if (warp == 1 && KIND == G_RTR) {
@@ -612,13 +637,14 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
-    int it = 0, tcount = 0;
+    int it = 0, tcount = 0, ntr = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
       const int tile = consume_tile(ti, ok);
       if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (t.nkb == 0) continue;
+      if (lane == 0) trace_ev(p, 1, ntr, tile, 0);
       const int b = tcount & 1;
       const int use = tcount >> 1;
       if (!mbar_wait(smem_u32(&acc_empty[b]), (use & 1) ^ 1, abort_flag, p.st, KIND * 16 + 2)) {
@@ -626,6 +652,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         break;
       }
       tc_fence_after();
+      if (lane == 0) trace_ev(p, 1, ntr, tile, 1);
       const uint32_t d_tmem = tmem_base + (uint32_t)(b * SH::kAccStride);
       for (int kb = 0; kb < t.nkb; ++kb, ++it) {
         const int sa = it % SA, sb = it % SB;
@@ -635,6 +662,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           break;
         }
         tc_fence_after();
+        if (kb == 0 && lane == 0) trace_ev(p, 1, ntr, tile, 2);
         if (lane == 0) {
           const uint32_t a_s = a_slot(sa);
           const uint32_t b_s = b_slot(sb);
@@ -669,7 +697,10 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) tc_commit(smem_u32(&acc_full[b]));
+      if (lane == 0) {
+        tc_commit(smem_u32(&acc_full[b]));
+        trace_ev(p, 1, ntr, tile, 3);
+      }
       __syncwarp();
       ++tcount;
     }
@@ -761,12 +792,14 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       fence_proxy_async_smem();
       __syncwarp();
     };
-    int tcount = 0;
+    int tcount = 0, ntr = 0;
+    const bool tracer = (warp == 2 && lane == 0);
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
       const int tile = consume_tile(ti, ok);
       if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if (tracer) trace_ev(p, 2, ntr, tile, 0);
       const int row0 = t.m0 + q * 32;  // first output row of this warp's slice
       if constexpr (KT::kGroupedK) {
         if (t.nkb == 0) {  // expert without tokens: its weight gradient is zero
@@ -830,6 +863,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       const int use = tcount >> 1;
       if (!mbar_wait(smem_u32(&acc_full[b]), use & 1, abort_flag, p.st, KIND * 16 + 4)) break;
       tc_fence_after();
+      if (tracer) trace_ev(p, 2, ntr, tile, 1);
       const uint32_t tacc = lane_addr + (uint32_t)(b * SH::kAccStride);
 
       if constexpr (KIND == G_UP) {
@@ -1051,6 +1085,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[b]));
+      if (tracer) trace_ev(p, 2, ntr, tile, 2);
       ++tcount;
     }
     if (lane == 0) bulk_wait_all();  // stores finished before the CTA exits
@@ -1064,13 +1099,14 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     constexpr int GS = KT::kAGather ? SA : SB;
     uint64_t* g_full = KT::kAGather ? full_a : full_b;
     uint64_t* g_empty = KT::kAGather ? empty_a : empty_b;
-    int it = 0;
+    int it = 0, ntr = 0;
     int pending = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
       const int tile = consume_tile(ti, ok);
       if (!ok || tile >= num_tiles) break;
       const TileInfo t = gemm_tile<KIND, BN>(p, tile);
+      if (gt == 0) trace_ev(p, 3, ntr, tile, 0);
       if constexpr (KIND == G_UP || KIND == G_DH || KIND == G_UPQ) {
         // A tile = 128 gathered rows x 128 bytes of K; this thread: lines
         // line0 + 16 j (MXFP8: the codes are read as pairs of bytes, so the
@@ -1116,6 +1152,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
             ++pending;
           }
         }
+        if (gt == 0) trace_ev(p, 3, ntr, tile, 1);
       } else {
         // MN-major gathered operand: 64 K-rows (tokens) per k-block.  The row
         // indices of the next two k-blocks are loaded ahead, so the dependent
@@ -1164,6 +1201,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
             ++pending;
           }
         }
+        if (gt == 0) trace_ev(p, 3, ntr, tile, 1);
         if constexpr (kDyn) {
           // Before blocking on the queue for the next tile, publish this
           // tile's last k-blocks: a stage held back while this warp waits on

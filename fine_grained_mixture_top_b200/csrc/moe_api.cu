@@ -1069,6 +1069,14 @@ moe_status moe_profile_read(int32_t i, const char** name, float* ms) {
   return MOE_OK;
 }
 
+moe_status moe_trace_gemm(int32_t kind, void* buf, int64_t records_per_role) {
+  if (kind < -1 || kind > G_DOWNQ) return MOE_ERR_INVALID_ARG;
+  if (buf && kind >= 0 && (records_per_role < 1 || records_per_role > (1 << 24) || !aligned16(buf)))
+    return MOE_ERR_INVALID_ARG;
+  set_gemm_trace(kind, kind >= 0 ? buf : nullptr, (int)records_per_role);
+  return MOE_OK;
+}
+
 const char* moe_last_error(void) { return g_last_error; }
 
 const char* moe_status_str(moe_status s) {

@@ -40,7 +40,31 @@ cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
   return cudaSuccess;
 }
 
-cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s) {
+// Role timeline of one GEMM kind (moe_trace_gemm): the next launches of that
+// kind write their records into the selected buffer.
+namespace {
+std::mutex g_trace_mu;
+int g_trace_kind = -1;
+uint8_t* g_trace_buf = nullptr;
+int g_trace_cap = 0;
+}  // namespace
+
+void set_gemm_trace(int kind, void* buf, int cap) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_kind = buf ? kind : -1;
+  g_trace_buf = static_cast<uint8_t*>(buf);
+  g_trace_cap = cap;
+}
+
+cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p_in, int grid, cudaStream_t s) {
+  GemmParams p = p_in;
+  {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (kind == g_trace_kind) {
+      p.trace = g_trace_buf;
+      p.trace_cap = g_trace_cap;
+    }
+  }
 #define MOE_CASE(K, B, W) \
   if (kind == K && bn == B && epi == W) return launch_one<K, B, W>(p, grid, s);
   MOE_CASE(G_UP, 128, 4)

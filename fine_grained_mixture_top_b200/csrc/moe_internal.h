@@ -41,6 +41,10 @@ constexpr int kChunk = 256;       // tokens per ranking chunk of the permutation
 // (function, device); thread-safe.
 cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
 
+// Role timeline of GEMM kind `kind` (GemmKind) into `buf` (null: off), `cap`
+// records per CTA and role.
+void set_gemm_trace(int kind, void* buf, int cap);
+
 // epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
 

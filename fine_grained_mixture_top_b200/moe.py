@@ -108,6 +108,8 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_count.restype = c_int32
         L.moe_profile_read.argtypes = [c_int32, P(ctypes.c_char_p), P(ctypes.c_float)]
         L.moe_profile_read.restype = c_int32
+        L.moe_trace_gemm.argtypes = [c_int32, c_void_p, c_int64]
+        L.moe_trace_gemm.restype = c_int32
         L.moe_status_str.argtypes = [c_int32]
         L.moe_status_str.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
@@ -339,6 +341,48 @@ def moe_profile_records() -> list[tuple[str, float]]:
         _check(L.moe_profile_read(i, ctypes.byref(name), ctypes.byref(ms)), "moe_profile_read")
         out.append((name.value.decode(), float(ms.value)))
     return out
+
+
+GEMM_KINDS = {"up_proj_gemm": 0, "down_proj_gemm": 1, "dh_gemm": 2, "dxt_gemm": 3, "dw1_gemm": 4, "dw2_gemm": 5,
+              "router_logits_gemm": 6, "router_dwr_gemm": 7, "up_proj_gemm_mx": 8, "down_proj_gemm_mx": 9}
+
+
+class GemmTrace:
+    """Role timeline of one grouped-GEMM kind (moe_trace_gemm): start() before
+    the launches to trace, stop() after them, then records() gives one numpy
+    structured array per (CTA, role) with fields ns, clk, tile, event."""
+
+    ROLES = ("producer", "mma", "epilogue", "gather")
+
+    def __init__(self, kernel: str, records_per_role: int = 4096, device="cuda"):
+        import torch
+        self.kind = GEMM_KINDS[kernel]
+        self.cap = int(records_per_role)
+        sms = torch.cuda.get_device_properties(torch.device(device)).multi_processor_count
+        self.ctas = sms
+        self.buf = torch.zeros(self.ctas * 4 * self.cap * 16, dtype=torch.uint8, device=device)
+
+    def start(self):
+        self.buf.zero_()
+        _check(lib().moe_trace_gemm(self.kind, _ptr(self.buf), self.cap), "moe_trace_gemm")
+
+    def stop(self):
+        _check(lib().moe_trace_gemm(-1, None, 0), "moe_trace_gemm")
+
+    def records(self):
+        import numpy as np
+        raw = self.buf.cpu().numpy()
+        dt = np.dtype([("ns", "<u8"), ("clk", "<u4"), ("info", "<u4")])
+        rec = raw.view(dt).reshape(self.ctas, 4, self.cap)
+        out = {}
+        for c in range(self.ctas):
+            for r in range(4):
+                x = rec[c, r]
+                x = x[x["ns"] != 0]
+                out[(c, self.ROLES[r])] = {"ns": x["ns"].astype(np.int64), "clk": x["clk"].astype(np.int64),
+                                           "tile": (x["info"] >> 8).astype(np.int64),
+                                           "event": (x["info"] & 0xFF).astype(np.int64)}
+        return out
 
 
 class MoELayer:

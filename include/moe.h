@@ -344,6 +344,29 @@ int32_t moe_profile_count(void);
 moe_status moe_profile_read(int32_t i, const char** name, float* ms);
 
 /*
+ * Role timeline of one grouped-GEMM kind (tracing; the pages report per-kernel
+ * tensor-core utilisation and HBM traffic of their kernels, page
+ * "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE", section "第二，IO 感知的
+ * 算子融合" -- this shows where inside one of these kernels the time goes).
+ * kind: 0 up-proj, 1 down-proj, 2 dH, 3 dX~, 4 dW1, 5 dW2, 6 router logits,
+ * 7 router dWr, 8 MXFP8 up-proj, 9 MXFP8 down-proj; -1 (or buf NULL) turns
+ * tracing off.  While on, every launch of that kind writes, per CTA and role
+ * (0 TMA producer, 1 MMA issuer, 2 epilogue, 3 gather warps), up to
+ * `records_per_role` 16-byte records {u64 %globaltimer ns, u32 clock64 low
+ * bits, u32 tile << 8 | event} at
+ *   buf + 16 * ((cta * 4 + role) * records_per_role + i),
+ * so buf needs 64 * grid * records_per_role bytes (grid <= the SM count).
+ * The caller zeroes buf (a zero record is unused).  Events per tile:
+ * producer 0 tile taken, 1 last k-block issued; MMA 0 tile taken,
+ * 1 accumulator free, 2 first k-block's operands ready, 3 last MMA committed;
+ * epilogue 0 tile taken, 1 accumulator full, 2 accumulator released (its
+ * stores issued); gather 0 tile taken, 1 last k-block's copies issued.
+ * Launches in flight keep the buffer: turn tracing off or synchronize before
+ * freeing it.  Results do not depend on tracing.
+ */
+moe_status moe_trace_gemm(int32_t kind, void* buf, int64_t records_per_role);
+
+/*
  * moe_route_noalloc -- moe_route for callers that cannot allocate device
  * memory.  Such callers exist: a plugin that a host runtime hands only its
  * input and output buffers, or code running under an allocator that owns the
