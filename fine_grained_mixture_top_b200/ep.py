@@ -81,10 +81,19 @@ class ExpertParallelMoE:
         counts = eng.counts().to(torch.int64)
         recv_counts = torch.empty_like(counts)
         dist.all_to_all_single(recv_counts, counts.contiguous(), group=self.group)
-        sc = counts.cpu().numpy().reshape(self.G, self.E_loc)
-        rc = recv_counts.cpu().numpy().reshape(self.G, self.E_loc)
-        send_splits, recv_splits, local_expert = exchange_plan(sc, rc)
-        rows, gate, pair_pos = eng.pack(X, with_gate=True)
+        # The one host synchronisation of the step: the all-to-alls take their
+        # split sizes as host integers.  Both count vectors come back in one
+        # copy; everything else stays on the device.
+        both = torch.stack([counts, recv_counts]).cpu().numpy()
+        sc = both[0].reshape(self.G, self.E_loc)
+        rc = both[1].reshape(self.G, self.E_loc)
+        send_splits, recv_splits, _ = exchange_plan(sc, rc)
+        # local expert of every received row, built on the device from the
+        # received counts (rows arrive source by source, expert-major)
+        R = int(sum(recv_splits))
+        ids = torch.arange(self.E_loc, dtype=torch.int32, device=recv_counts.device).repeat(self.G)
+        local_expert = torch.repeat_interleave(ids, recv_counts, output_size=R)
+        rows, gate, pair_pos = eng.pack(X, with_gate=True, n=int(sum(send_splits)))
         recv_rows = self._a2a(rows, send_splits, recv_splits)
         recv_gate = self._a2a(gate, send_splits, recv_splits)
         out_loc = eng.local_forward(recv_rows, local_expert, recv_gate, W1_loc, W2_loc)
@@ -102,7 +111,7 @@ class ExpertParallelMoE:
             raise RuntimeError("backward before forward")
         eng = self.engine
         send_splits, recv_splits, pair_pos = self._saved
-        rows, _, _ = eng.pack(dO, with_gate=False)
+        rows, _, _ = eng.pack(dO, with_gate=False, n=int(sum(send_splits)))
         recv_rows = self._a2a(rows, send_splits, recv_splits)
         dXt_loc, dS_loc, dW1_loc, dW2_loc = eng.local_backward(recv_rows, W1_loc, W2_loc)
         dXt = self._a2a(dXt_loc, recv_splits, send_splits)
@@ -168,11 +177,12 @@ class CudaEngine:
     def counts(self):
         return self.routing["counts"]
 
-    def pack(self, src, with_gate):
+    def pack(self, src, with_gate, n):
+        """Routed rows of `src` in expert-major send order (n of them: the
+        routing's total count, known on the host from the exchange plan)."""
         m = self.moe
         m.moe_ep_pack(self.dims, self.opts, self.routing, src, self.send_rows,
                       self.send_gate if with_gate else None, self.pair_pos if with_gate else None, self.ws_route)
-        n = int(self.routing["counts"].sum().item())
         return self.send_rows[:n], (self.send_gate[:n] if with_gate else None), self.pair_pos
 
     def _loc_dims(self, R):
@@ -186,7 +196,7 @@ class CudaEngine:
         if R == 0:
             return self.out_loc[:0]
         rt = self.loc_routing
-        rt["topk_idx"][:R, 0].copy_(torch.from_numpy(np.ascontiguousarray(local_expert, np.int32)))
+        rt["topk_idx"][:R, 0].copy_(local_expert)
         rt["topk_gate"][:R, 0].copy_(gate)
         dims = self._loc_dims(R)
         m.moe_route_given(dims, self.loc_opts, rt, self.loc_ws_route)

@@ -457,6 +457,28 @@ class MoELayer:
         return self.backward(dO, X, Wr, W1, W2, stream, grad_events)
 
 
+class CudaStreamHooks:
+    """Stream and event plumbing of OverlappedGradReduce on a CUDA device:
+    three events the backward records (dW2, dW1, dWr written), and a
+    communication stream that waits on each before its all-reduce."""
+
+    def __init__(self):
+        import torch
+        self.comm = torch.cuda.Stream()
+        self.events = [torch.cuda.Event() for _ in range(3)]
+
+    def on_comm(self):
+        import torch
+        return torch.cuda.stream(self.comm)
+
+    def wait(self, ev):
+        self.comm.wait_event(ev)
+
+    def join(self):
+        import torch
+        torch.cuda.current_stream().wait_stream(self.comm)
+
+
 class OverlappedGradReduce:
     """Data-parallel steps whose weight-gradient sums over `group` overlap the
     backward.  The backward records an event as soon as dW2, then dW1, then dWr
@@ -464,28 +486,30 @@ class OverlappedGradReduce:
     all-reduce waits on its event on a separate stream, so the reductions of
     dW2 and dW1 run while the dX~ GEMM and the dX aggregation do.  The current
     stream waits for the reductions at the end of the step, before the next
-    step can overwrite the gradients."""
+    step can overwrite the gradients.
 
-    def __init__(self, layer, group=None):
-        import torch
+    `hooks` supplies the streams and events (CudaStreamHooks by default); the
+    CPU tests pass host stand-ins so that the ordering logic runs on gloo
+    ranks."""
+
+    def __init__(self, layer, group=None, hooks=None):
         self.layer = layer
         self.group = group
-        self.comm = torch.cuda.Stream()
-        self.events = [torch.cuda.Event() for _ in range(3)]
+        self.hooks = hooks if hooks is not None else CudaStreamHooks()
 
     def step(self, X, Wr, bias, W1, W2, dO):
-        import torch
         import torch.distributed as dist
         L = self.layer
-        L.step(X, Wr, bias, W1, W2, dO, grad_events=self.events)
+        h = self.hooks
+        L.step(X, Wr, bias, W1, W2, dO, grad_events=h.events)
         grads = (L.dW2, L.dW1, L.dWr if L.opts.router_grad else None)
-        with torch.cuda.stream(self.comm):
-            for ev, g in zip(self.events, grads):
+        with h.on_comm():
+            for ev, g in zip(h.events, grads):
                 if g is None:
                     continue
-                self.comm.wait_event(ev)
+                h.wait(ev)
                 dist.all_reduce(g, group=self.group)
-        torch.cuda.current_stream().wait_stream(self.comm)
+        h.join()
         return L.dX, L.dW1, L.dW2, L.dWr
 
 

@@ -31,8 +31,9 @@ class OracleEngine:
     def counts(self):
         return torch.from_numpy(self.perm["counts"].astype(np.int64))
 
-    def pack(self, src, with_gate):
+    def pack(self, src, with_gate, n):
         # expert-major rows without padding: the oracle's permutation order
+        assert n == len(self.perm["row_tok"])
         rows = torch.from_numpy(np.ascontiguousarray(src.numpy()[self.perm["row_tok"]]))
         if not with_gate:
             return rows, None, None
@@ -59,7 +60,7 @@ class OracleEngine:
     def local_forward(self, rows, local_expert, gate, W1_loc, W2_loc):
         R = rows.shape[0]
         self.loc_X = rows.numpy()
-        rt = {"tok_ptr": np.arange(R + 1), "pair_expert": np.asarray(local_expert, np.int64),
+        rt = {"tok_ptr": np.arange(R + 1), "pair_expert": np.asarray(local_expert.numpy(), np.int64),
               "pair_gate": gate.numpy()}
         self.loc_fw = orc.forward(self.loc_X, None, None, W1_loc.numpy(), W2_loc.numpy(), 1, routing=rt)
         return torch.from_numpy(self.loc_fw["O"])

@@ -205,3 +205,111 @@ def test_expert_parallel_with_token_rounding():
         np.testing.assert_allclose(dW1, bw["dW1"][es], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dW2, bw["dW2"][es], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dWr, bw["dWr"], rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# The product's overlapped data-parallel reduction (moe.OverlappedGradReduce)
+# on gloo ranks: host stand-ins replace the CUDA streams and events, and a
+# layer whose step is the oracle's stands in for the kernels.  Checks the
+# order the reductions are issued in (each after its gradient's event, dW2
+# then dW1 then dWr), that the stream join comes last, and that the reduced
+# gradients are the full-batch ones.
+# ----------------------------------------------------------------------------
+class _HostHooks:
+    def __init__(self, log):
+        import contextlib
+        self.log = log
+        self.events = ["dW2 ready", "dW1 ready", "dWr ready"]
+        self._ctx = contextlib.nullcontext
+
+    def on_comm(self):
+        self.log.append("comm stream")
+        return self._ctx()
+
+    def wait(self, ev):
+        assert ev in self.log, f"waited on {ev} before the backward recorded it"
+        self.log.append("wait " + ev)
+
+    def join(self):
+        self.log.append("join")
+
+
+class _OracleLayer:
+    """Stand-in for MoELayer: its step is the oracle's on this rank's shard,
+    and it 'records' the gradient events in the backward's order."""
+
+    def __init__(self, K, log, router_grad=1):
+        import types
+        self.K = K
+        self.log = log
+        self.opts = types.SimpleNamespace(router_grad=router_grad)
+
+    def step(self, X, Wr, bias, W1, W2, dO, grad_events=None):
+        fw = orc.forward(X, Wr, bias, W1, W2, self.K)
+        bw = orc.backward(fw, dO, X, Wr, W1, W2, router_grad=bool(self.opts.router_grad))
+        self.dW2 = torch.from_numpy(bw["dW2"].copy())
+        self.log.append(grad_events[0])
+        self.dW1 = torch.from_numpy(bw["dW1"].copy())
+        self.log.append(grad_events[1])
+        self.dWr = torch.from_numpy(bw["dWr"].copy()) if self.opts.router_grad else None
+        self.log.append(grad_events[2])
+        self.dX = bw["dX"]
+
+
+def _overlap_worker(rank, world, port, K, router_grad, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from fine_grained_mixture_top_b200 import moe
+    X, W1, W2, Wr, b, dO = _layer()
+    T = X.shape[0]
+    sl = slice(rank * T // world, (rank + 1) * T // world)
+    log = []
+    layer = _OracleLayer(K, log, router_grad)
+    red = moe.OverlappedGradReduce(layer, hooks=_HostHooks(log))
+    # all_reduce is logged by wrapping the collective the class calls
+    real = dist.all_reduce
+
+    def logged(g, group=None):
+        log.append("all_reduce " + ("dW2" if g is layer.dW2 else "dW1" if g is layer.dW1 else "dWr"))
+        return real(g, group=group)
+
+    dist.all_reduce = logged
+    try:
+        dX, dW1, dW2, dWr = red.step(X[sl], Wr, b, W1, W2, dO[sl])
+    finally:
+        dist.all_reduce = real
+    out_q.put((rank, log, dW1.numpy(), dW2.numpy(), None if dWr is None else dWr.numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("router_grad", [1, 0])
+def test_overlapped_reduce_orders_and_sums_on_two_ranks(router_grad):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world, K = 2, 2
+    port = _free_port()
+    procs = [ctx.Process(target=_overlap_worker, args=(r, world, port, K, router_grad, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    X, W1, W2, Wr, b, dO = _layer()
+    fw = orc.forward(X, Wr, b, W1, W2, K)
+    bw = orc.backward(fw, dO, X, Wr, W1, W2)
+    want = ["dW2 ready", "dW1 ready", "dWr ready", "comm stream", "wait dW2 ready", "all_reduce dW2",
+            "wait dW1 ready", "all_reduce dW1"]
+    if router_grad:
+        want += ["wait dWr ready", "all_reduce dWr"]
+    want += ["join"]
+    for rank, log, dW1, dW2, dWr in got:
+        assert log == want, (rank, log)
+        np.testing.assert_allclose(dW1, bw["dW1"], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dW2, bw["dW2"], rtol=1e-10, atol=1e-12)
+        if router_grad:
+            np.testing.assert_allclose(dWr, bw["dWr"], rtol=1e-10, atol=1e-12)
+        else:
+            assert dWr is None
