@@ -64,8 +64,9 @@ struct GemmParams {
   const __nv_bfloat16* hin;
   float* outf;
   const float* bias;
-  int* sched;                // weight-gradient kinds: zeroed tile counter of the dynamic scheduler
+  int* sched;                // weight-gradient kinds: zeroed 64-bit tile counter (8-byte aligned)
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
+  int dual_ended;            // weight-gradient kinds: odd CTAs claim from the smallest experts' end
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
   // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
@@ -261,6 +262,25 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
   return t;
 }
 
+// Weight-gradient kinds: the tile whose expert-dependent fields (expert id,
+// first row, k-blocks) are already resolved -- the producer resolves them once
+// and hands them to the other roles through the shared-memory tile queue.
+template <int KIND, int BN>
+__device__ __forceinline__ TileInfo gemm_tile_resolved(const GemmParams& p, int tile, int e, int krow0, int nkb) {
+  TileInfo t;
+  const int per_e = p.num_m_tiles * p.num_n_tiles;
+  const int rem = tile - (tile / per_e) * per_e;
+  t.e = e;
+  t.mt = rem / p.num_n_tiles;
+  t.nt = rem - t.mt * p.num_n_tiles;
+  t.m0 = t.mt * kBM;
+  t.n0 = t.nt * BN;
+  t.krow0 = krow0;
+  t.nkb = nkb;
+  t.split = 0;
+  return t;
+}
+
 // Token id of a gathered row.  The debug build (MOE_DEBUG=1) checks it and
 // turns an out-of-range id into a padding row (zero fill) after recording
 // the violation, so that no copy leaves the gathered tensor.
@@ -452,7 +472,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   uint64_t* tq_empty = bars + 44;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 48);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 49);
-  volatile int* tq_slots = reinterpret_cast<volatile int*>(bars + 50);  // [kTileQ]
+  // [kTileQ] queued tiles {tile, expert, first row, k-blocks}; written and
+  // read between the queue's mbarrier arrive (release) and wait (acquire)
+  int4* tq_info = reinterpret_cast<int4*>(bars + 50);
   auto a_slot = [&](int i) -> uint32_t { return base + SH::kAOffset + (uint32_t)(i * kABytes); };
   auto b_slot = [&](int i) -> uint32_t { return base + SH::kBOffset + (uint32_t)(i * SH::kBBytes); };
   // the router-logit kind keeps one tile buffer of 256 columns: [hi_a | hi_b | mid | lo]
@@ -510,37 +532,85 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
 
   // Tile order.  Static kinds walk tiles round-robin.  The weight-gradient
   // kinds, whose tiles differ in length with the expert's token count, take
-  // tiles dynamically: the TMA thread draws the next tile from a global
-  // counter and hands it to the other roles through a shared-memory queue.
+  // tiles dynamically from a list ordered by expert, largest first: even CTAs
+  // claim from its front (the long, L2-bound tiles of the busiest experts),
+  // odd CTAs from its back (the short tiles of the smallest experts, bound by
+  // storing their results), so that both kinds of work run at once and the
+  // last tiles taken are the middle-sized ones.  One 64-bit counter holds
+  // both ends (front claims in the low word, back claims in the high word);
+  // claim k (the sum of both before the increment) is valid iff k < tiles.
+  // The TMA thread claims a tile one tile ahead (the atomic's latency hides
+  // behind the current tile's loads), resolves its expert once, and hands it
+  // to the other roles through a shared-memory queue.
   constexpr bool kDyn = KT::kGroupedK;
-  auto produce_tile = [&](int i, bool& good) -> int {
+  const bool front_end = !p.dual_ended || (blockIdx.x & 1u) == 0u;
+  const int nfront0 = p.dual_ended ? ((int)gridDim.x + 1) / 2 : (int)gridDim.x;  // first tiles, taken unclaimed
+  const int nback0 = (int)gridDim.x - nfront0;
+  auto claim = [&]() -> unsigned long long {
+    return atomicAdd(reinterpret_cast<unsigned long long*>(p.sched), front_end ? 1ull : (1ull << 32));
+  };
+  auto claimed_tile = [&](unsigned long long old) -> int {
+    const int f = (int)(old & 0xffffffffull) + nfront0;
+    const int b = (int)(old >> 32) + nback0;
+    if (f + b >= num_tiles) return num_tiles;
+    return front_end ? f : num_tiles - 1 - b;
+  };
+  unsigned long long next_claim = 0;
+  int res_ei = -1, res_e = 0, res_krow0 = 0, res_nkb = 0;  // the producer's last resolved expert
+  auto produce_tile = [&](int i, bool& good, TileInfo& t) -> int {
     if constexpr (kDyn) {
-      const int tile = i == 0 ? (int)blockIdx.x : atomicAdd(p.sched, 1) + (int)gridDim.x;
+      int tile;
+      if (i == 0) {
+        const int j = p.dual_ended ? ((int)blockIdx.x >> 1) : (int)blockIdx.x;
+        tile = front_end ? j : num_tiles - 1 - j;
+      } else {
+        tile = claimed_tile(next_claim);
+      }
+      if (tile < num_tiles) next_claim = claim();  // the next tile's claim, in flight meanwhile
+      int e = 0, krow0 = 0, nkb = 0;
+      if (tile < num_tiles) {
+        const int ei = tile / (p.num_m_tiles * p.num_n_tiles);
+        if (ei != res_ei) {
+          res_ei = ei;
+          res_e = p.expert_order ? __ldg(p.expert_order + ei) : ei;
+          res_krow0 = __ldg(p.offsets + res_e);
+          res_nkb = (__ldg(p.counts + res_e) + kBK - 1) / kBK;
+        }
+        e = res_e;
+        krow0 = res_krow0;
+        nkb = res_nkb;
+        t = gemm_tile_resolved<KIND, BN>(p, tile, e, krow0, nkb);
+      }
       const int slot = i % kTileQ;
       if (!mbar_wait(smem_u32(&tq_empty[slot]), ((i / kTileQ) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 10)) {
         good = false;
         return num_tiles;
       }
-      tq_slots[slot] = tile;
+      tq_info[slot] = make_int4(tile, e, krow0, nkb);
       mbar_arrive(smem_u32(&tq_full[slot]));
       return tile;
     } else {
-      return (int)blockIdx.x + i * (int)gridDim.x;
+      const int tile = (int)blockIdx.x + i * (int)gridDim.x;
+      if (tile < num_tiles) t = gemm_tile<KIND, BN>(p, tile);
+      return tile;
     }
   };
-  auto consume_tile = [&](int i, bool& good) -> int {
+  auto consume_tile = [&](int i, bool& good, TileInfo& t) -> int {
     if constexpr (kDyn) {
       const int slot = i % kTileQ;
       if (!mbar_wait(smem_u32(&tq_full[slot]), (i / kTileQ) & 1, abort_flag, p.st, KIND * 16 + 11)) {
         good = false;
         return num_tiles;
       }
-      const int tile = tq_slots[slot];
+      const int4 q = tq_info[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tq_empty[slot]));
-      return tile;
+      if (q.x < num_tiles) t = gemm_tile_resolved<KIND, BN>(p, q.x, q.y, q.z, q.w);
+      return q.x;
     } else {
-      return (int)blockIdx.x + i * (int)gridDim.x;
+      const int tile = (int)blockIdx.x + i * (int)gridDim.x;
+      if (tile < num_tiles) t = gemm_tile<KIND, BN>(p, tile);
+      return tile;
     }
   };
 
@@ -550,9 +620,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       int it = 0, ntr = 0;
       bool ok = true;
       for (int ti = 0; ok; ++ti) {
-        const int tile = produce_tile(ti, ok);
+        TileInfo t;
+        const int tile = produce_tile(ti, ok, t);
         if (!ok || tile >= num_tiles) break;
-        const TileInfo t = gemm_tile<KIND, BN>(p, tile);
         trace_ev(p, 0, ntr, tile, 0);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int sa = it % SA, sb = it % SB;
@@ -585,9 +655,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     int it = 0, tcount = 0, hg = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
-      const int tile = consume_tile(ti, ok);
+      TileInfo t;
+      const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (!mbar_wait(smem_u32(&acc_empty[0]), (tcount & 1) ^ 1, abort_flag, p.st, KIND * 16 + 7)) {
         ok = false;
         break;
@@ -640,9 +710,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     int it = 0, tcount = 0, ntr = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
-      const int tile = consume_tile(ti, ok);
+      TileInfo t;
+      const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (t.nkb == 0) continue;
       if (lane == 0) trace_ev(p, 1, ntr, tile, 0);
       const int b = tcount & 1;
@@ -712,9 +782,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     int tcount = 0, hg = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
-      const int tile = consume_tile(ti, ok);
+      TileInfo t;
+      const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       float hs[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) hs[i] = 0.f;
@@ -796,9 +866,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     const bool tracer = (warp == 2 && lane == 0);
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
-      const int tile = consume_tile(ti, ok);
+      TileInfo t;
+      const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (tracer) trace_ev(p, 2, ntr, tile, 0);
       const int row0 = t.m0 + q * 32;  // first output row of this warp's slice
       if constexpr (KT::kGroupedK) {
@@ -1102,10 +1172,12 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     int it = 0, ntr = 0;
     int pending = 0;
     bool ok = true;
+    int first_tk[2][4];                    // weight-gradient kinds: row tokens of the
+    int first_krow0 = -1, first_nkb = -1;  // last expert's first two k-blocks
     for (int ti = 0; ok; ++ti) {
-      const int tile = consume_tile(ti, ok);
+      TileInfo t;
+      const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      const TileInfo t = gemm_tile<KIND, BN>(p, tile);
       if (gt == 0) trace_ev(p, 3, ntr, tile, 0);
       if constexpr (KIND == G_UP || KIND == G_DH || KIND == G_UPQ) {
         // A tile = 128 gathered rows x 128 bytes of K; this thread: lines
@@ -1159,11 +1231,24 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         // index load does not sit in front of every k-block's copies.
         constexpr int nbox = (KIND == G_DW1) ? 2 : BN / 64;
         int tk[3][4];
+        if (t.krow0 == first_krow0 && t.nkb == first_nkb) {
+          // same expert as this warp's previous tile (an expert has many
+          // tiles): its first two k-blocks' row tokens are already known
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+          for (int q = 0; q < 2; ++q)
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tk[q + 1][j] = q < t.nkb ? gather_tok<KIND>(p, t.krow0 + q * kBK + line0 + 16 * j) : -1;
+            for (int j = 0; j < 4; ++j) tk[q + 1][j] = first_tk[q][j];
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tk[q + 1][j] = q < t.nkb ? gather_tok<KIND>(p, t.krow0 + q * kBK + line0 + 16 * j) : -1;
+              first_tk[q][j] = tk[q + 1][j];
+            }
+          first_krow0 = t.krow0;
+          first_nkb = t.nkb;
+        }
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % GS;
 #pragma unroll

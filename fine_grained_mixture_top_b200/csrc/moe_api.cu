@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -112,6 +113,7 @@ struct Plan {
   int nds;  // dS partials per row: N tiles x column parts of the dH epilogue
   int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
   int epi_dw;           // epilogue warps of the weight-gradient kernels
+  int dw_dual;          // weight-gradient tiles claimed from both ends of the expert order
   int ksplit, ksplit_rows;
 };
 
@@ -159,6 +161,13 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   // expert (at most 8 k-blocks on average) a tile is bound by storing its
   // 128 x BN result, so the epilogue gets 8 warps.
   p.epi_dw = (T * K / E <= 8 * 64) ? 8 : 4;
+  p.dw_dual = 1;
+  // tuning overrides, for measurements: MOE_EPI_DW (4 or 8), MOE_DW_DUAL (0 or 1)
+  if (const char* v = std::getenv("MOE_EPI_DW")) {
+    const int x = std::atoi(v);
+    if (x == 4 || x == 8) p.epi_dw = x;
+  }
+  if (const char* v = std::getenv("MOE_DW_DUAL")) p.dw_dual = std::atoi(v) != 0;
   p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
@@ -388,11 +397,12 @@ inline int grid_for(int64_t max_tiles, int sms) { return (int)std::max<int64_t>(
 
 // The last CUDA runtime error a call returned, with the source line that saw
 // it (read back through moe_last_error).
-thread_local char g_last_error[256] = "";
+thread_local char g_last_error[512] = "";
 
 moe_status cuda_failed(cudaError_t e, int line) {
-  std::snprintf(g_last_error, sizeof(g_last_error), "%s (%s) at moe_api.cu:%d", cudaGetErrorName(e),
-                cudaGetErrorString(e), line);
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s (%s) at moe_api.cu:%d%s%s", cudaGetErrorName(e),
+                cudaGetErrorString(e), line, g_launch_diag[0] ? "; " : "", g_launch_diag);
+  g_launch_diag[0] = 0;
   return MOE_ERR_CUDA;
 }
 
@@ -839,7 +849,8 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.num_m_tiles = (int)cdiv(p.n, 128);
     g.num_n_tiles = p.d / p.bn_dw2;
     g.out0 = static_cast<__nv_bfloat16*>(dW2);
-    g.sched = w.sched + 0;
+    g.sched = w.sched + 0;  // 64-bit tile counter (front and back claims)
+    g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
@@ -856,7 +867,8 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.num_m_tiles = (int)cdiv(p.d, 128);
     g.num_n_tiles = 2 * p.n / p.bn_dw1;
     g.out0 = static_cast<__nv_bfloat16*>(dW1);
-    g.sched = w.sched + 1;
+    g.sched = w.sched + 2;  // a 64-bit counter of its own
+    g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");

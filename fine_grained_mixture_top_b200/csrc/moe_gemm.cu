@@ -1,6 +1,7 @@
 // Instantiations and launcher of the tcgen05 grouped GEMM (see gemm.cuh).
 #include <cuda_runtime.h>
 
+#include <cstdio>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -10,6 +11,8 @@
 
 namespace moe {
 
+thread_local char g_launch_diag[256] = "";
+
 template <int KIND, int BN, int EPI>
 static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream) {
   using EC = EpiCfg<KIND, EPI>;
@@ -17,9 +20,18 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
   constexpr int threads = EC::kThreads;
   auto fn = moe_gemm_kernel<KIND, BN, EPI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
-  if (e != cudaSuccess) return e;
-  if (grid <= 0) return cudaSuccess;
-  return launch_pdl(fn, dim3(grid), dim3(threads), (size_t)smem, stream, p);
+  if (e == cudaSuccess && grid > 0) e = launch_pdl(fn, dim3(grid), dim3(threads), (size_t)smem, stream, p);
+  if (e != cudaSuccess) {
+    // what the launch asked for against what the compiled kernel allows
+    cudaFuncAttributes fa = {};
+    cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(fn));
+    std::snprintf(g_launch_diag, sizeof(g_launch_diag),
+                  "gemm kind %d BN %d epilogue warps %d: grid %d x %d threads, %d B dynamic smem; kernel: %d regs, "
+                  "max %d threads, max dynamic smem %d B",
+                  KIND, BN, EPI, grid, threads, smem, fa.numRegs, fa.maxThreadsPerBlock,
+                  fa.maxDynamicSharedSizeBytes);
+  }
+  return e;
 }
 
 // The dynamic shared-memory limit is a per-device property of a function: it

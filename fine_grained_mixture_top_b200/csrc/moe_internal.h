@@ -45,6 +45,10 @@ cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
 // records per CTA and role.
 void set_gemm_trace(int kind, void* buf, int cap);
 
+// The calling thread's last failed GEMM launch: what it asked for and what
+// the kernel allows (empty if none failed).
+extern thread_local char g_launch_diag[256];
+
 // epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
 
