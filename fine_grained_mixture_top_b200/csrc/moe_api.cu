@@ -114,6 +114,7 @@ struct Plan {
   int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
   int epi_dw;           // epilogue warps of the weight-gradient kernels
   int dw_dual;          // weight-gradient tiles claimed from both ends of the expert order
+  int dw1_pair, dw2_pair;  // weight-gradient GEMMs on CTA pairs (256 x 256 tiles)
   int ksplit, ksplit_rows;
 };
 
@@ -168,6 +169,11 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
     if (x == 4 || x == 8) p.epi_dw = x;
   }
   if (const char* v = std::getenv("MOE_DW_DUAL")) p.dw_dual = std::atoi(v) != 0;
+  // 256 x 256 pair tiles where both output dimensions are multiples of 256
+  // (MOE_DW_PAIR=1 turns them on)
+  const bool pair_on = std::getenv("MOE_DW_PAIR") && std::atoi(std::getenv("MOE_DW_PAIR")) != 0;
+  p.dw1_pair = pair_on && (d % 256 == 0) && ((2 * n) % 256 == 0);
+  p.dw2_pair = pair_on && (d % 256 == 0) && (n % 256 == 0);
   p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
@@ -854,8 +860,15 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, p.epi_dw, g,
-                             grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+    if (p.dw2_pair) {
+      g.num_m_tiles = p.n / 256;
+      g.num_n_tiles = p.d / 256;
+      MOE_TRY_CUDA(launch_gemm_pair(G_DW2, p.epi_dw, g,
+                                    grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms / 2), st));
+    } else {
+      MOE_TRY_CUDA(launch_gemm(G_DW2, p.bn_dw2, p.epi_dw, g,
+                               grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+    }
   }
   record_ready(grad_ready, 0, st);  // dW2 final
   // dW1[e] = X[tok]^T dH
@@ -872,8 +885,15 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.expert_order = w.expert_order;
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, p.epi_dw, g,
-                             grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+    if (p.dw1_pair) {
+      g.num_m_tiles = p.d / 256;
+      g.num_n_tiles = 2 * p.n / 256;
+      MOE_TRY_CUDA(launch_gemm_pair(G_DW1, p.epi_dw, g,
+                                    grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms / 2), st));
+    } else {
+      MOE_TRY_CUDA(launch_gemm(G_DW1, p.bn_dw1, p.epi_dw, g,
+                               grid_for((int64_t)p.E * g.num_m_tiles * g.num_n_tiles, sms), st));
+    }
   }
   record_ready(grad_ready, 1, st);  // dW1 final
   // dX~ = dH W1[e]^T

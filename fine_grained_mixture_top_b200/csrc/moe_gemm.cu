@@ -7,6 +7,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -29,6 +30,26 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
                   "gemm kind %d BN %d epilogue warps %d: grid %d x %d threads, %d B dynamic smem; kernel: %d regs, "
                   "max %d threads, max dynamic smem %d B",
                   KIND, BN, EPI, grid, threads, smem, fa.numRegs, fa.maxThreadsPerBlock,
+                  fa.maxDynamicSharedSizeBytes);
+  }
+  return e;
+}
+
+template <int KIND, int EPI>
+static cudaError_t launch_pair_one(const GemmParams& p, int pairs, cudaStream_t stream) {
+  using SH = PairShape<KIND, EPI>;
+  constexpr int smem = SH::kSmemBytes;
+  auto fn = moe_dw_pair_kernel<KIND, EPI>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
+  if (e == cudaSuccess && pairs > 0)
+    e = launch_pdl(fn, dim3(2 * pairs), dim3(SH::kThreads), (size_t)smem, stream, p);
+  if (e != cudaSuccess) {
+    cudaFuncAttributes fa = {};
+    cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(fn));
+    std::snprintf(g_launch_diag, sizeof(g_launch_diag),
+                  "pair gemm kind %d epilogue warps %d: %d pairs x %d threads, %d B dynamic smem; kernel: %d regs, "
+                  "max %d threads, max dynamic smem %d B",
+                  KIND, EPI, pairs, SH::kThreads, smem, fa.numRegs, fa.maxThreadsPerBlock,
                   fa.maxDynamicSharedSizeBytes);
   }
   return e;
@@ -106,6 +127,22 @@ cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p_in, int g
   MOE_CASE(G_RTR, 192, 4)
   MOE_CASE(G_DWR, 128, 4)
 #undef MOE_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_pair(int kind, int epi, const GemmParams& p_in, int pairs, cudaStream_t s) {
+  GemmParams p = p_in;
+  {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (kind == g_trace_kind) {
+      p.trace = g_trace_buf;
+      p.trace_cap = g_trace_cap;
+    }
+  }
+  if (kind == G_DW1 && epi == 4) return launch_pair_one<G_DW1, 4>(p, pairs, s);
+  if (kind == G_DW1 && epi == 8) return launch_pair_one<G_DW1, 8>(p, pairs, s);
+  if (kind == G_DW2 && epi == 4) return launch_pair_one<G_DW2, 4>(p, pairs, s);
+  if (kind == G_DW2 && epi == 8) return launch_pair_one<G_DW2, 8>(p, pairs, s);
   return cudaErrorInvalidValue;
 }
 

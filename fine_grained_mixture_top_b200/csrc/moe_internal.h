@@ -51,6 +51,9 @@ extern thread_local char g_launch_diag[256];
 
 // epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
 cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
+// Weight-gradient kinds on CTA pairs (256 x 256 tiles, gemm_pair.cuh):
+// p.num_m_tiles / p.num_n_tiles count 256-wide tiles; `pairs` clusters of 2.
+cudaError_t launch_gemm_pair(int kind, int epi, const GemmParams& p, int pairs, cudaStream_t s);
 
 // Per-kernel timing (moe_profile_enable): while on, each launch site brackets
 // its kernel with two CUDA events recorded on the launching stream.
