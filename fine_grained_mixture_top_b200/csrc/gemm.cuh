@@ -113,6 +113,16 @@ struct KindTraits {
   static constexpr bool kBMN = !(KIND == G_DH || KIND == G_DXT || KIND == G_UPQ || KIND == G_DOWNQ);
 };
 
+// Registers per thread at which a block of `threads` still launches: the
+// register file is split over the SM's four sub-partitions (16384 each) and
+// a block's warps are spread over them, so the sub-partition with the most
+// warps, ceil(warps / 4), bounds the count (allocated in multiples of 8 per
+// thread, at most 255): 128 for 14 warps, 168 for 10 or 12, 255 for 6.
+__host__ __device__ constexpr int max_regs_for(int threads) {
+  return ((16384 / (32 * ((threads / 32 + 3) / 4))) & ~7) > 255 ? 255
+                                                                : ((16384 / (32 * ((threads / 32 + 3) / 4))) & ~7);
+}
+
 // Epilogue configuration: EPI = 4 or 8 epilogue warps.  With 8, two warps
 // share each TMEM lane quarter and each takes half of the tile's columns;
 // that pays where the epilogue, not the main loop, bounds a tile (the dH
@@ -131,10 +141,7 @@ struct EpiCfg {
                                    ? 3
                                    : (EPI == 8 ? (KindTraits<KIND>::kGroupedK ? 4 : 2) : 3);
   static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
-  // registers per thread for one resident block (multiple of 8, at most 255);
-  // 448-thread blocks stay under 61440 registers
-  static constexpr int kMaxRegRaw = (kThreads > 320 ? 61440 / kThreads : 65536 / kThreads) & ~7;
-  static constexpr int kMaxReg = kMaxRegRaw > 255 ? 255 : kMaxRegRaw;
+  static constexpr int kMaxReg = max_regs_for(kThreads);
 };
 
 constexpr int kBM = 128;

@@ -19,7 +19,8 @@
 //   warp 0 lane 0   TMA loads of this CTA's half of the TMA operand; in the
 //                   first CTA also the tile claims (one queue for the pair)
 //   warp 1          TMEM allocation (both CTAs); MMA issue (first CTA only)
-//   warps 2..2+EPI  epilogue: this CTA's 128 accumulator rows
+//   warps 2..2+EPI  epilogue: this CTA's 128 accumulator rows (p.tmC1: a store
+//                   map of 32-row x 64-column boxes with the 128-byte swizzle)
 //   last 4 warps    cp.async gather of this CTA's half of the gathered operand
 // Barriers that pair members arrive on remotely live in the first CTA:
 //   full[s]      TMA bytes of both CTAs + 4 gather warps of each CTA
@@ -40,8 +41,12 @@ struct PairShape {
   static constexpr int kABytes = kHalf * kBK * 2;    // 16 KB: two 64 x 64 MN-major boxes
   static constexpr int kBBytes = kHalf * kBK * 2;    // 16 KB
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kBufs = EPI == 8 ? 4 : 3;     // 2 KB epilogue staging buffers per warp
-  static constexpr int kStoreBytes = EPI * kBufs * kStoreBuf;
+  // Epilogue staging: per warp, kBufs boxes of 32 rows x 64 columns (4 KB,
+  // 128-byte swizzle), each leaving as one TMA store of whole 128-byte row
+  // segments (a 32-column box writes half-lines, twice the store requests).
+  static constexpr int kBoxBytesOut = 32 * 64 * 2;
+  static constexpr int kBufs = 2;
+  static constexpr int kStoreBytes = EPI * kBufs * kBoxBytesOut;
   static constexpr int kBudget = (kSmemLimit - 2048 - kStoreBytes) < 200 * 1024 ? (kSmemLimit - 2048 - kStoreBytes)
                                                                                    : 200 * 1024;
   static constexpr int kStagesRaw = kBudget / kStage;
@@ -52,8 +57,7 @@ struct PairShape {
   static constexpr int kBarOffset = kStoreOffset + kStoreBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;
   static constexpr int kThreads = 32 * (2 + EPI + 4);
-  static constexpr int kMaxRegRaw = (kThreads > 320 ? 61440 / kThreads : 65536 / kThreads) & ~7;
-  static constexpr int kMaxReg = kMaxRegRaw > 255 ? 255 : kMaxRegRaw;
+  static constexpr int kMaxReg = max_regs_for(kThreads);
   static_assert(kStages >= 3, "pair ring depth");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
@@ -302,7 +306,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     const int ew = warp - 2;
     const int part = ew >> 2;  // column part of this warp (kColSplit parts)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-    const uint32_t stg = base + SH::kStoreOffset + ew * (kBufs * kStoreBuf);
+    const uint32_t stg = base + SH::kStoreOffset + ew * (kBufs * SH::kBoxBytesOut);
     const int M = (KIND == G_DW1) ? p.d : p.n;
     constexpr int kCols = 256 / kColSplit;
     int ring = 0, tcount = 0, ntr = 0;
@@ -321,15 +325,14 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
       const int orow = t.e * M + row0;
       const int c0 = part * kCols;
       if (t.nkb == 0) {  // expert without tokens: its weight gradient is zero
-        float z[32];
-        zero32(z);
-        const uint32_t buf = stg + ring * kStoreBuf;
+        const uint32_t buf = stg + ring * SH::kBoxBytesOut;
         stage_wait();
-        stage_row32(buf, lane, z);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_shared_v4(buf + sw128(lane, j), make_uint4(0u, 0u, 0u, 0u));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          for (int c = c0; c < c0 + kCols; c += 32) tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
+          for (int c = c0; c < c0 + kCols; c += 64) tma_store_2d(&p.tmC1, buf, t.n0 + c, orow);
           bulk_commit();
         }
         ring = ring + 1 == kBufs ? 0 : ring + 1;
@@ -342,20 +345,28 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
       if (tracer) trace_ev(p, 2, ntr, tile, 1);
       const uint32_t tacc = lane_addr + (uint32_t)(b * kAccStride);
 #pragma unroll 1
-      for (int c = c0; c < c0 + kCols; c += 32) {
-        uint32_t a[32];
+      for (int c = c0; c < c0 + kCols; c += 64) {
+        uint32_t a[32], a2[32];
         tmem_ld32(tacc + c, a);
+        tmem_ld32(tacc + c + 32, a2);
         tc_wait_ld();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
-        const uint32_t buf = stg + ring * kStoreBuf;
+        const uint32_t buf = stg + ring * SH::kBoxBytesOut;
         stage_wait();
-        stage_row32(buf, lane, v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float v[8], w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[i] = __uint_as_float(a[8 * j + i]);
+            w[i] = __uint_as_float(a2[8 * j + i]);
+          }
+          st_shared_v4(buf + sw128(lane, j), pack8f(v));
+          st_shared_v4(buf + sw128(lane, 4 + j), pack8f(w));
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
+          tma_store_2d(&p.tmC1, buf, t.n0 + c, orow);
           bulk_commit();
         }
         ring = ring + 1 == kBufs ? 0 : ring + 1;

@@ -861,6 +861,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
     if (p.dw2_pair) {
+      MOE_TRY_MAP(make_tmap(&g.tmC1, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 32));
       g.num_m_tiles = p.n / 256;
       g.num_n_tiles = p.d / 256;
       MOE_TRY_CUDA(launch_gemm_pair(G_DW2, p.epi_dw, g,
@@ -886,6 +887,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
     if (p.dw1_pair) {
+      MOE_TRY_MAP(make_tmap(&g.tmC1, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 32));
       g.num_m_tiles = p.d / 256;
       g.num_n_tiles = 2 * p.n / 256;
       MOE_TRY_CUDA(launch_gemm_pair(G_DW1, p.epi_dw, g,

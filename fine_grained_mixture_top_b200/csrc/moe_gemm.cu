@@ -23,6 +23,7 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
   if (e == cudaSuccess && grid > 0) e = launch_pdl(fn, dim3(grid), dim3(threads), (size_t)smem, stream, p);
   if (e != cudaSuccess) {
+    cudaGetLastError();  // the error is returned here; do not leave it for a later call to find
     // what the launch asked for against what the compiled kernel allows
     cudaFuncAttributes fa = {};
     cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(fn));
@@ -44,6 +45,7 @@ static cudaError_t launch_pair_one(const GemmParams& p, int pairs, cudaStream_t 
   if (e == cudaSuccess && pairs > 0)
     e = launch_pdl(fn, dim3(2 * pairs), dim3(SH::kThreads), (size_t)smem, stream, p);
   if (e != cudaSuccess) {
+    cudaGetLastError();  // the error is returned here; do not leave it for a later call to find
     cudaFuncAttributes fa = {};
     cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(fn));
     std::snprintf(g_launch_diag, sizeof(g_launch_diag),
