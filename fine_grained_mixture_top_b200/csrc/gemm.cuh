@@ -137,9 +137,16 @@ struct EpiCfg {
   // dX~ kernel keeps 2 (so that its stage ring keeps its depth), while the
   // weight-gradient kinds, which get 8 warps when their tiles are store-bound
   // (few rows per expert), keep 4 bulk stores in flight per warp.
+  // One-output kinds (down-proj, dX~, dW1, dW2) stage 32 rows x 64 columns
+  // per buffer (4 KB, 128-byte swizzle) so that each TMA store writes whole
+  // 128-byte row segments: a 32-column box writes half-lines, twice the store
+  // requests, and the per-SM store path then bounds store-heavy tiles.  They
+  // keep 2 such buffers per warp.
+  static constexpr bool kWide = (KIND == G_DOWN || KIND == G_DXT || KindTraits<KIND>::kGroupedK);
   static constexpr int kBufs = (KIND == G_UP || KIND == G_DH || KIND == G_UPQ)
                                    ? 3
-                                   : (EPI == 8 ? (KindTraits<KIND>::kGroupedK ? 4 : 2) : 3);
+                                   : (kWide ? 2 : (EPI == 8 ? 2 : 3));
+  static constexpr int kBufBytes = kWide ? 4096 : 2048;
   static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
   static constexpr int kMaxReg = max_regs_for(kThreads);
 };
@@ -453,7 +460,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     moe_gemm_kernel(const __grid_constant__ GemmParams p) {
   using KT = KindTraits<KIND>;
   using EC = EpiCfg<KIND, EPI>;
-  using SH = GemmShape<KIND, BN, EPI * EC::kBufs>;
+  using SH = GemmShape<KIND, BN, EPI * EC::kBufs * (EC::kBufBytes / kStoreBuf)>;
   constexpr int kEpiEnd = 2 + EPI;  // epilogue warps are [2, kEpiEnd)
   constexpr bool kSplit = SH::kSplit;  // separate A and B rings
   constexpr int SA = SH::kSA;      // A ring slots
@@ -857,7 +864,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     const int half = ew >> 2;  // column part of this warp (EC::kColSplit parts)
     const int rloc = q * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-    const uint32_t stg = base + SH::kStoreOffset + ew * (EC::kBufs * kStoreBuf);
+    const uint32_t stg = base + SH::kStoreOffset + ew * (EC::kBufs * EC::kBufBytes);
     int ring = 0;  // next staging buffer for one-output kinds
     // Make staging buffer(s) free: `pending` store groups may still be reading.
     auto stage_wait = [&](auto pending_tag) {
@@ -884,15 +891,14 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           // warp's rows as one bulk group
           const int M = (KIND == G_DW1) ? p.d : p.n;
           if (row0 < M) {
-            float z[32];
-            zero32(z);
-            const uint32_t buf = stg + ring * kStoreBuf;
+            const uint32_t buf = stg + ring * EC::kBufBytes;
             stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
-            stage_row32(buf, lane, z);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_shared_v4(buf + sw128(lane, j), make_uint4(0u, 0u, 0u, 0u));
             stage_publish();
             if (lane == 0) {
               constexpr int kC = BN / EC::kColSplit;
-              for (int c = half * kC; c < half * kC + kC; c += 32) tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
+              for (int c = half * kC; c < half * kC + kC; c += 64) tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
               bulk_commit();
             }
             ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
@@ -926,14 +932,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       // (the same for every row of the tile) while the MMAs run
       float rz = 0.f;
       const float4* rv = nullptr;
-      float4 r_nx[8];
       if constexpr (KIND == G_DXT) {
         if (p.rvec) {
           const int r = t.m0 + rloc;
           rz = __ldg(p.row_tok + r) >= 0 ? __ldg(p.rscale + r) : 0.f;
           rv = reinterpret_cast<const float4*>(p.rvec + (size_t)t.e * p.d + t.n0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) r_nx[i] = __ldg(rv + half * kCols / 4 + i);
         }
       }
       const int b = tcount & 1;
@@ -1019,7 +1022,27 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         }
         *reinterpret_cast<uint16_t*>(p.sa_out + ((size_t)t.mt * (p.n / 128) + t.n0 / 128) * 512 +
                                      16 * (rloc & 31) + 4 * (rloc >> 5) + (t.n0 % 128) / 32) = (uint16_t)sc2;
-      } else if constexpr (KIND == G_DOWN || KIND == G_DXT || KIND == G_DOWNQ || KT::kGroupedK) {
+      } else if constexpr (KIND == G_DOWNQ) {
+        const int c0 = half * kCols;
+#pragma unroll 1
+        for (int c = c0; c < c0 + kCols; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(tacc + c, a);
+          tc_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+          const uint32_t buf = stg + ring * EC::kBufBytes;
+          stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
+          stage_row32(buf, lane, v);
+          stage_publish();
+          if (lane == 0) {
+            tma_store_2d(&p.tmC0, buf, t.n0 + c, row0);
+            bulk_commit();
+          }
+          ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
+        }
+      } else if constexpr (KIND == G_DOWN || KIND == G_DXT || KT::kGroupedK) {
         int orow = row0;
         bool live = true;
         if constexpr (KT::kGroupedK) {
@@ -1028,41 +1051,44 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           orow = t.e * M + row0;
         }
         const int c0 = half * kCols;  // this warp's columns: [c0, c0 + kCols)
+        static_assert(!EC::kWide || (BN / EC::kColSplit) % 64 == 0, "64-column store chunks");
 #pragma unroll 1
-        for (int c = c0; c < c0 + kCols; c += 32) {
-          uint32_t a[32];
+        for (int c = c0; c < c0 + kCols; c += 64) {
+          uint32_t a[32], a2[32];
           tmem_ld32(tacc + c, a);
-          float4 r_cur[8];
+          tmem_ld32(tacc + c + 32, a2);
+          float4 r_cur[16];
           if constexpr (KIND == G_DXT) {
-            if (rv) {  // router path: this chunk's Wr^T values; prefetch the next chunk's
+            if (rv) {  // router path: this chunk's Wr^T values (the same for every row), loaded
+                       // while the accumulator loads are in flight
 #pragma unroll
-              for (int i = 0; i < 8; ++i) r_cur[i] = r_nx[i];
-              if (c + 32 < c0 + kCols) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) r_nx[i] = __ldg(rv + (c + 32) / 4 + i);
-              }
+              for (int i = 0; i < 16; ++i) r_cur[i] = __ldg(rv + c / 4 + i);
             }
           }
           tc_wait_ld();
           if (live) {
-            float v[32];
+            const uint32_t buf = stg + ring * EC::kBufBytes;
+            stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
-            if constexpr (KIND == G_DXT) {
-              if (rv) {  // + dz_r * Wr[n0 + c + j, e]
+            for (int j = 0; j < 8; ++j) {  // 8 columns per 16-byte chunk of the 128-byte row
+              float v[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 w = r_cur[i];
-                  v[4 * i + 0] = fmaf(rz, w.x, v[4 * i + 0]);
-                  v[4 * i + 1] = fmaf(rz, w.y, v[4 * i + 1]);
-                  v[4 * i + 2] = fmaf(rz, w.z, v[4 * i + 2]);
-                  v[4 * i + 3] = fmaf(rz, w.w, v[4 * i + 3]);
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(j < 4 ? a[8 * j + i] : a2[8 * (j - 4) + i]);
+              if constexpr (KIND == G_DXT) {
+                if (rv) {  // + dz_r * Wr[n0 + c + 8 j + i, e]
+                  const float4 w0 = r_cur[2 * j], w1 = r_cur[2 * j + 1];
+                  v[0] = fmaf(rz, w0.x, v[0]);
+                  v[1] = fmaf(rz, w0.y, v[1]);
+                  v[2] = fmaf(rz, w0.z, v[2]);
+                  v[3] = fmaf(rz, w0.w, v[3]);
+                  v[4] = fmaf(rz, w1.x, v[4]);
+                  v[5] = fmaf(rz, w1.y, v[5]);
+                  v[6] = fmaf(rz, w1.z, v[6]);
+                  v[7] = fmaf(rz, w1.w, v[7]);
                 }
               }
+              st_shared_v4(buf + sw128(lane, j), pack8f(v));
             }
-            const uint32_t buf = stg + ring * kStoreBuf;
-            stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
-            stage_row32(buf, lane, v);
             stage_publish();
             if (lane == 0) {
               tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);

@@ -18,12 +18,20 @@
 // Roles (both CTAs, same warp layout as moe_gemm_kernel):
 //   warp 0 lane 0   TMA loads of this CTA's half of the TMA operand; in the
 //                   first CTA also the tile claims (one queue for the pair)
-//   warp 1          TMEM allocation (both CTAs); MMA issue (first CTA only)
+//   warp 1          TMEM allocation (both CTAs); MMA issue (first CTA); in
+//                   the second CTA, lane 0 forwards each stage once it is
+//                   complete there to the first CTA's full barrier
 //   warps 2..2+EPI  epilogue: this CTA's 128 accumulator rows (p.tmC1: a store
 //                   map of 32-row x 64-column boxes with the 128-byte swizzle)
 //   last 4 warps    cp.async gather of this CTA's half of the gathered operand
+// Each CTA fills its own stage and completes its own full[s] (its TMA bytes +
+// its 128 gather threads, as in moe_gemm_kernel).  The forwarding thread has
+// no copies in flight, so its cluster-scope release (which waits for the
+// issuing thread's outstanding memory operations) costs nothing; a gather
+// thread releasing at cluster scope itself would wait for its next k-block's
+// copies each time and serialise the copy pipeline.
 // Barriers that pair members arrive on remotely live in the first CTA:
-//   full[s]      TMA bytes of both CTAs + 4 gather warps of each CTA
+//   full[s]      (also) the second CTA's forwarded stage
 //   acc_empty[b] the epilogue warps of both CTAs
 //   tq_empty[q]  every queue consumer of both CTAs
 // Barriers the first CTA's MMA thread completes in both CTAs (two commits):
@@ -103,14 +111,16 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // queue consumers per CTA: the first CTA's MMA warp or the second CTA's
-  // producer warp, the epilogue warps and the gather warps
-  constexpr int kQConsumers = 1 + EPI + 4;
+  // queue consumers: the first CTA's MMA warp, epilogue and gather warps; the
+  // second CTA's producer, forwarder, epilogue and gather warps
+  constexpr int kQConsumers = (1 + EPI + 4) + (2 + EPI + 4);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1 + 2 * 4);  // first CTA's producer (expect_tx) + 4 gather warps per CTA
-      mbar_init(&empty[s], 1);         // the MMA commit
+      // own producer (expect_tx of own TMA bytes) + 128 own gather threads,
+      // + in the first CTA the second CTA's forwarded stage
+      mbar_init(&full[s], 1 + 128 + (lead ? 1 : 0));
+      mbar_init(&empty[s], 1);  // the MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -118,7 +128,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     }
     for (int b = 0; b < kTileQ; ++b) {
       mbar_init(&tq_full[b], 1);
-      mbar_init(&tq_empty[b], 2 * kQConsumers);
+      mbar_init(&tq_empty[b], kQConsumers);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -171,7 +181,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     }
     const int4 q = tq_info[slot];
     if (whole_warp) __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(lead_bar(&tq_empty[slot]));
+    if (lane == 0) mbar_arrive_remote(lead_bar(&tq_empty[slot]));
     if (q.x < num_tiles) t = decode(q.x, q.y, q.z, q.w);
     return q.x;
   };
@@ -233,24 +243,45 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
         trace_ev(p, 0, ntr, tile, 0);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait_cl(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
+          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
             ok = false;
             break;
           }
-          const uint32_t fb = lead ? smem_u32(&full[s]) : lead_bar(&full[s]);
-          if (lead) mbar_arrive_expect_tx(fb, 2u * (uint32_t)tma_step);  // both CTAs' TMA bytes
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, (uint32_t)tma_step);  // this CTA's TMA bytes
           const uint32_t dst = tma_dst0 + (uint32_t)s * tma_step;
           const int krow = t.krow0 + kb * kBK;
           const int col = ((KIND == G_DW2) ? t.m0 : t.n0) + half0;
-          tma_load_2d_pair(dst, tm, fb, col, krow);
-          tma_load_2d_pair(dst + kBoxBytes, tm, fb, col + 64, krow);
+          tma_load_2d(dst, tm, fb, col, krow);
+          tma_load_2d(dst + kBoxBytes, tm, fb, col + 64, krow);
         }
         trace_ev(p, 0, ntr, tile, 1);
       }
     }
+  } else if (warp == 1 && !lead) {
+    // ---------------- forwarder (second CTA): each stage, once complete here
+    // (this CTA's TMA bytes and gather copies), is signalled on the first
+    // CTA's full barrier
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int ti = 0; ok; ++ti) {
+        TileInfo t;
+        const int tile = consume_tile(ti, ok, t, false);
+        if (!ok || tile >= num_tiles) break;
+        for (int kb = 0; kb < t.nkb; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 14)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_cluster(lead_bar(&full[s]));
+        }
+      }
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer (first CTA only)
-    if (lead) {
+    {
       int it = 0, tcount = 0, ntr = 0;
       bool ok = true;
       for (int ti = 0; ok; ++ti) {
@@ -340,7 +371,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
       }
       const int b = tcount & 1;
       const int use = tcount >> 1;
-      if (!mbar_wait_cl(smem_u32(&acc_full[b]), use & 1, abort_flag, p.st, KIND * 16 + 4)) break;
+      if (!mbar_wait(smem_u32(&acc_full[b]), use & 1, abort_flag, p.st, KIND * 16 + 4)) break;
       tc_fence_after();
       if (tracer) trace_ev(p, 2, ntr, tile, 1);
       const uint32_t tacc = lane_addr + (uint32_t)(b * kAccStride);
@@ -373,7 +404,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_bar(&acc_empty[b]));
+      if (lane == 0) mbar_arrive_remote(lead_bar(&acc_empty[b]));
       if (tracer) trace_ev(p, 2, ntr, tile, 2);
       ++tcount;
     }
@@ -382,8 +413,8 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     // ---------------- gather warps: this CTA's half of the gathered operand
     // (DW1: A = X columns [m0 + half0, +128); DW2: B = dO columns
     // [n0 + half0, +128)) for 64 routed rows per k-block, cp.async into the
-    // 128B-swizzled MN-major layout TMA would produce; each warp publishes its
-    // k-blocks on the first CTA's full barrier one k-block after issuing them.
+    // 128B-swizzled MN-major layout TMA would produce; each thread publishes
+    // its k-blocks on this CTA's full barrier one k-block after issuing them.
     const int gt = threadIdx.x - 32 * kEpiEnd;  // 0..127
     const int chunk = gt & 7;
     const int line0 = gt >> 3;  // 0..15
@@ -392,10 +423,9 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     bool ok = true;
     int first_tk[2][4];
     int first_krow0 = -1, first_nkb = -1;
-    auto publish = [&](int k_it) {  // k-block k_it of this warp's copies is complete
+    auto publish = [&](int k_it) {  // k-block k_it of this thread's copies is complete
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_bar(&full[k_it % S]));
+      mbar_arrive(smem_u32(&full[k_it % S]));
     };
     for (int ti = 0; ok; ++ti) {
       TileInfo t;
@@ -431,7 +461,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
 #pragma unroll
           for (int j = 0; j < 4; ++j) tk[2][j] = gather_tok<KIND>(p, t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
         }
-        if (!mbar_wait_cl(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
+        if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
           ok = false;
           break;
         }

@@ -102,6 +102,11 @@ bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
 bool make_store_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   return make_tmap(m, base, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
+// Store map of the one-output epilogues: 32-row x 64-column boxes, 128-byte
+// swizzle (whole 128-byte row segments per store).
+bool make_store_map_wide(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  return make_tmap(m, base, rows, cols, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
 // ----------------------------------------------------------------- shapes
 struct Plan {
@@ -583,7 +588,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     MOE_TRY_MAP(make_tmap(&g.tmB, W2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 64));
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
-    MOE_TRY_MAP(make_store_map(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
+    MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "down_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -858,7 +863,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.sched = w.sched + 0;  // 64-bit tile counter (front and back claims)
     g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
-    MOE_TRY_MAP(make_store_map(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
+    MOE_TRY_MAP(make_store_map_wide(&g.tmC0, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d));
     ProfScope ps(st, "dw2_gemm");
     if (p.dw2_pair) {
       MOE_TRY_MAP(make_tmap(&g.tmC1, dW2, (uint64_t)p.E * p.n, (uint64_t)p.d, 64, 32));
@@ -884,7 +889,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.sched = w.sched + 2;  // a 64-bit counter of its own
     g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
-    MOE_TRY_MAP(make_store_map(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
+    MOE_TRY_MAP(make_store_map_wide(&g.tmC0, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n));
     ProfScope ps(st, "dw1_gemm");
     if (p.dw1_pair) {
       MOE_TRY_MAP(make_tmap(&g.tmC1, dW1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 32));
@@ -909,7 +914,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
       g.rvec = w.WrT;
       g.rscale = w.dz_row;
     }
-    MOE_TRY_MAP(make_store_map(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
+    MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "dxt_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }

@@ -76,9 +76,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 // Arrive on a barrier of any CTA of the cluster (a shared::cluster address),
-// releasing this thread's prior writes at cluster scope.
+// releasing this thread's prior writes at cluster scope.  The release waits
+// for the thread's own outstanding memory operations: a thread with cp.async
+// copies in flight should not issue it (see mbar_arrive_remote).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive on a barrier of any CTA of the cluster with the default (CTA-scope)
+// semantics: for "this slot / accumulator is free" signals, which publish no
+// data of their own.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
