@@ -147,6 +147,9 @@ struct EpiCfg {
                                    ? 3
                                    : (kWide ? 2 : (EPI == 8 ? 2 : 3));
   static constexpr int kBufBytes = kWide ? 4096 : 2048;
+  // staging of all epilogue warps in 2 KB units: the GemmShape NBUF that both
+  // the kernel's layout and its launch (the dynamic shared-memory size) use
+  static constexpr int kNbuf = EPI * kBufs * (kBufBytes / 2048);
   static constexpr int kThreads = 32 * (2 + EPI + (KindTraits<KIND>::kGather ? 4 : 0));
   static constexpr int kMaxReg = max_regs_for(kThreads);
 };
@@ -460,7 +463,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     moe_gemm_kernel(const __grid_constant__ GemmParams p) {
   using KT = KindTraits<KIND>;
   using EC = EpiCfg<KIND, EPI>;
-  using SH = GemmShape<KIND, BN, EPI * EC::kBufs * (EC::kBufBytes / kStoreBuf)>;
+  using SH = GemmShape<KIND, BN, EC::kNbuf>;
   constexpr int kEpiEnd = 2 + EPI;  // epilogue warps are [2, kEpiEnd)
   constexpr bool kSplit = SH::kSplit;  // separate A and B rings
   constexpr int SA = SH::kSA;      // A ring slots
@@ -469,6 +472,12 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   constexpr uint32_t kIdesc = idesc_bf16_f32(BN, KT::kAMN, KT::kBMN);
 
   extern __shared__ uint8_t smem_raw[];
+  // a launch with less shared memory than this layout needs stops here with
+  // a status instead of touching memory past its allocation
+  if (dynamic_smem_bytes() < (uint32_t)SH::kSmemBytes) {
+    if (threadIdx.x == 0) raise_status(p.st, ST_DEVICE_CHECK, 0x300 + KIND);
+    return;
+  }
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);

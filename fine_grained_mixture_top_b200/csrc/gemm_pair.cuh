@@ -84,6 +84,10 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
   constexpr int kTmemCols = 512;
 
   extern __shared__ uint8_t smem_raw[];
+  if (dynamic_smem_bytes() < (uint32_t)SH::kSmemBytes) {  // both CTAs of the pair leave alike
+    if (threadIdx.x == 0) raise_status(p.st, ST_DEVICE_CHECK, 0x300 + KIND);
+    return;
+  }
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);

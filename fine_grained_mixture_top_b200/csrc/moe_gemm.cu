@@ -17,7 +17,7 @@ thread_local char g_launch_diag[256] = "";
 template <int KIND, int BN, int EPI>
 static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream) {
   using EC = EpiCfg<KIND, EPI>;
-  constexpr int smem = GemmShape<KIND, BN, EPI * EC::kBufs>::kSmemBytes;
+  constexpr int smem = GemmShape<KIND, BN, EC::kNbuf>::kSmemBytes;  // the kernel's own layout
   constexpr int threads = EC::kThreads;
   auto fn = moe_gemm_kernel<KIND, BN, EPI>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);

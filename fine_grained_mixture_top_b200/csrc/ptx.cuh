@@ -22,6 +22,13 @@ __device__ __forceinline__ void raise_status(const DevStatus& s, int code, int w
   }
 }
 
+// Dynamic shared memory this block was launched with.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
