@@ -663,6 +663,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           issue_tma<KIND, BN>(p, t, kb, a_slot(sa), smem_u32(&full_a[sa]), b_slot(sb), smem_u32(&full_b[sb]),
                               base + SH::kSFAOffset + (uint32_t)(sa * SH::kSFABytes),
                               base + SH::kSFBOffset + (uint32_t)(sb * SH::kSFBBytes));
+          if (ti == 0) trace_ev(p, 0, ntr, kb, 16);  // first tile: each k-block's issue
         }
         trace_ev(p, 0, ntr, tile, 1);
       }
@@ -756,6 +757,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
         }
         tc_fence_after();
         if (kb == 0 && lane == 0) trace_ev(p, 1, ntr, tile, 2);
+        if (ti == 0 && lane == 0) trace_ev(p, 1, ntr, kb, 16);  // first tile: each k-block's operands ready
         if (lane == 0) {
           const uint32_t a_s = a_slot(sa);
           const uint32_t b_s = b_slot(sb);

@@ -258,6 +258,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
           const int col = ((KIND == G_DW2) ? t.m0 : t.n0) + half0;
           tma_load_2d(dst, tm, fb, col, krow);
           tma_load_2d(dst + kBoxBytes, tm, fb, col + 64, krow);
+          if (ti == 0) trace_ev(p, 0, ntr, kb, 16);  // first tile: each k-block's issue
         }
         trace_ev(p, 0, ntr, tile, 1);
       }
@@ -267,7 +268,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
     // (this CTA's TMA bytes and gather copies), is signalled on the first
     // CTA's full barrier
     if (lane == 0) {
-      int it = 0;
+      int it = 0, ntr = 0;
       bool ok = true;
       for (int ti = 0; ok; ++ti) {
         TileInfo t;
@@ -280,6 +281,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
             break;
           }
           mbar_arrive_cluster(lead_bar(&full[s]));
+          if (ti == 0) trace_ev(p, 1, ntr, kb, 16);  // first tile: stage complete here, forwarded
         }
       }
     }
@@ -311,6 +313,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
           }
           tc_fence_after();
           if (kb == 0 && lane == 0) trace_ev(p, 1, ntr, tile, 2);
+          if (ti == 0 && lane == 0) trace_ev(p, 1, ntr, kb, 16);  // first tile: each k-block's operands ready
           if (lane == 0) {
             const uint32_t a_s = a_slot(s);
             const uint32_t b_s = b_slot(s);
@@ -483,9 +486,11 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
           }
         }
         cp_async_commit();
+        if (ti == 0 && gt == 0) trace_ev(p, 3, ntr, kb, 16);  // first tile: each k-block's copies issued
         if (pending == kLag) {
           cp_async_wait<kLag>();
           publish(it - kLag);
+          if (ti == 0 && gt == 0) trace_ev(p, 3, ntr, kb - kLag, 17);  // ... and published
         } else {
           ++pending;
         }
