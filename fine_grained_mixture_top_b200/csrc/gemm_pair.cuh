@@ -70,7 +70,10 @@ struct PairShape {
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
 
-template <int KIND, int EPI>
+// POLL: the waits whose last arrival crosses the pair (the MMA's wait for a
+// forwarded stage, the second CTA's waits for the MMA's commits and the
+// forwarder's wait) poll instead of suspending.
+template <int KIND, int EPI, bool POLL>
 __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2, 1, 1)
     moe_dw_pair_kernel(const __grid_constant__ GemmParams p) {
   using SH = PairShape<KIND, EPI>;
@@ -115,6 +118,9 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  auto xwait = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+    return POLL ? mbar_poll(bar, parity, abort_flag, p.st, where) : mbar_wait(bar, parity, abort_flag, p.st, where);
+  };
   // queue consumers: the first CTA's MMA warp, epilogue and gather warps; the
   // second CTA's producer, forwarder, epilogue and gather warps
   constexpr int kQConsumers = (1 + EPI + 4) + (2 + EPI + 4);
@@ -247,7 +253,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
         trace_ev(p, 0, ntr, tile, 0);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 1)) {
+          if (!xwait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, KIND * 16 + 1)) {
             ok = false;
             break;
           }
@@ -276,7 +282,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
         if (!ok || tile >= num_tiles) break;
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 14)) {
+          if (!xwait(smem_u32(&full[s]), (it / S) & 1, KIND * 16 + 14)) {
             ok = false;
             break;
           }
@@ -307,7 +313,8 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
         const uint32_t d_tmem = tmem_base + (uint32_t)(b * kAccStride);
         for (int kb = 0; kb < t.nkb; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait_cl(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)) {
+          if (!(POLL ? mbar_poll(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3)
+                     : mbar_wait_cl(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.st, KIND * 16 + 3))) {
             ok = false;
             break;
           }
@@ -468,7 +475,7 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
 #pragma unroll
           for (int j = 0; j < 4; ++j) tk[2][j] = gather_tok<KIND>(p, t.krow0 + (kb + 2) * kBK + line0 + 16 * j);
         }
-        if (!mbar_wait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, abort_flag, p.st, KIND * 16 + 6)) {
+        if (!xwait(smem_u32(&empty[s]), ((it / S) & 1) ^ 1, KIND * 16 + 6)) {
           ok = false;
           break;
         }

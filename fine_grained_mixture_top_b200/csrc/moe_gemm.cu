@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -36,11 +37,11 @@ static cudaError_t launch_one(const GemmParams& p, int grid, cudaStream_t stream
   return e;
 }
 
-template <int KIND, int EPI>
+template <int KIND, int EPI, bool POLL>
 static cudaError_t launch_pair_one(const GemmParams& p, int pairs, cudaStream_t stream) {
   using SH = PairShape<KIND, EPI>;
   constexpr int smem = SH::kSmemBytes;
-  auto fn = moe_dw_pair_kernel<KIND, EPI>;
+  auto fn = moe_dw_pair_kernel<KIND, EPI, POLL>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
   if (e == cudaSuccess && pairs > 0)
     e = launch_pdl(fn, dim3(2 * pairs), dim3(SH::kThreads), (size_t)smem, stream, p);
@@ -141,10 +142,11 @@ cudaError_t launch_gemm_pair(int kind, int epi, const GemmParams& p_in, int pair
       p.trace_cap = g_trace_cap;
     }
   }
-  if (kind == G_DW1 && epi == 4) return launch_pair_one<G_DW1, 4>(p, pairs, s);
-  if (kind == G_DW1 && epi == 8) return launch_pair_one<G_DW1, 8>(p, pairs, s);
-  if (kind == G_DW2 && epi == 4) return launch_pair_one<G_DW2, 4>(p, pairs, s);
-  if (kind == G_DW2 && epi == 8) return launch_pair_one<G_DW2, 8>(p, pairs, s);
+  static const bool poll = std::getenv("MOE_PAIR_POLL") && std::atoi(std::getenv("MOE_PAIR_POLL")) != 0;
+  if (kind == G_DW1 && epi == 4) return poll ? launch_pair_one<G_DW1, 4, true>(p, pairs, s) : launch_pair_one<G_DW1, 4, false>(p, pairs, s);
+  if (kind == G_DW1 && epi == 8) return poll ? launch_pair_one<G_DW1, 8, true>(p, pairs, s) : launch_pair_one<G_DW1, 8, false>(p, pairs, s);
+  if (kind == G_DW2 && epi == 4) return poll ? launch_pair_one<G_DW2, 4, true>(p, pairs, s) : launch_pair_one<G_DW2, 4, false>(p, pairs, s);
+  if (kind == G_DW2 && epi == 8) return poll ? launch_pair_one<G_DW2, 8, true>(p, pairs, s) : launch_pair_one<G_DW2, 8, false>(p, pairs, s);
   return cudaErrorInvalidValue;
 }
 
