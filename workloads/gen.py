@@ -76,6 +76,10 @@ CONFIGS: dict[str, MoEConfig] = {
     "dsv3": MoEConfig("dsv3", T=8192, d=7168, E=256, n=2048, K=8, bias="zipf", seed=4),
     # OLMoE-shaped layer (the pages' runtime-breakdown workload), balanced router
     "olmoe": MoEConfig("olmoe", T=32768, d=2048, E=64, n=1024, K=8, seed=5),
+    # a small layer with the DeepSeek-V3-shaped layer's load pattern (many
+    # experts of a few dozen rows, a Zipf head), about 4 GB resident: for
+    # profiler captures of the weight-gradient kernels' short tiles
+    "smallexp": MoEConfig("smallexp", T=4096, d=2048, E=256, n=512, K=8, bias="zipf", seed=6),
 }
 for _i, (_E, _n) in enumerate([(64, 512), (128, 256), (256, 128), (512, 64)]):
     for _tr in (False, True):
