@@ -67,9 +67,6 @@ struct GemmParams {
   int* sched;                // weight-gradient kinds: zeroed 64-bit tile counter (8-byte aligned)
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
   int dual_ended;            // weight-gradient kinds: odd CTAs claim from the smallest experts' end
-  int lsu_store;             // one-output kinds: write the staged boxes with coalesced st.global
-                             // (128-byte lines) instead of TMA stores
-  int ld_out;                // elements per row of out0 (lsu_store)
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
   // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
@@ -906,26 +903,17 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           const int M = (KIND == G_DW1) ? p.d : p.n;
           if (row0 < M) {
             constexpr int kC = BN / EC::kColSplit;
-            if (p.lsu_store) {
-              __nv_bfloat16* dst = p.out0 + (size_t)(t.e * M + row0) * p.ld_out + t.n0;
+            const uint32_t buf = stg + ring * EC::kBufBytes;
+            stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_shared_v4(buf + sw128(lane, j), make_uint4(0u, 0u, 0u, 0u));
+            stage_publish();
+            if (lane == 0) {
               for (int c = half * kC; c < half * kC + kC; c += 64)
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  *reinterpret_cast<uint4*>(dst + (size_t)(4 * i + (lane >> 3)) * p.ld_out + c + 8 * (lane & 7)) =
-                      make_uint4(0u, 0u, 0u, 0u);
-            } else {
-              const uint32_t buf = stg + ring * EC::kBufBytes;
-              stage_wait(std::integral_constant<int, EC::kBufs - 1>{});
-#pragma unroll
-              for (int j = 0; j < 8; ++j) st_shared_v4(buf + sw128(lane, j), make_uint4(0u, 0u, 0u, 0u));
-              stage_publish();
-              if (lane == 0) {
-                for (int c = half * kC; c < half * kC + kC; c += 64)
-                  tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
-                bulk_commit();
-              }
-              ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
+                tma_store_2d(&p.tmC0, buf, t.n0 + c, t.e * M + row0);
+              bulk_commit();
             }
+            ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
           }
           continue;
         }
@@ -1113,26 +1101,12 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
               }
               st_shared_v4(buf + sw128(lane, j), pack8f(v));
             }
-            if (p.lsu_store) {
-              // the warp reads the box back a quarter-row per lane -- 4 whole
-              // 128-byte lines per instruction -- and stores them with st.global
-              __syncwarp();
-              __nv_bfloat16* dst = p.out0 + (size_t)orow * p.ld_out + t.n0 + c;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int row = 4 * i + (lane >> 3), ch = lane & 7;
-                const uint4 w = ld_shared_v4(buf + sw128(row, ch));
-                *reinterpret_cast<uint4*>(dst + (size_t)row * p.ld_out + 8 * ch) = w;
-              }
-              __syncwarp();
-            } else {
-              stage_publish();
-              if (lane == 0) {
-                tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
-                bulk_commit();
-              }
-              ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
+            stage_publish();
+            if (lane == 0) {
+              tma_store_2d(&p.tmC0, buf, t.n0 + c, orow);
+              bulk_commit();
             }
+            ring = ring + 1 == EC::kBufs ? 0 : ring + 1;
           }
         }
       } else if constexpr (KIND == G_DH) {

@@ -119,7 +119,6 @@ struct Plan {
   int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
   int epi_dw;           // epilogue warps of the weight-gradient kernels
   int dw_dual;          // weight-gradient tiles claimed from both ends of the expert order
-  int lsu_store;        // one-output epilogues store with st.global instead of TMA
   int dw1_pair, dw2_pair;  // weight-gradient GEMMs on CTA pairs (256 x 256 tiles)
   int ksplit, ksplit_rows;
 };
@@ -175,7 +174,6 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
     if (x == 4 || x == 8) p.epi_dw = x;
   }
   if (const char* v = std::getenv("MOE_DW_DUAL")) p.dw_dual = std::atoi(v) != 0;
-  p.lsu_store = std::getenv("MOE_LSU_STORE") && std::atoi(std::getenv("MOE_LSU_STORE")) != 0;
   // 256 x 256 pair tiles where both output dimensions are multiples of 256
   // (MOE_DW_PAIR=1 turns them on)
   const bool pair_on = std::getenv("MOE_DW_PAIR") && std::atoi(std::getenv("MOE_DW_PAIR")) != 0;
@@ -591,8 +589,6 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
-    g.lsu_store = p.lsu_store;
-    g.ld_out = p.d;
     ProfScope ps(st, "down_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -864,8 +860,6 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.num_m_tiles = (int)cdiv(p.n, 128);
     g.num_n_tiles = p.d / p.bn_dw2;
     g.out0 = static_cast<__nv_bfloat16*>(dW2);
-    g.lsu_store = p.lsu_store;
-    g.ld_out = p.d;
     g.sched = w.sched + 0;  // 64-bit tile counter (front and back claims)
     g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
@@ -892,8 +886,6 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     g.num_m_tiles = (int)cdiv(p.d, 128);
     g.num_n_tiles = 2 * p.n / p.bn_dw1;
     g.out0 = static_cast<__nv_bfloat16*>(dW1);
-    g.lsu_store = p.lsu_store;
-    g.ld_out = 2 * p.n;
     g.sched = w.sched + 2;  // a 64-bit counter of its own
     g.dual_ended = p.dw_dual;
     g.expert_order = w.expert_order;
@@ -918,8 +910,6 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     MOE_TRY_MAP(make_tmap(&g.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, (uint32_t)p.bn_dxt));
     g.num_n_tiles = p.d / p.bn_dxt;
     g.out0 = w.dXt;
-    g.lsu_store = p.lsu_store;
-    g.ld_out = p.d;
     if (rg) {
       g.rvec = w.WrT;
       g.rscale = w.dz_row;
