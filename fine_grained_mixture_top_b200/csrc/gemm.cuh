@@ -67,6 +67,9 @@ struct GemmParams {
   int* sched;                // weight-gradient kinds: zeroed 64-bit tile counter (8-byte aligned)
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
   int dual_ended;            // weight-gradient kinds: odd CTAs claim from the smallest experts' end
+  // grouped-M kinds: the 128-row M tiles to run, [count, tile...], or null
+  // for all of them (the pair kernel's list: the first of each pair of tiles)
+  const int* mlist;
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
   // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
@@ -218,6 +221,7 @@ template <int KIND, int BN>
 __device__ __forceinline__ int gemm_num_tiles(const GemmParams& p) {
   using KT = KindTraits<KIND>;
   if constexpr (KT::kGroupedM) {
+    if (p.mlist) return __ldg(p.mlist) * p.num_n_tiles;
     return (__ldg(p.offsets + p.E) / kBM) * p.num_n_tiles;
   } else if constexpr (KT::kGroupedK) {
     return p.E * p.num_m_tiles * p.num_n_tiles;
@@ -237,6 +241,7 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
   if constexpr (KT::kGroupedM) {
     t.mt = tile / p.num_n_tiles;
     t.nt = tile - t.mt * p.num_n_tiles;
+    if (p.mlist) t.mt = __ldg(p.mlist + 1 + t.mt);
     t.e = __ldg(p.tile_expert + t.mt);
     t.m0 = t.mt * kBM;
     if constexpr (KIND == G_UP || KIND == G_UPQ) t.n0 = t.nt * (BN / 2);

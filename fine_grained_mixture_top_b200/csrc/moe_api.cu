@@ -120,6 +120,7 @@ struct Plan {
   int epi_dw;           // epilogue warps of the weight-gradient kernels
   int dw_dual;          // weight-gradient tiles claimed from both ends of the expert order
   int dw1_pair, dw2_pair;  // weight-gradient GEMMs on CTA pairs (256 x 256 tiles)
+  int gm_pair;             // down-proj and dX~ on CTA pairs (256 x 256 tiles of two M tiles)
   int ksplit, ksplit_rows;
 };
 
@@ -179,6 +180,11 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   const bool pair_on = std::getenv("MOE_DW_PAIR") && std::atoi(std::getenv("MOE_DW_PAIR")) != 0;
   p.dw1_pair = pair_on && (d % 256 == 0) && ((2 * n) % 256 == 0);
   p.dw2_pair = pair_on && (d % 256 == 0) && (n % 256 == 0);
+  // Down-proj and dX~ on CTA pairs (MOE_GM_PAIR=1, where N = d splits into
+  // 256-column tiles).  Off by default: measured no faster than one CTA per
+  // 128 x 256 tile on any workload here, and slower on the balanced ones.
+  p.gm_pair = 0;
+  if (const char* v = std::getenv("MOE_GM_PAIR")) p.gm_pair = (d % 256 == 0) && std::atoi(v) != 0;
   p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
@@ -232,6 +238,7 @@ size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
 struct FwdWs {
   __nv_bfloat16* A;
   __nv_bfloat16* Y;
+  int *mpair, *mleft;  // pair and leftover lists of the M tiles (CTA-pair down-proj)
 };
 // MXFP8 forward: codes and scales of X, W1, W2 and A, and Y
 // MXFP8 expert weights: codes K-major and scales in the MMA's tile layout
@@ -249,6 +256,8 @@ size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
   Carve c{static_cast<char*>(ws)};
   w->A = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
   w->Y = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
+  w->mpair = c.take<int>((size_t)(p.R_max / 256 + 2));
+  w->mleft = c.take<int>((size_t)p.E + 1);
   return c.off;
 }
 
@@ -284,6 +293,7 @@ struct BwdWs {
   __nv_bfloat16 *dH, *Ahat, *dXt, *dz_split;
   float *dS_part, *dz_row, *WrT, *dWr_part;
   int *sched, *expert_order;
+  int *mpair, *mleft;  // pair and leftover lists of the M tiles (CTA-pair dX~)
 };
 size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   Carve c{static_cast<char*>(ws)};
@@ -297,6 +307,8 @@ size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   w->dWr_part = c.take<float>((size_t)p.ksplit * p.d * p.Epad);
   w->sched = c.take<int>(16);
   w->expert_order = c.take<int>((size_t)p.E);
+  w->mpair = c.take<int>((size_t)(p.R_max / 256 + 2));
+  w->mleft = c.take<int>((size_t)p.E + 1);
   return c.off;
 }
 
@@ -590,7 +602,18 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "down_proj_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    if (p.gm_pair) {
+      // pairs of M tiles on CTA pairs, then each expert's odd last M tile on one CTA
+      MOE_TRY_CUDA(launch_pair_lists(rt->offsets, p.E, w.mpair, w.mleft, st));
+      g.num_n_tiles = p.d / 256;
+      g.mlist = w.mpair;
+      MOE_TRY_CUDA(launch_gemm_pair_m(G_DOWN, 4, g, (int)std::min<int64_t>(sms / 2, (mtiles / 2) * g.num_n_tiles), st));
+      g.mlist = w.mleft;
+      MOE_TRY_CUDA(launch_gemm(G_DOWN, 256, 4, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
+                               false));
+    } else {
+      MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    }
   }
   {
     ProfScope ps(st, "aggregate_fwd");
@@ -916,7 +939,24 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     }
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
     ProfScope ps(st, "dxt_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    if (p.gm_pair) {
+      // pairs of M tiles on CTA pairs (each CTA loading 128 of a tile's 256 W1
+      // rows), then each expert's odd last M tile on one CTA
+      MOE_TRY_CUDA(launch_pair_lists(rt->offsets, p.E, w.mpair, w.mleft, st));
+      GemmParams gp = g;
+      MOE_TRY_MAP(make_tmap(&gp.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 128));
+      gp.num_n_tiles = p.d / 256;
+      gp.mlist = w.mpair;
+      MOE_TRY_CUDA(
+          launch_gemm_pair_m(G_DXT, p.epi_dxt, gp, (int)std::min<int64_t>(sms / 2, (mtiles / 2) * gp.num_n_tiles), st));
+      g.num_n_tiles = p.d / 256;
+      g.mlist = w.mleft;
+      MOE_TRY_CUDA(
+          launch_gemm(G_DXT, 256, p.epi_dxt, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
+                      false));
+    } else {
+      MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
+    }
   }
   if (rg) MOE_TRY_CUDA(run_dwr(p, rt, w, X, dWr, status, sms, st));
   record_ready(grad_ready, 2, st);  // dWr final (or nothing to wait for without the router path)

@@ -50,10 +50,20 @@ void set_gemm_trace(int kind, void* buf, int cap);
 extern thread_local char g_launch_diag[256];
 
 // epi: epilogue warps (4, or 8 for the dH and dX~ kinds)
-cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s);
+// traced = false: the launch writes no role timeline even while its kind is
+// traced (the second launch of a kind that runs as two)
+cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p, int grid, cudaStream_t s, bool traced = true);
 // Weight-gradient kinds on CTA pairs (256 x 256 tiles, gemm_pair.cuh):
 // p.num_m_tiles / p.num_n_tiles count 256-wide tiles; `pairs` clusters of 2.
 cudaError_t launch_gemm_pair(int kind, int epi, const GemmParams& p, int pairs, cudaStream_t s);
+// Down-proj and dX~ on CTA pairs (gemm_pair_m.cuh) over the pair list p.mlist;
+// p.num_n_tiles counts 256-column tiles; at most `max_pairs` clusters of 2
+// (fewer if fewer fit the device at once).
+cudaError_t launch_gemm_pair_m(int kind, int epi, const GemmParams& p, int max_pairs, cudaStream_t s);
+// Pair list and leftover list of the grouped-M tiles from the segment offsets
+// (each [count, tile...]; `pairs` holds up to R_max / 256 + 1 entries after the
+// count, `left` up to E).
+cudaError_t launch_pair_lists(const int* offsets, int E, int* pairs, int* left, cudaStream_t s);
 
 // Per-kernel timing (moe_profile_enable): while on, each launch site brackets
 // its kernel with two CUDA events recorded on the launching stream.

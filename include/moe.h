@@ -361,6 +361,9 @@ moe_status moe_profile_read(int32_t i, const char** name, float* ms);
  * 1 accumulator free, 2 first k-block's operands ready, 3 last MMA committed;
  * epilogue 0 tile taken, 1 accumulator full, 2 accumulator released (its
  * stores issued); gather 0 tile taken, 1 last k-block's copies issued.
+ * Where a kind runs as two launches -- down-proj and dX~ with d % 256 == 0:
+ * pairs of M tiles on 2-CTA clusters, then each expert's odd last M tile on
+ * single CTAs -- the first (pair) launch is the one traced.
  * Launches in flight keep the buffer: turn tracing off or synchronize before
  * freeing it.  Results do not depend on tracing.
  */

@@ -21,6 +21,11 @@ SHAPES = [
     MoEConfig("dense", T=200, d=128, E=1, n=64, K=1, w_std=0.05, seed=13),
     # fewer tokens than a tile, E not a multiple of 64, empty experts
     MoEConfig("sparse", T=64, d=128, E=70, n=64, K=4, w_std=0.05, seed=14),
+    # several M tiles per expert, even and odd counts: down-proj and dX~ on CTA
+    # pairs plus each expert's leftover tile on one CTA (dX~ with 8 epilogue warps)
+    MoEConfig("pairs", T=1500, d=512, E=6, n=128, K=3, w_std=0.05, bias="normal", seed=15),
+    # the same with a long dX~ main loop (2n = 1280: 4 epilogue warps)
+    MoEConfig("pairs_n640", T=600, d=256, E=3, n=640, K=2, w_std=0.05, bias="normal", seed=16),
 ]
 
 
@@ -62,6 +67,18 @@ def test_layer_parity(cfg):
     X, Wr, b, *_ = _np_inputs(inp)
     z = orc.router_logits(X, Wr, b)
     P.check_router(g, z, orc.softmax_rows(z), cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["pairs", "pairs_n640"])
+def test_layer_parity_pair_tiles(name, monkeypatch):
+    """Down-proj and dX~ on CTA pairs (256-row tiles over two M tiles of one
+    expert, leftover tiles on single CTAs), an opt-in path."""
+    monkeypatch.setenv("MOE_GM_PAIR", "1")
+    cfg = next(c for c in SHAPES if c.name == name)
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
     _compare_layer(layer, cfg, inp)
 
 
