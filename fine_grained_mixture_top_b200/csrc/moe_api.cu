@@ -216,6 +216,7 @@ struct RouteWs {
   uint32_t* memberT;  // token rounding: [E, ceil(T/32)]
   uint32_t* finalT;   // token rounding: [E, ceil(T/32)]
   float* probsT;      // token rounding: [E, T]
+  int* rowpre;        // token rounding: [E, ceil(T/32)]
   int* local;         // token rounding: [T]
   int* blk;           // token rounding: [ceil(T/256) + 1]
 };
@@ -230,6 +231,7 @@ size_t carve_route(const Plan& p, void* ws, RouteWs* w) {
   w->memberT = c.take<uint32_t>((size_t)p.E * W);
   w->finalT = c.take<uint32_t>((size_t)p.E * W);
   w->probsT = c.take<float>((size_t)p.E * p.T);
+  w->rowpre = c.take<int>((size_t)p.E * W);
   w->local = c.take<int>((size_t)p.T);
   w->blk = c.take<int>((size_t)cdiv(p.T, 256) + 1);
   return c.off;
@@ -551,6 +553,7 @@ moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe
   r.probsT = w.probsT;
   r.memberT = w.memberT;
   r.finalT = w.finalT;
+  r.rowpre = w.rowpre;
   r.local = w.local;
   r.blk = w.blk;
   r.sync = w.sync + 1;

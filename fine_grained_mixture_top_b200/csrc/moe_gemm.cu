@@ -115,7 +115,7 @@ static cudaError_t launch_gm_pair_one(const GemmParams& p, int max_pairs, cudaSt
 // The dynamic shared-memory limit is a per-device property of a function: it
 // is set once for each (function, device), under a lock, so that host threads
 // driving different devices (or the same one) all see it set before they
-// launch.
+// launch.  Callers pass the largest size the function is ever launched with.
 cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
   static std::mutex mu;
   static std::set<std::pair<const void*, int>> done;

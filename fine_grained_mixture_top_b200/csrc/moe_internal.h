@@ -109,7 +109,8 @@ struct RoundArgs {
   float* probsT;        // [E, T]
   uint32_t* memberT;    // [E, ceil(T/32)] routed tokens of each expert
   uint32_t* finalT;     // [E, ceil(T/32)] tokens of each expert after rounding
-  int* local;           // [T] offset of each token's pairs inside its block of 256
+  int* rowpre;          // [E, ceil(T/32)] final tokens of each expert before each word
+  int* local;           // [T] pair count of each token, then its pairs' offset inside its block of 256
   int* blk;             // [ceil(T/256) + 1] block offsets, total last
   int* sync;            // [1] blocks done
 };

@@ -342,15 +342,17 @@ __device__ __forceinline__ unsigned long long splitmix64_dev(unsigned long long 
 
 // Token rounding works on per-expert rows: memberT[e][w] holds bit t & 31 of
 // word w = t / 32 for each token t routed to e, probsT[e][t] = p[t, e].  One
-// block per expert then reads its row contiguously.
+// block per expert then reads its row contiguously.  tr_member also records
+// each token's pair count, which the selection adjusts token by token.
 __global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int W, uint32_t* memberT,
-                                 int* sync) {
+                                 int* tok_count, int* sync) {
   pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t == 0) *sync = 0;  // for tr_count_kernel's last block
+  if (t == 0) *sync = 0;  // for tr_scan_kernel's last block
   if (t >= T) return;
-  for (int p = tok_ptr[t]; p < tok_ptr[t + 1]; ++p)
-    atomicOr(&memberT[(size_t)pair_expert[p] * W + (t >> 5)], 1u << (t & 31));
+  const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
+  tok_count[t] = p1 - p0;
+  for (int p = p0; p < p1; ++p) atomicOr(&memberT[(size_t)pair_expert[p] * W + (t >> 5)], 1u << (t & 31));
 }
 
 // probsT[e, t] = probs[t, e], 32 x 32 tiles through shared memory
@@ -369,73 +371,117 @@ __global__ void tr_transpose_kernel(const float* __restrict__ probs, float* __re
   }
 }
 
-// One block per expert: radix select (8 passes of 8 bits) of the k extreme
-// 64-bit keys (p bits << 32 | ~t) among the candidate tokens, then the
-// expert's final row finalT[e] = memberT[e] with the selected tokens added
-// (rounding up) or removed (rounding down).  With STAGED the expert's p row
-// and candidate mask are first copied into shared memory; histogram updates
-// are aggregated per warp over lanes with the same digit.
+// Exclusive scan over the block (blockDim.x a multiple of 32, at most 1024);
+// *total gets the sum.  sh: 32 ints of shared memory.
+__device__ int block_exclusive_scan(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nw ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;  // inclusive warp totals
+  }
+  __syncthreads();
+  *total = sh[nw - 1];
+  const int r = (warp > 0 ? sh[warp - 1] : 0) + x - v;
+  __syncthreads();
+  return r;
+}
+
+// The selection of one expert (one block): the k smallest 64-bit keys among
+// the candidate tokens, key = (p bits << 32) | (~0 - t) when rounding down
+// (least p first, ties: larger t first) and (~p bits << 32) | t when rounding
+// up (largest p first, ties: smaller t first).  Keys are distinct, so "key <=
+// the k-th smallest" selects exactly k tokens.
+//
+// The expert's candidate words and 32-bit p keys are first staged in shared
+// memory (when its row fits) with many loads in flight per thread, and each
+// thread takes the smallest key among its own candidates on the way.  The
+// k-th smallest of these per-thread minima, tau, bounds the k-th smallest
+// key from above (k threads each hold a candidate <= tau), so only the
+// candidates <= tau -- about k of them when the candidates are spread over
+// the threads -- are collected and sorted, which gives the k-th key.  If
+// more than kTrListCap candidates are <= tau (fewer than k threads hold
+// candidates, or many equal p), 8 radix passes of 8 bits over all
+// candidates find it instead.
+constexpr int kTrListCap = 2048;
+constexpr int kTrSelThreads = 256;  // > the largest k (127)
+constexpr size_t kTrSelFixed = (size_t)256 * 4 + (size_t)kTrListCap * 8;  // radix histogram + list
+constexpr size_t kTrSelMax = 200 * 1024;  // dynamic shared memory of the staged selection, at most
+
+// Candidates and keys of one expert's selection.  STAGED: the keys [T] and
+// candidate words [W] are in shared memory; otherwise they are read from the
+// expert's rows in global memory.
 template <bool STAGED>
-__global__ void __launch_bounds__(1024) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
-                                                         const int* counts, const float* probsT,
-                                                         const uint32_t* memberT, uint32_t* finalT) {
-  pdl_wait();
-  extern __shared__ uint32_t stage[];  // STAGED: p bits [T], then the candidate mask [W]
-  __shared__ unsigned int hist[256];
+struct TrSelect {
+  int T, W;
+  bool up;
+  const uint32_t* mrow;    // routed tokens of the expert (global)
+  const float* prow;       // p of the expert (global)
+  const uint32_t* s_key;   // STAGED: keys [T]
+  const uint32_t* s_cand;  // STAGED: candidate words [W]
+  __device__ __forceinline__ uint32_t valid(int w) const {
+    return (w == W - 1 && (T & 31)) ? ((1u << (T & 31)) - 1u) : 0xFFFFFFFFu;
+  }
+  __device__ __forceinline__ uint32_t cand_word(int w) const {
+    if constexpr (STAGED) {
+      return s_cand[w];
+    } else {
+      const uint32_t m = mrow[w];
+      return (up ? ~m : m) & valid(w);
+    }
+  }
+  __device__ __forceinline__ uint32_t mem_word(int w) const {  // the routed tokens
+    if constexpr (STAGED) {
+      const uint32_t c = s_cand[w];
+      return up ? (~c & valid(w)) : c;
+    } else {
+      return mrow[w];
+    }
+  }
+  __device__ __forceinline__ uint32_t key32(int t) const {
+    if constexpr (STAGED) {
+      return s_key[t];
+    } else {
+      const uint32_t pb = __float_as_uint(prow[t]);
+      return up ? ~pb : pb;
+    }
+  }
+  __device__ __forceinline__ unsigned long long key64(int t) const {
+    return ((unsigned long long)key32(t) << 32) | (up ? (unsigned)t : (0xFFFFFFFFu - (unsigned)t));
+  }
+};
+
+// 8 passes of 8 bits over all candidates (warp-aggregated histogram
+// updates): the k-th smallest key.
+template <bool STAGED>
+__device__ unsigned long long tr_radix_kth(const TrSelect<STAGED>& s, int k, unsigned* hist /*[256]*/) {
   __shared__ unsigned long long s_prefix;
   __shared__ int s_k;
-  const int e = blockIdx.x;
   const int lane = threadIdx.x & 31;
-  const uint32_t* mrow = memberT + (size_t)e * W;
-  uint32_t* frow = finalT + (size_t)e * W;
-  const float* prow = probsT + (size_t)e * T;
-  const int c = counts[e];
-  const int rem = c % kTile;
-  if (rem == 0) {  // already a multiple of the tile: keep the routed set
-    for (int w = threadIdx.x; w < W; w += blockDim.x) frow[w] = mrow[w];
-    return;
-  }
-  bool up;
-  if (mode == 1) up = rem >= kTile / 2;
-  else up = (int)(splitmix64_dev(seed ^ (unsigned long long)e) % (unsigned long long)kTile) < rem;
-  if (up && c - rem + kTile > T) up = false;
-  const int k = up ? kTile - rem : rem;
-  // candidates: unrouted tokens when rounding up, routed ones when rounding down
-  const uint32_t tail = (T & 31) ? ((1u << (T & 31)) - 1u) : 0xFFFFFFFFu;
-  auto cand_word = [&](int w) -> uint32_t {
-    const uint32_t m = mrow[w];
-    const uint32_t valid = (w == W - 1) ? tail : 0xFFFFFFFFu;
-    return (up ? ~m : m) & valid;
-  };
-  uint32_t* s_p = stage;
-  uint32_t* s_cand = stage + T;
-  if constexpr (STAGED) {
-    for (int t = threadIdx.x; t < T; t += blockDim.x) s_p[t] = __float_as_uint(prow[t]);
-    for (int w = threadIdx.x; w < W; w += blockDim.x) s_cand[w] = cand_word(w);
-    __syncthreads();
-  }
-  auto is_cand = [&](int t) -> bool {
-    const uint32_t cw = STAGED ? s_cand[t >> 5] : cand_word(t >> 5);
-    return (cw >> (t & 31)) & 1u;
-  };
-  auto key_of = [&](int t) -> unsigned long long {
-    const uint32_t pb = STAGED ? s_p[t] : __float_as_uint(prow[t]);
-    const unsigned long long kk = ((unsigned long long)pb << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)t);
-    return up ? ~kk : kk;   // select the k smallest of this key
-  };
-  __shared__ int s_done;
   unsigned long long prefix = 0ull, mask = 0ull;
   int kk = k;
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
-    for (int t0 = 0; t0 < T; t0 += blockDim.x) {  // warp-uniform trip count
+    for (int t0 = 0; t0 < s.T; t0 += blockDim.x) {  // warp-uniform trip count
       const int t = t0 + threadIdx.x;
       bool hit = false;
       uint32_t digit = 0u;
-      if (t < T && is_cand(t)) {
-        const unsigned long long key = key_of(t);
+      if (t < s.T && ((s.cand_word(t >> 5) >> (t & 31)) & 1u)) {
+        const unsigned long long key = s.key64(t);
         hit = (key & mask) == prefix;
         digit = (uint32_t)((key >> shift) & 255ull);
       }
@@ -460,7 +506,7 @@ __global__ void __launch_bounds__(1024) tr_select_kernel(int T, int W, int mode,
         if (lane >= o) incl += y;
       }
       const uint32_t reach = __ballot_sync(0xffffffffu, incl >= kk);
-      const int owner = __ffs(reach) - 1;  // kk <= number of matching candidates, so some lane reaches it
+      const int owner = __ffs(reach) - 1;  // kk <= number of matching candidates
       if (lane == owner) {
         int cum = incl - sum, dg = 8 * lane;
 #pragma unroll 1
@@ -468,69 +514,284 @@ __global__ void __launch_bounds__(1024) tr_select_kernel(int T, int W, int mode,
           if (cum + loc[i] >= kk) break;
           cum += loc[i];
         }
-        const int left = kk - cum;
         s_prefix = prefix | ((unsigned long long)dg << shift);
-        s_k = left;
-        // once the p bits are fixed (after 4 passes), stop if every candidate
-        // with that p is selected: the token bits only break ties
-        s_done = (shift == 32 && left == (int)hist[dg]) ? 1 : 0;
+        s_k = kk - cum;
       }
     }
     __syncthreads();
     prefix = s_prefix;
     kk = s_k;
     mask |= 255ull << shift;
-    const bool done = s_done != 0 && shift == 32;
     __syncthreads();
-    if (done) {
-      prefix |= 0xFFFFFFFFull;  // select every candidate whose p bits are <= the k-th one's
-      break;
-    }
   }
-  // the selected candidates are those with key <= prefix (exactly k of them)
-  for (int w = threadIdx.x; w < W; w += blockDim.x) {
-    uint32_t sel = 0u;
-    const uint32_t cw = STAGED ? s_cand[w] : cand_word(w);
-    for (uint32_t m = cw; m; m &= m - 1u) {
-      const int b = __ffs(m) - 1;
-      if (key_of(w * 32 + b) <= prefix) sel |= 1u << b;
+  return prefix;  // all 64 bits fixed: the k-th smallest key itself
+}
+
+// Ascending bitonic sort of n keys in shared memory, padded with ~0 to a
+// power of two (the buffer holds it).
+__device__ __forceinline__ void tr_sort(unsigned long long* a, int n) {
+  int P = 2;
+  while (P < n) P <<= 1;
+  for (int i = n + threadIdx.x; i < P; i += blockDim.x) a[i] = ~0ull;
+  __syncthreads();
+  for (int kk = 2; kk <= P; kk <<= 1) {
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = a[i], y = a[ixj];
+          if ((x > y) == ((i & kk) == 0)) {
+            a[i] = y;
+            a[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
     }
-    const uint32_t mem = mrow[w];
-    frow[w] = up ? (mem | sel) : (mem & ~sel);
   }
 }
 
-// A warp holds 32 consecutive tokens (one word column w of finalT).  For each
-// group of 32 experts, lane j loads expert (32 c + j)'s word and 32 ballots
-// transpose the 32 x 32 bit block, so that lane i ends with the group's
-// expert mask of token 32 w + i.
-__device__ __forceinline__ uint32_t tr_token_mask(const uint32_t* finalT, int E, int W, int w, int c, int lane) {
-  const int e = 32 * c + lane;
-  const uint32_t x = (e < E && w < W) ? finalT[(size_t)e * W + w] : 0u;
-  uint32_t mine = 0u;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t b = __ballot_sync(0xffffffffu, (x >> i) & 1u);
-    if (lane == i) mine = b;
+// Ascending bitonic sort over the block, one key per thread (blockDim.x a
+// power of two): returns the key of rank threadIdx.x.  Partners within a
+// warp exchange by shuffles; wider strides go through shared memory
+// (buf: blockDim.x keys).
+__device__ __forceinline__ unsigned long long tr_block_sort1(unsigned long long v, unsigned long long* buf) {
+  const int n = (int)blockDim.x, i = (int)threadIdx.x;
+  for (int kk = 2; kk <= n; kk <<= 1) {
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      unsigned long long o;
+      if (j >= 32) {
+        buf[i] = v;
+        __syncthreads();
+        o = buf[i ^ j];
+        __syncthreads();
+      } else {
+        o = __shfl_xor_sync(0xffffffffu, v, j);
+      }
+      const bool asc = (i & kk) == 0;
+      const bool lower = (i & j) == 0;
+      v = (lower == asc) ? (o < v ? o : v) : (o > v ? o : v);
+    }
   }
-  return mine;
+  return v;
 }
 
-// Per token: its expert count after rounding; a block-wide exclusive scan
-// gives its offset inside the block, and the last block to finish scans the
-// block totals (exclusive, total at [nblocks]).
-__global__ void __launch_bounds__(256) tr_count_kernel(const uint32_t* finalT, int T, int E, int W, int* local,
-                                                       int* blk, int* sync) {
+// One block per expert: the expert's final token row finalT[e] (memberT[e]
+// with the selected tokens added when rounding up, removed when rounding
+// down), its final count (counts[e], rewritten in place), each token's pair
+// count adjusted (tok_count[t] += 1 or -= 1), and rowpre[e][w], the number of
+// the expert's final tokens before word w (the rank of a token's row inside
+// the expert's segment is rowpre plus a popcount within its word).
+// STAGED: shared memory holds, after the radix histogram and the list, the
+// expert's keys [T rounded up to 4] and candidate words [W].  Tokens are
+// visited four at a time (one vector load, one candidate nibble).
+template <bool STAGED>
+__global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
+                                                                 int* counts, const float* probsT,
+                                                                 const uint32_t* memberT, uint32_t* finalT,
+                                                                 int* rowpre, int* tok_count) {
   pdl_wait();
-  __shared__ int sh[8];
+  extern __shared__ __align__(16) uint8_t tr_smem[];
+  unsigned* hist = reinterpret_cast<unsigned*>(tr_smem);                                 // [256]
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(tr_smem + 256 * 4);  // [kTrListCap]
+  const int T4 = (T + 3) & ~3;
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(tr_smem + kTrSelFixed);  // STAGED: [T4]
+  uint32_t* s_cand = s_key + T4;                                         // STAGED: [W]
+  __shared__ int sh[32];
+  __shared__ int s_cnt;
+  __shared__ unsigned long long s_thr;
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthr = (int)blockDim.x;
+  uint32_t* frow = finalT + (size_t)e * W;
+  const int c = counts[e];
+  const int rem = c % kTile;
+  bool up = false;
+  if (rem != 0) {
+    if (mode == 1) up = rem >= kTile / 2;
+    else up = (int)(splitmix64_dev(seed ^ (unsigned long long)e) % (unsigned long long)kTile) < rem;
+    if (up && c - rem + kTile > T) up = false;
+  }
+  const int k = rem == 0 ? 0 : (up ? kTile - rem : rem);
+  TrSelect<STAGED> s;
+  s.T = T;
+  s.W = W;
+  s.up = up;
+  s.mrow = memberT + (size_t)e * W;
+  s.prow = probsT + (size_t)e * T;
+  s.s_key = s_key;
+  s.s_cand = s_cand;
+  const bool vec = (T & 3) == 0;  // the row is 16-byte aligned: float4 loads
+  auto tie = [&](int t) -> unsigned long long { return up ? (unsigned)t : (0xFFFFFFFFu - (unsigned)t); };
+  // p keys of tokens 4q .. 4q+3 (past T: the largest key, never a candidate)
+  auto load_quad = [&](int q, uint32_t (&kq)[4]) {
+    const int t0 = 4 * q;
+    float v[4];
+    if (vec) {
+      const float4 f = reinterpret_cast<const float4*>(s.prow)[q];
+      v[0] = f.x;
+      v[1] = f.y;
+      v[2] = f.z;
+      v[3] = f.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = t0 + j < T ? s.prow[t0 + j] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t pb = __float_as_uint(v[j]);
+      kq[j] = t0 + j < T ? (up ? ~pb : pb) : 0xFFFFFFFFu;
+    }
+  };
+  auto nibble = [&](int q) -> uint32_t { return (s.cand_word(q >> 3) >> ((4 * q) & 31)) & 0xFu; };
+  const int Q = T4 / 4;
+  // 1. staging (STAGED) and each thread's smallest candidate key
+  unsigned long long mn = ~0ull;
+  if constexpr (STAGED) {
+    for (int w = threadIdx.x; w < W; w += nthr) {
+      const uint32_t m = s.mrow[w];
+      s_cand[w] = (up ? ~m : m) & s.valid(w);
+    }
+    __syncthreads();
+  }
+  if (k > 0) {
+    for (int q = threadIdx.x; q < Q; q += nthr) {
+      uint32_t kq[4];
+      load_quad(q, kq);
+      if constexpr (STAGED) *reinterpret_cast<uint4*>(s_key + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
+      const uint32_t nb = nibble(q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if ((nb >> j) & 1u) {
+          const unsigned long long x = ((unsigned long long)kq[j] << 32) | tie(4 * q + j);
+          mn = x < mn ? x : mn;
+        }
+    }
+  }
+  if constexpr (STAGED) __syncthreads();
+  unsigned long long thr = 0ull;
+  bool listed = false;  // the selected tokens are the list entries <= thr
+  int len = 0;
+  if (k > 0) {
+    // 2. tau: the k-th smallest thread minimum (k < 128 <= nthr)
+    const unsigned long long r = tr_block_sort1(mn, list);
+    if (threadIdx.x == k - 1) s_thr = r;
+    if (threadIdx.x == 0) s_cnt = 0;
+    __syncthreads();
+    const unsigned long long tau = s_thr;
+    // 3. the candidates <= tau; the k-th smallest of them is the k-th key
+    for (int q = threadIdx.x; q < Q; q += nthr) {
+      const uint32_t nb = nibble(q);
+      if (nb == 0u) continue;
+      uint32_t kq[4];
+      if constexpr (STAGED) {
+        const uint4 u = *reinterpret_cast<const uint4*>(s_key + 4 * q);
+        kq[0] = u.x;
+        kq[1] = u.y;
+        kq[2] = u.z;
+        kq[3] = u.w;
+      } else {
+        load_quad(q, kq);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if ((nb >> j) & 1u) {
+          const unsigned long long x = ((unsigned long long)kq[j] << 32) | tie(4 * q + j);
+          if (x <= tau) {
+            const int i = atomicAdd(&s_cnt, 1);
+            if (i < kTrListCap) list[i] = x;
+          }
+        }
+    }
+    __syncthreads();
+    len = s_cnt;
+    if (len <= nthr) {
+      const unsigned long long v = threadIdx.x < len ? list[threadIdx.x] : ~0ull;
+      __syncthreads();  // list[] is reused as the sort's exchange buffer
+      const unsigned long long r2 = tr_block_sort1(v, list);
+      if (threadIdx.x == k - 1) s_thr = r2;
+      __syncthreads();
+      if (threadIdx.x < len) list[threadIdx.x] = r2;  // sorted: the first k are the selected
+      __syncthreads();
+      thr = s_thr;
+      listed = true;
+    } else if (len <= kTrListCap) {
+      tr_sort(list, len);
+      thr = list[k - 1];
+      listed = true;
+    } else {
+      thr = tr_radix_kth<STAGED>(s, k, hist);
+    }
+  }
+  if (STAGED && (listed || k == 0)) {
+    // 4a. final row in shared memory: the routed words with the k selected
+    // tokens (the first k sorted list entries) set or cleared
+    for (int w = threadIdx.x; w < W; w += nthr) s_cand[w] = s.mem_word(w);
+    __syncthreads();
+    for (int i = threadIdx.x; i < k; i += nthr) {
+      const unsigned lo = (unsigned)(list[i] & 0xFFFFFFFFull);
+      const int t = up ? (int)lo : (int)(0xFFFFFFFFu - lo);
+      if (up) atomicOr(&s_cand[t >> 5], 1u << (t & 31));
+      else atomicAnd(&s_cand[t >> 5], ~(1u << (t & 31)));
+      atomicAdd(&tok_count[t], up ? 1 : -1);
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < W; w += nthr) frow[w] = s_cand[w];
+  } else {
+    // 4b. final row: a warp per word of 32 tokens; the selected candidates
+    // are the keys <= thr
+    for (int w0 = 0; w0 < W; w0 += nthr / 32) {
+      const int w = w0 + warp;
+      if (w < W) {  // warp-uniform
+        const int t = 32 * w + lane;
+        const uint32_t mem = s.mem_word(w);
+        uint32_t sel = 0u;
+        if (k > 0) {
+          const bool take = ((s.cand_word(w) >> lane) & 1u) && s.key64(t) <= thr;
+          sel = __ballot_sync(0xffffffffu, take);
+          if (take) atomicAdd(&tok_count[t], up ? 1 : -1);
+        }
+        const uint32_t fin = up ? (mem | sel) : (mem & ~sel);
+        __syncwarp();
+        if (lane == 0) {
+          frow[w] = fin;
+          if constexpr (STAGED) s_cand[w] = fin;  // only this warp reads word w here
+        }
+      }
+    }
+  }
+  if (threadIdx.x == 0) counts[e] = rem == 0 ? c : (up ? c - rem + kTile : c - rem);
+  __syncthreads();  // the row's words are written (visible to the block after the barrier)
+  // 5. rowpre: exclusive prefix popcount of the row, contiguous chunks per thread
+  const uint32_t* fin_row = STAGED ? s_cand : frow;
+  const int per = (W + nthr - 1) / nthr;
+  const int w_lo = threadIdx.x * per, w_hi = min(W, w_lo + per);
+  int loc = 0;
+  for (int w = w_lo; w < w_hi; ++w) loc += __popc(fin_row[w]);
+  int tot;
+  int run = block_exclusive_scan(loc, sh, &tot);
+  int* rp = rowpre + (size_t)e * W;
+  for (int w = w_lo; w < w_hi; ++w) {
+    rp[w] = run;
+    run += __popc(fin_row[w]);
+  }
+}
+
+// Per token: exclusive scan of the final pair counts inside each block of
+// 256 tokens (local[t]) and the block totals; the last block to finish scans
+// the block totals (blk, total at [nblocks]), the experts' final counts into
+// segment offsets (no padding: every count is a multiple of the tile) and
+// writes the tile -> expert list.
+__global__ void __launch_bounds__(256) tr_scan_kernel(int T, int E, int* local /* in: counts, out: offsets */,
+                                                      int* blk, int* sync, const int* counts, int* offsets,
+                                                      int* tile_expert) {
+  pdl_wait();
+  __shared__ int sh[32];
   __shared__ int is_last;
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  const int lane = threadIdx.x & 31;
-  int c = 0;
-  for (int g = 0; g < (E + 31) / 32; ++g) c += __popc(tr_token_mask(finalT, E, W, t >> 5, g, lane));
-  if (t >= T) c = 0;
+  const int c = t < T ? local[t] : 0;
   int total;
-  const int ex = block_exclusive_scan_256(c, sh, &total);
+  const int ex = block_exclusive_scan(c, sh, &total);
   if (t < T) local[t] = ex;
   if (threadIdx.x == 0) blk[blockIdx.x] = total;
   __threadfence();
@@ -545,49 +806,146 @@ __global__ void __launch_bounds__(256) tr_count_kernel(const uint32_t* finalT, i
     const int b = b0 + threadIdx.x;
     const int v = b < nb ? __ldcg(blk + b) : 0;
     int tot;
-    const int bex = block_exclusive_scan_256(v, sh, &tot);
+    const int bex = block_exclusive_scan(v, sh, &tot);
     if (b < nb) blk[b] = carry + bex;
     carry += tot;
   }
   if (threadIdx.x == 0) blk[nb] = carry;
+  carry = 0;
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int v = e < E ? __ldcg(counts + e) : 0;
+    int tot;
+    const int eex = block_exclusive_scan(v, sh, &tot);
+    if (e < E) {
+      const int o = carry + eex;
+      offsets[e] = o;
+      for (int tt = o / kTile; tt < (o + v) / kTile; ++tt) tile_expert[tt] = e;
+    }
+    carry += tot;
+  }
+  if (threadIdx.x == 0) offsets[E] = carry;
 }
 
-// Per token: tok_ptr and its pairs in ascending expert order, gates = p
-// renormalised over the token's final expert set.
-__global__ void __launch_bounds__(256) tr_write_kernel(const uint32_t* finalT, const float* probs, int T, int E,
-                                                       int W, const int* local, const int* blk, int* tok_ptr,
-                                                       int* pair_expert, float* pair_gate) {
-  pdl_wait();
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  const int lane = threadIdx.x & 31;
-  const bool live = t < T;
-  int p = live ? blk[blockIdx.x] + local[t] : 0;
-  if (live) {
-    tok_ptr[t] = p;
-    if (t == T - 1) tok_ptr[T] = blk[gridDim.x];
+// Column `lane` of the 32 x 32 bit matrix whose row i is lane i's x (bit j
+// of row i = entry (i, j)): five exchange steps of halving block size.
+__device__ __forceinline__ uint32_t transpose32(uint32_t x, int lane) {
+  uint32_t m = 0x0000FFFFu;
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1, m ^= (m << s)) {
+    const uint32_t o = __shfl_xor_sync(0xffffffffu, x, s);
+    x = (lane & s) ? ((x & ~m) | ((o >> s) & m)) : ((x & m) | ((o & m) << s));
   }
-  const float* pr = probs + (size_t)(live ? t : 0) * E;
+  return x;
+}
+
+// Per token (a warp holds the 32 tokens of one finalT word): the token's
+// final experts from the expert rows (one 32 x 32 bit transpose per group of
+// 32 experts), its gates (p renormalised over the final set, summed in
+// ascending expert order), its pairs in ascending expert order, and each
+// pair's row in the expert-major layout: the expert's offset + rowpre + the
+// expert's tokens before it in the word.  Writes tok_ptr, pair_*, row_tok,
+// row_gate.  Blocks of kTwThreads tokens (small, so that the T / 32 warps
+// spread over every SM); the pair offsets come from tr_scan_kernel's blocks of
+// 256 tokens.  Shared memory: the finalT words of each warp's column [E],
+// each token's expert masks [groups][kTwThreads] and its first kTwList
+// experts [kTwList][kTwThreads].
+constexpr int kTwThreads = 64;
+constexpr int kTwList = 16;
+__global__ void __launch_bounds__(kTwThreads) tr_write_kernel(const uint32_t* finalT, const int* rowpre,
+                                                              const float* probs, int T, int E, int W,
+                                                              const int* local, const int* blk, int nblk,
+                                                              const int* offsets, int* tok_ptr, int* pair_expert,
+                                                              float* pair_gate, int* pair_row, int* row_tok,
+                                                              float* row_gate) {
+  pdl_wait();
+  extern __shared__ uint32_t tw_smem[];
   const int groups = (E + 31) / 32;
-  float sum = 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* s_x = tw_smem + (size_t)warp * groups * 32;  // [groups * 32]: finalT[e][w] of this warp's word
+  uint32_t* s_y = tw_smem + (size_t)(kTwThreads / 32) * groups * 32;  // [groups][kTwThreads]: token masks
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int w = t >> 5;
+  const bool live = t < T;
+  const float* pr = probs + (size_t)(live ? t : 0) * E;
+  // the warp's word of every expert first (independent loads in flight),
+  // then one transpose per group of 32 experts
   for (int g = 0; g < groups; ++g) {
-    const uint32_t m = tr_token_mask(finalT, E, W, t >> 5, g, lane);
-    if (live)
-      for (uint32_t r = m; r; r &= r - 1u) sum += pr[32 * g + __ffs(r) - 1];
+    const int e = 32 * g + lane;
+    s_x[32 * g + lane] = (e < E && w < W) ? finalT[(size_t)e * W + w] : 0u;
+  }
+  __syncwarp();
+  for (int g = 0; g < groups; ++g) s_y[g * kTwThreads + threadIdx.x] = transpose32(s_x[32 * g + lane], lane);
+  __syncwarp();
+  if (!live) return;
+  // the token's final experts in ascending order; the first kTwList of them
+  // have their p, segment offset and row prefix loaded together
+  uint32_t* s_e = s_y + (size_t)groups * kTwThreads;  // [kTwList][kTwThreads]
+  int n = 0;
+  for (int g = 0; g < groups; ++g)
+    for (uint32_t r = s_y[g * kTwThreads + threadIdx.x]; r; r &= r - 1u) {
+      if (n < kTwList) s_e[n * kTwThreads + threadIdx.x] = 32 * g + __ffs(r) - 1;
+      ++n;
+    }
+  float pv[kTwList];
+  int ro[kTwList];
+#pragma unroll
+  for (int j = 0; j < kTwList; ++j) {
+    pv[j] = 0.f;
+    ro[j] = 0;
+    if (j < n) {
+      const int e = s_e[j * kTwThreads + threadIdx.x];
+      pv[j] = pr[e];
+      ro[j] = offsets[e] + rowpre[(size_t)e * W + w];
+    }
+  }
+  float sum = 0.f;  // in ascending expert order
+#pragma unroll
+  for (int j = 0; j < kTwList; ++j)
+    if (j < n) sum += pv[j];
+  if (n > kTwList) {  // the rest, one at a time
+    int i = 0;
+    for (int g = 0; g < groups; ++g)
+      for (uint32_t r = s_y[g * kTwThreads + threadIdx.x]; r; r &= r - 1u, ++i)
+        if (i >= kTwList) sum += pr[32 * g + __ffs(r) - 1];
   }
   const float inv = sum > 0.f ? 1.0f / sum : 0.f;
-  for (int g = 0; g < groups; ++g) {
-    const uint32_t m = tr_token_mask(finalT, E, W, t >> 5, g, lane);
-    if (live)
-      for (uint32_t r = m; r; r &= r - 1u) {
-        const int e = 32 * g + __ffs(r) - 1;
+  int p = blk[t >> 8] + local[t];
+  tok_ptr[t] = p;
+  if (t == T - 1) tok_ptr[T] = blk[nblk];
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kTwList; ++j) {
+    if (j < n) {
+      const int e = s_e[j * kTwThreads + threadIdx.x];
+      const float gate = pv[j] * inv;
+      const int row = ro[j] + __popc(s_x[e] & below);
+      pair_expert[p] = e;
+      pair_gate[p] = gate;
+      pair_row[p] = row;
+      row_tok[row] = t;
+      row_gate[row] = gate;
+      ++p;
+    }
+  }
+  if (n > kTwList) {
+    int i = 0;
+    for (int g = 0; g < groups; ++g)
+      for (uint32_t r = s_y[g * kTwThreads + threadIdx.x]; r; r &= r - 1u, ++i) {
+        if (i < kTwList) continue;
+        const int b = __ffs(r) - 1;
+        const int e = 32 * g + b;
+        const float gate = pr[e] * inv;
+        const int row = offsets[e] + rowpre[(size_t)e * W + w] + __popc(s_x[e] & below);
         pair_expert[p] = e;
-        pair_gate[p] = pr[e] * inv;
+        pair_gate[p] = gate;
+        pair_row[p] = row;
+        row_tok[row] = t;
+        row_gate[row] = gate;
         ++p;
       }
   }
 }
-
-constexpr size_t kTrStageMax = 200 * 1024;  // dynamic shared memory of the staged select
 
 cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStream_t s) {
   const int W = (r.T + 31) / 32;
@@ -596,7 +954,8 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
   const int tb = (r.T + 255) / 256;
   {
     ProfScope ps(s, "round_member");
-    launch_pdl(tr_member_kernel, dim3(tb), dim3(256), 0, s, a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.sync);
+    launch_pdl(tr_member_kernel, dim3(tb), dim3(256), 0, s, a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.local,
+               r.sync);
   }
   {
     ProfScope ps(s, "round_transpose");
@@ -605,30 +964,33 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
   }
   {
     ProfScope ps(s, "round_select");
-    // stage the expert's p row and candidate mask when they fit in shared memory
-    const size_t staged = ((size_t)r.T + (size_t)W) * sizeof(uint32_t);
-    if (staged <= kTrStageMax) {
-      err = set_max_dynamic_smem(reinterpret_cast<const void*>(tr_select_kernel<true>), (int)kTrStageMax);
+    // stage the expert's keys and routed-token words when they fit
+    const size_t staged = kTrSelFixed + ((size_t)((r.T + 3) & ~3) + (size_t)W) * sizeof(uint32_t);
+    if (staged <= kTrSelMax) {
+      err = set_max_dynamic_smem(reinterpret_cast<const void*>(tr_select_kernel<true>), (int)kTrSelMax);
       if (err != cudaSuccess) return err;
-      launch_pdl(tr_select_kernel<true>, dim3(r.E), dim3(1024), staged, s, r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
-                                                        r.finalT);
+      launch_pdl(tr_select_kernel<true>, dim3(r.E), dim3(kTrSelThreads), staged, s, r.T, W, r.mode, r.seed, a.counts,
+                 r.probsT, r.memberT, r.finalT, r.rowpre, r.local);
     } else {
-      launch_pdl(tr_select_kernel<false>, dim3(r.E), dim3(1024), 0, s, r.T, W, r.mode, r.seed, a.counts, r.probsT, r.memberT,
-                                                    r.finalT);
+      launch_pdl(tr_select_kernel<false>, dim3(r.E), dim3(kTrSelThreads), kTrSelFixed, s, r.T, W, r.mode, r.seed,
+                 a.counts, r.probsT, r.memberT, r.finalT, r.rowpre, r.local);
     }
   }
   {
-    ProfScope ps(s, "round_count");
-    launch_pdl(tr_count_kernel, dim3(tb), dim3(256), 0, s, r.finalT, r.T, r.E, W, r.local, r.blk, r.sync);
+    ProfScope ps(s, "round_scan");
+    launch_pdl(tr_scan_kernel, dim3(tb), dim3(256), 0, s, r.T, r.E, r.local, r.blk, r.sync, a.counts, a.offsets,
+               a.tile_expert);
   }
   {
     ProfScope ps(s, "round_write");
-    launch_pdl(tr_write_kernel, dim3(tb), dim3(256), 0, s, r.finalT, r.probs, r.T, r.E, W, r.local, r.blk, a.tok_ptr, a.pair_expert,
-                                       a.pair_gate);
+    const int groups = (r.E + 31) / 32;
+    const size_t smem = ((size_t)(kTwThreads + kTwThreads) * groups + (size_t)kTwList * kTwThreads) *
+                        sizeof(uint32_t);  // at most 20 KB
+    launch_pdl(tr_write_kernel, dim3((r.T + kTwThreads - 1) / kTwThreads), dim3(kTwThreads), smem, s, r.finalT,
+               r.rowpre, r.probs, r.T, r.E, W, r.local, r.blk, tb, a.offsets, a.tok_ptr, a.pair_expert, a.pair_gate,
+               a.pair_row, a.row_tok, a.row_gate);
   }
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  return launch_permute(a, s);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -91,11 +91,17 @@ def test_expert_only_gradient_without_router_path():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("mode,T", [(1, 2048), (2, 2048), (2, 53248)])
-def test_token_rounding_parity(mode, T):
-    """T = 53248: an expert's column of p no longer fits in shared memory, so
-    the selection reads it from global memory in every pass."""
-    cfg = MoEConfig("tr", T=T, d=128, E=16, n=64, K=2, w_std=0.05, bias="normal", seed=21)
+@pytest.mark.parametrize("mode,T,E,K,wr_std", [(1, 2048, 16, 2, 0.02), (2, 2048, 16, 2, 0.02), (2, 53248, 16, 2, 0.02),
+                                                (2, 16384, 512, 8, 0.02), (1, 4096, 130, 4, 0.02),
+                                                (2, 6000, 8, 2, 0.0)])
+def test_token_rounding_parity(mode, T, E, K, wr_std):
+    """E = 512 and 130: several groups of 32 experts per token in the pair
+    writer.  wr_std = 0 (no bias): every p is exactly 1 / E, so each expert's
+    candidates share one histogram bin, more than the sorted list holds, and
+    the selection falls back to radix passes over all candidates; the ties
+    are then broken by token index alone."""
+    cfg = MoEConfig("tr", T=T, d=128, E=E, n=64, K=K, w_std=0.05, wr_std=wr_std,
+                    bias="normal" if wr_std > 0 else "none", seed=21)
     seed = 1234
     inp = make_inputs(cfg, "cuda")
     layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=mode, seed=seed)
