@@ -355,19 +355,51 @@ __global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int
   for (int p = p0; p < p1; ++p) atomicOr(&memberT[(size_t)pair_expert[p] * W + (t >> 5)], 1u << (t & 31));
 }
 
-// probsT[e, t] = probs[t, e], 32 x 32 tiles through shared memory
-__global__ void tr_transpose_kernel(const float* __restrict__ probs, float* __restrict__ probsT, int T, int E) {
+// probsT[e, t] = probs[t, e] through shared memory, 64 x 64 tiles (256
+// threads; float4 loads and stores where E and T are multiples of 4, the
+// rows then being 16-byte aligned).
+constexpr int kTrTile = 64;
+__global__ void __launch_bounds__(256) tr_transpose_kernel(const float* __restrict__ probs, float* __restrict__ probsT,
+                                                          int T, int E) {
   pdl_wait();
-  __shared__ float tile[32][33];
-  const int e0 = blockIdx.x * 32, t0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int t = t0 + i, e = e0 + threadIdx.x;
-    if (t < T && e < E) tile[i][threadIdx.x] = probs[(size_t)t * E + e];
+  __shared__ float tile[kTrTile][kTrTile + 1];
+  const int e0 = blockIdx.x * kTrTile, t0 = blockIdx.y * kTrTile;
+  const int c4 = (threadIdx.x & 15) * 4;  // 4 consecutive columns of the tile
+  const int r0 = threadIdx.x >> 4;        // rows r0, r0 + 16, r0 + 32, r0 + 48
+  const bool vec = ((E | T) & 3) == 0;
+  float v[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // tokens t0 + r, experts e0 + c4 .. + 3
+    const int t = t0 + r0 + 16 * i, e = e0 + c4;
+    if (vec && t < T && e + 3 < E) {
+      const float4 f = *reinterpret_cast<const float4*>(probs + (size_t)t * E + e);
+      v[i][0] = f.x;
+      v[i][1] = f.y;
+      v[i][2] = f.z;
+      v[i][3] = f.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[i][j] = (t < T && e + j < E) ? probs[(size_t)t * E + e + j] : 0.f;
+    }
   }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tile[r0 + 16 * i][c4 + j] = v[i][j];
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int e = e0 + i, t = t0 + threadIdx.x;
-    if (t < T && e < E) probsT[(size_t)e * T + t] = tile[threadIdx.x][i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // experts e0 + r, tokens t0 + c4 .. + 3
+    const int e = e0 + r0 + 16 * i, t = t0 + c4;
+    float o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = tile[c4 + j][r0 + 16 * i];
+    if (vec && e < E && t + 3 < T) {
+      *reinterpret_cast<float4*>(probsT + (size_t)e * T + t) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (e < E && t + j < T) probsT[(size_t)e * T + t + j] = o[j];
+    }
   }
 }
 
@@ -405,9 +437,10 @@ __device__ int block_exclusive_scan(int v, int* sh, int* total) {
 // up (largest p first, ties: smaller t first).  Keys are distinct, so "key <=
 // the k-th smallest" selects exactly k tokens.
 //
-// The expert's candidate words and 32-bit p keys are first staged in shared
-// memory (when its row fits) with many loads in flight per thread, and each
-// thread takes the smallest key among its own candidates on the way.  The
+// The expert's candidate words are staged in shared memory (when they fit);
+// its p row is read from L2 four tokens per load with several loads in
+// flight per thread.  Each thread keeps the four smallest keys among its own
+// candidates; the
 // k-th smallest of these per-thread minima, tau, bounds the k-th smallest
 // key from above (k threads each hold a candidate <= tau), so only the
 // candidates <= tau -- about k of them when the candidates are spread over
@@ -420,16 +453,15 @@ constexpr int kTrSelThreads = 256;  // > the largest k (127)
 constexpr size_t kTrSelFixed = (size_t)256 * 4 + (size_t)kTrListCap * 8;  // radix histogram + list
 constexpr size_t kTrSelMax = 200 * 1024;  // dynamic shared memory of the staged selection, at most
 
-// Candidates and keys of one expert's selection.  STAGED: the keys [T] and
-// candidate words [W] are in shared memory; otherwise they are read from the
-// expert's rows in global memory.
+// Candidates and keys of one expert's selection.  STAGED: the candidate
+// words [W] are in shared memory; otherwise they are read from the expert's
+// row in global memory, like the keys always are.
 template <bool STAGED>
 struct TrSelect {
   int T, W;
   bool up;
   const uint32_t* mrow;    // routed tokens of the expert (global)
   const float* prow;       // p of the expert (global)
-  const uint32_t* s_key;   // STAGED: keys [T]
   const uint32_t* s_cand;  // STAGED: candidate words [W]
   __device__ __forceinline__ uint32_t valid(int w) const {
     return (w == W - 1 && (T & 31)) ? ((1u << (T & 31)) - 1u) : 0xFFFFFFFFu;
@@ -451,12 +483,8 @@ struct TrSelect {
     }
   }
   __device__ __forceinline__ uint32_t key32(int t) const {
-    if constexpr (STAGED) {
-      return s_key[t];
-    } else {
-      const uint32_t pb = __float_as_uint(prow[t]);
-      return up ? ~pb : pb;
-    }
+    const uint32_t pb = __float_as_uint(prow[t]);
+    return up ? ~pb : pb;
   }
   __device__ __forceinline__ unsigned long long key64(int t) const {
     return ((unsigned long long)key32(t) << 32) | (up ? (unsigned)t : (0xFFFFFFFFu - (unsigned)t));
@@ -583,10 +611,10 @@ __device__ __forceinline__ unsigned long long tr_block_sort1(unsigned long long 
 // the expert's final tokens before word w (the rank of a token's row inside
 // the expert's segment is rowpre plus a popcount within its word).
 // STAGED: shared memory holds, after the radix histogram and the list, the
-// expert's keys [T rounded up to 4] and candidate words [W].  Tokens are
-// visited four at a time (one vector load, one candidate nibble).
+// expert's candidate words [W].  Tokens are visited four at a time (one
+// vector load, one candidate nibble).
 template <bool STAGED>
-__global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
+__global__ void __launch_bounds__(kTrSelThreads, 4) tr_select_kernel(int T, int W, int mode, unsigned long long seed,
                                                                  int* counts, const float* probsT,
                                                                  const uint32_t* memberT, uint32_t* finalT,
                                                                  int* rowpre, int* tok_count) {
@@ -595,8 +623,7 @@ __global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, 
   unsigned* hist = reinterpret_cast<unsigned*>(tr_smem);                                 // [256]
   unsigned long long* list = reinterpret_cast<unsigned long long*>(tr_smem + 256 * 4);  // [kTrListCap]
   const int T4 = (T + 3) & ~3;
-  uint32_t* s_key = reinterpret_cast<uint32_t*>(tr_smem + kTrSelFixed);  // STAGED: [T4]
-  uint32_t* s_cand = s_key + T4;                                         // STAGED: [W]
+  uint32_t* s_cand = reinterpret_cast<uint32_t*>(tr_smem + kTrSelFixed);  // STAGED: [W]
   __shared__ int sh[32];
   __shared__ int s_cnt;
   __shared__ unsigned long long s_thr;
@@ -619,7 +646,6 @@ __global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, 
   s.up = up;
   s.mrow = memberT + (size_t)e * W;
   s.prow = probsT + (size_t)e * T;
-  s.s_key = s_key;
   s.s_cand = s_cand;
   const bool vec = (T & 3) == 0;  // the row is 16-byte aligned: float4 loads
   auto tie = [&](int t) -> unsigned long long { return up ? (unsigned)t : (0xFFFFFFFFu - (unsigned)t); };
@@ -645,8 +671,32 @@ __global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, 
   };
   auto nibble = [&](int q) -> uint32_t { return (s.cand_word(q >> 3) >> ((4 * q) & 31)) & 0xFu; };
   const int Q = T4 / 4;
-  // 1. staging (STAGED) and each thread's smallest candidate key
-  unsigned long long mn = ~0ull;
+  // 1. the candidate words staged (STAGED); each thread's four smallest
+  // candidate keys (m[0] <= .. <= m[3], ~0 past its count cnt)
+  unsigned long long m[4] = {~0ull, ~0ull, ~0ull, ~0ull};
+  uint32_t m3hi = 0xFFFFFFFFu;  // high word of m[3]: keys above it are rejected with one compare
+  int cnt = 0;
+  auto keep = [&](unsigned long long x) {
+    if (x < m[3]) {
+      if (x < m[2]) {
+        m[3] = m[2];
+        if (x < m[1]) {
+          m[2] = m[1];
+          if (x < m[0]) {
+            m[1] = m[0];
+            m[0] = x;
+          } else {
+            m[1] = x;
+          }
+        } else {
+          m[2] = x;
+        }
+      } else {
+        m[3] = x;
+      }
+      m3hi = (uint32_t)(m[3] >> 32);
+    }
+  };
   if constexpr (STAGED) {
     for (int w = threadIdx.x; w < W; w += nthr) {
       const uint32_t m = s.mrow[w];
@@ -655,53 +705,60 @@ __global__ void __launch_bounds__(kTrSelThreads) tr_select_kernel(int T, int W, 
     __syncthreads();
   }
   if (k > 0) {
-    for (int q = threadIdx.x; q < Q; q += nthr) {
-      uint32_t kq[4];
-      load_quad(q, kq);
-      if constexpr (STAGED) *reinterpret_cast<uint4*>(s_key + 4 * q) = make_uint4(kq[0], kq[1], kq[2], kq[3]);
-      const uint32_t nb = nibble(q);
+    constexpr int kBatch = 4;  // quads per thread whose loads are in flight together
+    for (int q0 = threadIdx.x; q0 < Q; q0 += kBatch * nthr) {
+      uint32_t kq[kBatch][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if ((nb >> j) & 1u) {
-          const unsigned long long x = ((unsigned long long)kq[j] << 32) | tie(4 * q + j);
-          mn = x < mn ? x : mn;
+      for (int u = 0; u < kBatch; ++u)
+        if (q0 + u * nthr < Q) load_quad(q0 + u * nthr, kq[u]);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + u * nthr;
+        if (q < Q) {
+          const uint32_t nb = nibble(q);
+          cnt += __popc(nb);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (((nb >> j) & 1u) && kq[u][j] <= m3hi) keep(((unsigned long long)kq[u][j] << 32) | tie(4 * q + j));
         }
+      }
     }
   }
-  if constexpr (STAGED) __syncthreads();
   unsigned long long thr = 0ull;
   bool listed = false;  // the selected tokens are the list entries <= thr
   int len = 0;
   if (k > 0) {
     // 2. tau: the k-th smallest thread minimum (k < 128 <= nthr)
-    const unsigned long long r = tr_block_sort1(mn, list);
+    const unsigned long long r = tr_block_sort1(m[0], list);
     if (threadIdx.x == k - 1) s_thr = r;
     if (threadIdx.x == 0) s_cnt = 0;
     __syncthreads();
     const unsigned long long tau = s_thr;
-    // 3. the candidates <= tau; the k-th smallest of them is the k-th key
-    for (int q = threadIdx.x; q < Q; q += nthr) {
-      const uint32_t nb = nibble(q);
-      if (nb == 0u) continue;
-      uint32_t kq[4];
-      if constexpr (STAGED) {
-        const uint4 u = *reinterpret_cast<const uint4*>(s_key + 4 * q);
-        kq[0] = u.x;
-        kq[1] = u.y;
-        kq[2] = u.z;
-        kq[3] = u.w;
-      } else {
+    // 3. the candidates <= tau; the k-th smallest of them is the k-th key.
+    // A thread's kept keys hold all of its candidates <= tau unless it saw
+    // more than four and its fourth is <= tau; only then does it read its
+    // tokens again.
+    auto push = [&](unsigned long long x) {
+      const int i = atomicAdd(&s_cnt, 1);
+      if (i < kTrListCap) list[i] = x;
+    };
+    if (cnt > 4 && m[3] <= tau) {
+      for (int q = threadIdx.x; q < Q; q += nthr) {
+        const uint32_t nb = nibble(q);
+        if (nb == 0u) continue;
+        uint32_t kq[4];
         load_quad(q, kq);
-      }
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if ((nb >> j) & 1u) {
-          const unsigned long long x = ((unsigned long long)kq[j] << 32) | tie(4 * q + j);
-          if (x <= tau) {
-            const int i = atomicAdd(&s_cnt, 1);
-            if (i < kTrListCap) list[i] = x;
+        for (int j = 0; j < 4; ++j)
+          if ((nb >> j) & 1u) {
+            const unsigned long long x = ((unsigned long long)kq[j] << 32) | tie(4 * q + j);
+            if (x <= tau) push(x);
           }
-        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (i < cnt && m[i] <= tau) push(m[i]);
     }
     __syncthreads();
     len = s_cnt;
@@ -959,13 +1016,13 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
   }
   {
     ProfScope ps(s, "round_transpose");
-    dim3 grid((r.E + 31) / 32, (r.T + 31) / 32), block(32, 8);
-    launch_pdl(tr_transpose_kernel, dim3(grid), dim3(block), 0, s, r.probs, r.probsT, r.T, r.E);
+    dim3 grid((r.E + kTrTile - 1) / kTrTile, (r.T + kTrTile - 1) / kTrTile);
+    launch_pdl(tr_transpose_kernel, dim3(grid), dim3(256), 0, s, r.probs, r.probsT, r.T, r.E);
   }
   {
     ProfScope ps(s, "round_select");
     // stage the expert's keys and routed-token words when they fit
-    const size_t staged = kTrSelFixed + ((size_t)((r.T + 3) & ~3) + (size_t)W) * sizeof(uint32_t);
+    const size_t staged = kTrSelFixed + (size_t)W * sizeof(uint32_t);
     if (staged <= kTrSelMax) {
       err = set_max_dynamic_smem(reinterpret_cast<const void*>(tr_select_kernel<true>), (int)kTrSelMax);
       if (err != cudaSuccess) return err;
