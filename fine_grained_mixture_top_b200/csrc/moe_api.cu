@@ -523,6 +523,9 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
     ProfScope ps(st, "router_softmax_topk");
     MOE_TRY_CUDA(launch_softmax_topk(a, st));
   }
+  // with token rounding to follow, the permutation is left to moe_token_round
+  // (it rebuilds counts, segments and rows from the rounded expert sets)
+  if (opts->round_mode != 0) return MOE_OK;
   MOE_TRY_CUDA(launch_permute(a, st));
   MOE_VALIDATE(p, rt, status, st);
   return MOE_OK;

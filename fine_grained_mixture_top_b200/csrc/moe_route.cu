@@ -343,16 +343,31 @@ __device__ __forceinline__ unsigned long long splitmix64_dev(unsigned long long 
 // Token rounding works on per-expert rows: memberT[e][w] holds bit t & 31 of
 // word w = t / 32 for each token t routed to e, probsT[e][t] = p[t, e].  One
 // block per expert then reads its row contiguously.  tr_member also records
-// each token's pair count, which the selection adjusts token by token.
-__global__ void tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int W, uint32_t* memberT,
-                                 int* tok_count, int* sync) {
+// each token's pair count, which the selection adjusts token by token, and
+// counts each expert's routed tokens (counts zeroed before the launch): per
+// block in shared memory, then one global add per block and expert (a hot
+// expert's count would otherwise take thousands of same-address atomics).
+__global__ void __launch_bounds__(256) tr_member_kernel(const int* tok_ptr, const int* pair_expert, int T, int E,
+                                                        int W, uint32_t* memberT, int* tok_count, int* counts,
+                                                        int* sync) {
   pdl_wait();
+  __shared__ int s_cnt[1024];  // E <= 1024
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t == 0) *sync = 0;  // for tr_scan_kernel's last block
-  if (t >= T) return;
-  const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
-  tok_count[t] = p1 - p0;
-  for (int p = p0; p < p1; ++p) atomicOr(&memberT[(size_t)pair_expert[p] * W + (t >> 5)], 1u << (t & 31));
+  if (t < T) {
+    const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
+    tok_count[t] = p1 - p0;
+    for (int p = p0; p < p1; ++p) {
+      const int e = pair_expert[p];
+      atomicOr(&memberT[(size_t)e * W + (t >> 5)], 1u << (t & 31));
+      atomicAdd(&s_cnt[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (s_cnt[e]) atomicAdd(&counts[e], s_cnt[e]);
 }
 
 // probsT[e, t] = probs[t, e] through shared memory, 64 x 64 tiles (256
@@ -1007,12 +1022,13 @@ __global__ void __launch_bounds__(kTwThreads) tr_write_kernel(const uint32_t* fi
 cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStream_t s) {
   const int W = (r.T + 31) / 32;
   cudaError_t err = cudaMemsetAsync(r.memberT, 0, (size_t)r.E * W * sizeof(uint32_t), s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(a.counts, 0, (size_t)r.E * sizeof(int), s);
   if (err != cudaSuccess) return err;
   const int tb = (r.T + 255) / 256;
   {
     ProfScope ps(s, "round_member");
-    launch_pdl(tr_member_kernel, dim3(tb), dim3(256), 0, s, a.tok_ptr, a.pair_expert, r.T, W, r.memberT, r.local,
-               r.sync);
+    launch_pdl(tr_member_kernel, dim3(tb), dim3(256), 0, s, a.tok_ptr, a.pair_expert, r.T, r.E, W, r.memberT,
+               r.local, a.counts, r.sync);
   }
   {
     ProfScope ps(s, "round_transpose");

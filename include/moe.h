@@ -128,6 +128,10 @@ moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes
  *   X[T,d] bf16, Wr[d,E] f32, bias[E] f32 (nullable; added to the logits
  *   before the softmax).  Fills every array of *rt except pair_row's unused
  *   tail.  rt->logits may be NULL (then kept in ws only).
+ *   With opts->round_mode != 0 it stops after the top-K selection (logits,
+ *   probs, topk_idx, topk_gate, tok_ptr, pair_expert, pair_gate): the rounded
+ *   routing replaces the rest, and moe_token_round, which must follow on the
+ *   same stream, builds it.
  */
 moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
                      const float* bias, const moe_routing* rt, void* ws, size_t ws_bytes, void* stream);
@@ -156,7 +160,8 @@ moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe
  * probability; gates become p renormalised over each token's final experts,
  * listed in ascending expert order.  Rewrites tok_ptr, pair_*, counts,
  * offsets, row_*, tile_expert of *rt (topk_idx/topk_gate keep the unrounded
- * selection).  Must follow moe_route on the same stream.
+ * selection).  Must follow moe_route on the same stream; it needs only the
+ * top-K selection of that call (tok_ptr, pair_expert, probs).
  */
 moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
                            size_t ws_bytes, void* stream);
