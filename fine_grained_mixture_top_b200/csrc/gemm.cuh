@@ -399,10 +399,17 @@ __device__ __forceinline__ void issue_tma(const GemmParams& p, const TileInfo& t
     tma_load_2d(b_s, tB, bar_a, x, t.e * p.d + t.n0);
     bulk_load(sfb_s, p.sfb_src + ((size_t)(t.e * (p.d / 128) + t.nt) * (p.n / 128) + kb) * 512, 512, bar_a);
   } else if constexpr (KIND == G_RTR) {
+    // Wr column box j = (group j / 3, part j % 3: hi, mid, lo) goes to slot
+    // [hi of every group | mid, lo of group 0 | mid, lo of group 1 ...], so
+    // that one MMA covers every group's hi part and one every mid and lo part
+    constexpr int G = BN / 192;
     expect_a(kABytes);
     tma_load_2d(a_s, tA, bar_a, k0, t.m0);
     expect_b(nb * kBoxBytes);
-    for (int j = 0; j < nb; ++j) tma_load_2d(b_s + j * kBoxBytes, tB, bar_b, t.n0 + 64 * j, k0);
+    for (int j = 0; j < nb; ++j) {
+      const int pos = (j % 3 == 0) ? j / 3 : G + 2 * (j / 3) + (j % 3 - 1);
+      tma_load_2d(b_s + pos * kBoxBytes, tB, bar_b, t.n0 + 64 * j, k0);
+    }
   } else {  // G_DWR
     expect_a(2 * kBoxBytes);
     for (int h = 0; h < 2; ++h) tma_load_2d(a_s + h * kBoxBytes, tA, bar_a, t.m0 + 64 * h, t.krow0 + k0);
@@ -505,8 +512,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
   int4* tq_info = reinterpret_cast<int4*>(bars + 50);
   auto a_slot = [&](int i) -> uint32_t { return base + SH::kAOffset + (uint32_t)(i * kABytes); };
   auto b_slot = [&](int i) -> uint32_t { return base + SH::kBOffset + (uint32_t)(i * SH::kBBytes); };
-  // the router-logit kind keeps one tile buffer of 256 columns: [hi_a | hi_b | mid | lo]
-  constexpr int kTmemCols = (KIND == G_RTR) ? 256 : SH::kTmemCols;
+  // the router-logit kind covers G = BN / 192 groups of 64 experts per tile
+  // in 256 G TMEM columns: two alternating hi slots of 64 G columns (every
+  // group's hi part), then each group's mid and lo (128 columns per group)
+  constexpr int kRtrG = (KIND == G_RTR) ? BN / 192 : 1;
+  constexpr int kTmemCols = (KIND == G_RTR) ? 256 * kRtrG : SH::kTmemCols;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -679,8 +689,8 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     // k-blocks into two alternating TMEM slots; the epilogue adds every group
     // into fp32 registers, so the tensor core's long accumulation chain is cut
     // into short ones.  The mid and lo parts accumulate over the whole K.
-    constexpr uint32_t kIdescHi = idesc_bf16_f32(64, KT::kAMN, KT::kBMN);
-    constexpr uint32_t kIdescMl = idesc_bf16_f32(128, KT::kAMN, KT::kBMN);
+    constexpr uint32_t kIdescHi = idesc_bf16_f32(64 * kRtrG, KT::kAMN, KT::kBMN);
+    constexpr uint32_t kIdescMl = idesc_bf16_f32(128 * kRtrG, KT::kAMN, KT::kBMN);
     int it = 0, tcount = 0, hg = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
@@ -718,9 +728,9 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(a_s + kk * 32, 16, 1024);
             const uint64_t bhi = smem_desc_sw128(b_s + kk * 2048, kBoxBytes, 1024);
-            const uint64_t bml = smem_desc_sw128(b_s + kBoxBytes + kk * 2048, kBoxBytes, 1024);
-            tc_mma_bf16(tmem_base + (uint32_t)(slot * 64), ad, bhi, kIdescHi, (first && kk == 0) ? 0u : 1u);
-            tc_mma_bf16(tmem_base + 128u, ad, bml, kIdescMl, (kb > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bml = smem_desc_sw128(b_s + kRtrG * kBoxBytes + kk * 2048, kBoxBytes, 1024);
+            tc_mma_bf16(tmem_base + (uint32_t)(slot * 64 * kRtrG), ad, bhi, kIdescHi, (first && kk == 0) ? 0u : 1u);
+            tc_mma_bf16(tmem_base + (uint32_t)(128 * kRtrG), ad, bml, kIdescMl, (kb > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(smem_u32(&empty_a[sa]));
           if (kSplit) tc_commit(smem_u32(&empty_b[sb]));
@@ -815,9 +825,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       TileInfo t;
       const int tile = consume_tile(ti, ok, t);
       if (!ok || tile >= num_tiles) break;
-      float hs[64];
+      float hs[kRtrG][64];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) hs[i] = 0.f;
+      for (int g = 0; g < kRtrG; ++g)
+#pragma unroll
+        for (int i = 0; i < 64; ++i) hs[g][i] = 0.f;
       const int ngroups = (t.nkb + kRtrGroup - 1) / kRtrGroup;
       for (int grp = 0; grp < ngroups; ++grp, ++hg) {
         const int slot = hg & 1;
@@ -826,14 +838,17 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
           break;
         }
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_addr + slot * 64, r0);
-        tmem_ld32(lane_addr + slot * 64 + 32, r1);
-        tc_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          hs[i] += __uint_as_float(r0[i]);
-          hs[32 + i] += __uint_as_float(r1[i]);
+        for (int g = 0; g < kRtrG; ++g) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(lane_addr + slot * 64 * kRtrG + 64 * g, r0);
+          tmem_ld32(lane_addr + slot * 64 * kRtrG + 64 * g + 32, r1);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            hs[g][i] += __uint_as_float(r0[i]);
+            hs[g][32 + i] += __uint_as_float(r1[i]);
+          }
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&hi_empty[slot]));
@@ -844,21 +859,23 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
       // each warp's 32 rows x 32 logits go through shared memory (padded
       // rows, conflict-free both ways) and leave as 128-byte row pieces
       float* stg = reinterpret_cast<float*>(smem + SH::kStoreOffset + (warp - 2) * (EC::kBufs * kStoreBuf));
-#pragma unroll 1
-      for (int c = 0; c < 64; c += 32) {
+#pragma unroll
+      for (int gc = 0; gc < 2 * kRtrG; ++gc) {  // 32 columns of group gc / 2 at a time
+        const int g = gc >> 1, c = 32 * (gc & 1);
         uint32_t mid[32], lo[32];
-        tmem_ld32(lane_addr + 128 + c, mid);
-        tmem_ld32(lane_addr + 192 + c, lo);
+        tmem_ld32(lane_addr + 128 * kRtrG + 128 * g + c, mid);
+        tmem_ld32(lane_addr + 128 * kRtrG + 128 * g + 64 + c, lo);
         tc_wait_ld();
+        const int e0 = (t.nt * kRtrG + g) * 64 + c;  // first expert of these columns
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int e = t.nt * 64 + c + i;
-          float z = (c == 0 ? hs[i] : hs[32 + i]) + (__uint_as_float(mid[i]) + __uint_as_float(lo[i]));
+          const int e = e0 + i;
+          float z = hs[g][c + i] + (__uint_as_float(mid[i]) + __uint_as_float(lo[i]));
           if (p.bias && e < p.E) z += __ldg(p.bias + e);
           stg[lane * 33 + i] = z;
         }
         __syncwarp();
-        const int e = t.nt * 64 + c + lane;
+        const int e = e0 + lane;
 #pragma unroll 4
         for (int r = 0; r < 32; ++r) {
           const int trow = t.m0 + q * 32 + r;

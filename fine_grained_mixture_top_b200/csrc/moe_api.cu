@@ -510,13 +510,16 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
   GemmParams g = base_params(p, rt, status);
   MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
   MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
+  // one tile covers both groups of 64 experts where E <= 128 (TMEM holds two
+  // groups' hi slots and mid/lo accumulators), so X is read once per row tile
+  const int bn_rtr = p.Epad == 128 ? 384 : 192;
   g.num_m_tiles = (int)cdiv(p.T, 128);
-  g.num_n_tiles = p.Epad / 64;
+  g.num_n_tiles = 3 * p.Epad / bn_rtr;
   g.outf = const_cast<float*>(a.logits);
   g.bias = bias;
   {
     ProfScope ps(st, "router_logits_gemm");
-    MOE_TRY_CUDA(launch_gemm(G_RTR, 192, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+    MOE_TRY_CUDA(launch_gemm(G_RTR, bn_rtr, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
   }
 
   {
@@ -1249,11 +1252,12 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* op
   GemmParams g = base_params(p, rt, status);
   MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
   MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
+  const int bn_rtr = p.Epad == 128 ? 384 : 192;  // as in moe_route
   g.num_m_tiles = (int)cdiv(p.T, 128);
-  g.num_n_tiles = p.Epad / 64;
+  g.num_n_tiles = 3 * p.Epad / bn_rtr;
   g.outf = rt->logits;
   g.bias = bias;
-  MOE_TRY_CUDA(launch_gemm(G_RTR, 192, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
+  MOE_TRY_CUDA(launch_gemm(G_RTR, bn_rtr, 4, g, grid_for((int64_t)g.num_m_tiles * g.num_n_tiles, sms), st));
   MOE_TRY_CUDA(launch_softmax_topk(a, st));
   MOE_TRY_CUDA(launch_permute(a, st));
   MOE_VALIDATE(p, rt, status, st);

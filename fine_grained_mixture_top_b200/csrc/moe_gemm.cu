@@ -182,6 +182,7 @@ cudaError_t launch_gemm(int kind, int bn, int epi, const GemmParams& p_in, int g
   MOE_CASE(G_UPQ, 128, 4)
   MOE_CASE(G_DOWNQ, 128, 4)
   MOE_CASE(G_RTR, 192, 4)
+  MOE_CASE(G_RTR, 384, 4)
   MOE_CASE(G_DWR, 128, 4)
 #undef MOE_CASE
   return cudaErrorInvalidValue;
