@@ -133,7 +133,7 @@ def measured_traffic(kernel, workload_key):
         return None
     with open(path) as f:
         data = json.load(f)
-    rec = data.get(kernel)
+    rec = data.get(f"{kernel}@{workload_key}") or data.get(kernel)  # one record per kernel and workload
     if not rec or rec.get("src_digest") != source_digest() or rec.get("workload") != workload_key:
         return None
     return rec.get("dram_bytes_per_launch")

@@ -66,7 +66,8 @@ struct GemmParams {
   const float* bias;
   int* sched;                // weight-gradient kinds: zeroed 64-bit tile counter (8-byte aligned)
   const int* expert_order;   // weight-gradient kinds: experts by descending token count
-  int dual_ended;            // weight-gradient kinds: odd CTAs claim from the smallest experts' end
+  int dual_ended;            // weight-gradient kinds: 0 every claim from the largest experts' end; 1 odd
+                             // CTAs claim from the smallest experts' end; 2 every CTA alternates ends
   // grouped-M kinds: the 128-row M tiles to run, [count, tile...], or null
   // for all of them (the pair kernel's list: the first of each pair of tiles)
   const int* mlist;
@@ -570,28 +571,35 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
 
   // Tile order.  Static kinds walk tiles round-robin.  The weight-gradient
   // kinds, whose tiles differ in length with the expert's token count, take
-  // tiles dynamically from a list ordered by expert, largest first: even CTAs
-  // claim from its front (the long, L2-bound tiles of the busiest experts),
-  // odd CTAs from its back (the short tiles of the smallest experts, bound by
-  // storing their results), so that both kinds of work run at once and the
-  // last tiles taken are the middle-sized ones.  One 64-bit counter holds
-  // both ends (front claims in the low word, back claims in the high word);
-  // claim k (the sum of both before the increment) is valid iff k < tiles.
-  // The TMA thread claims a tile one tile ahead (the atomic's latency hides
-  // behind the current tile's loads), resolves its expert once, and hands it
-  // to the other roles through a shared-memory queue.
+  // tiles dynamically from a list ordered by expert, largest first.  Claims
+  // come from both ends of the list: the front holds the long, L2-bound tiles
+  // of the busiest experts, the back the short tiles of the smallest experts,
+  // bound by storing their results.  With dual_ended = 1, even CTAs claim from
+  // the front and odd CTAs from the back, so both kinds run at once on
+  // different SMs; with 2, every CTA takes its first tile from the front and
+  // then alternates ends, so that a short tile's stores run under the next
+  // long tile's main loop on the same SM.  One 64-bit counter holds both ends
+  // (front claims in the low word, back claims in the high word); claim k
+  // (the sum of both before the increment) is valid iff k < tiles, and the
+  // last tiles taken are the middle-sized ones.  The TMA thread claims a tile
+  // one tile ahead (the atomic's latency hides behind the current tile's
+  // loads), resolves its expert once, and hands it to the other roles through
+  // a shared-memory queue.
   constexpr bool kDyn = KT::kGroupedK;
-  const bool front_end = !p.dual_ended || (blockIdx.x & 1u) == 0u;
-  const int nfront0 = p.dual_ended ? ((int)gridDim.x + 1) / 2 : (int)gridDim.x;  // first tiles, taken unclaimed
+  const bool alternate = p.dual_ended == 2;
+  const bool front_cta = p.dual_ended != 1 || (blockIdx.x & 1u) == 0u;
+  // the end that claim i (the claim of this CTA's tile i >= 1) takes
+  auto front_of = [&](int i) -> bool { return alternate ? (i & 1) == 0 : front_cta; };
+  const int nfront0 = p.dual_ended == 1 ? ((int)gridDim.x + 1) / 2 : (int)gridDim.x;  // first tiles, unclaimed
   const int nback0 = (int)gridDim.x - nfront0;
-  auto claim = [&]() -> unsigned long long {
-    return atomicAdd(reinterpret_cast<unsigned long long*>(p.sched), front_end ? 1ull : (1ull << 32));
+  auto claim = [&](bool front) -> unsigned long long {
+    return atomicAdd(reinterpret_cast<unsigned long long*>(p.sched), front ? 1ull : (1ull << 32));
   };
-  auto claimed_tile = [&](unsigned long long old) -> int {
+  auto claimed_tile = [&](unsigned long long old, bool front) -> int {
     const int f = (int)(old & 0xffffffffull) + nfront0;
     const int b = (int)(old >> 32) + nback0;
     if (f + b >= num_tiles) return num_tiles;
-    return front_end ? f : num_tiles - 1 - b;
+    return front ? f : num_tiles - 1 - b;
   };
   unsigned long long next_claim = 0;
   int res_ei = -1, res_e = 0, res_krow0 = 0, res_nkb = 0;  // the producer's last resolved expert
@@ -599,12 +607,12 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     if constexpr (kDyn) {
       int tile;
       if (i == 0) {
-        const int j = p.dual_ended ? ((int)blockIdx.x >> 1) : (int)blockIdx.x;
-        tile = front_end ? j : num_tiles - 1 - j;
+        const int j = p.dual_ended == 1 ? ((int)blockIdx.x >> 1) : (int)blockIdx.x;
+        tile = front_cta ? j : num_tiles - 1 - j;
       } else {
-        tile = claimed_tile(next_claim);
+        tile = claimed_tile(next_claim, front_of(i));
       }
-      if (tile < num_tiles) next_claim = claim();  // the next tile's claim, in flight meanwhile
+      if (tile < num_tiles) next_claim = claim(front_of(i + 1));  // the next tile's claim, in flight meanwhile
       int e = 0, krow0 = 0, nkb = 0;
       if (tile < num_tiles) {
         const int ei = tile / (p.num_m_tiles * p.num_n_tiles);

@@ -9,6 +9,10 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <tuple>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -118,7 +122,8 @@ struct Plan {
   int nds;  // dS partials per row: N tiles x column parts of the dH epilogue
   int epi_dh, epi_dxt;  // epilogue warps of the dH and dX~ kernels
   int epi_dw;           // epilogue warps of the weight-gradient kernels
-  int dw_dual;          // weight-gradient tiles claimed from both ends of the expert order
+  int dw_dual;          // weight-gradient tile claims: 0 largest experts first, 1 from both ends by CTA parity,
+                        // 2 every CTA alternating ends
   int dw1_pair, dw2_pair;  // weight-gradient GEMMs on CTA pairs (256 x 256 tiles)
   int gm_pair;             // down-proj and dX~ on CTA pairs (256 x 256 tiles of two M tiles)
   int ksplit, ksplit_rows;
@@ -168,13 +173,16 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   // expert (at most 8 k-blocks on average) a tile is bound by storing its
   // 128 x BN result, so the epilogue gets 8 warps.
   p.epi_dw = (T * K / E <= 8 * 64) ? 8 : 4;
-  p.dw_dual = 1;
+  p.dw_dual = 2;  // every CTA alternates ends: short tiles' stores run under long tiles' main loops
   // tuning overrides, for measurements: MOE_EPI_DW (4 or 8), MOE_DW_DUAL (0 or 1)
   if (const char* v = std::getenv("MOE_EPI_DW")) {
     const int x = std::atoi(v);
     if (x == 4 || x == 8) p.epi_dw = x;
   }
-  if (const char* v = std::getenv("MOE_DW_DUAL")) p.dw_dual = std::atoi(v) != 0;
+  if (const char* v = std::getenv("MOE_DW_DUAL")) {
+    const int x = std::atoi(v);
+    if (x >= 0 && x <= 2) p.dw_dual = x;
+  }
   // 256 x 256 pair tiles where both output dimensions are multiples of 256
   // (MOE_DW_PAIR=1 turns them on)
   const bool pair_on = std::getenv("MOE_DW_PAIR") && std::atoi(std::getenv("MOE_DW_PAIR")) != 0;
@@ -192,6 +200,22 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   ks = std::min<int64_t>(ks, cdiv(T, 64));
   p.ksplit_rows = (int)(cdiv(cdiv(T, ks), 64) * 64);
   p.ksplit = (int)cdiv(T, p.ksplit_rows);
+  // MOE_LOG=1: the tile plan of each new shape, once, on stderr
+  if (const char* v = std::getenv("MOE_LOG")) {
+    if (std::atoi(v) != 0) {
+      static std::mutex mu;
+      static std::set<std::tuple<int64_t, int, int, int, int, int>> seen;
+      std::lock_guard<std::mutex> lk(mu);
+      if (seen.insert({T, d, E, n, K, opts->round_mode}).second)
+        std::fprintf(stderr,
+                     "moe plan T=%lld d=%d E=%d n=%d K=%d round=%d: P_max=%lld R_max=%lld; BN up %d down %d dH %d "
+                     "dX~ %d dW1 %d dW2 %d; epilogue warps dH %d dX~ %d dW %d; dW tiles from both ends %d; CTA pairs "
+                     "dW1 %d dW2 %d down/dX~ %d; router tile %d columns; dWr split-K %d x %d rows\n",
+                     (long long)T, d, E, n, K, opts->round_mode, (long long)p.P_max, (long long)p.R_max, p.bn_up,
+                     p.bn_down, p.bn_dh, p.bn_dxt, p.bn_dw1, p.bn_dw2, p.epi_dh, p.epi_dxt, p.epi_dw, p.dw_dual,
+                     p.dw1_pair, p.dw2_pair, p.gm_pair, p.Epad == 128 ? 384 : 192, p.ksplit, p.ksplit_rows);
+    }
+  }
   *pl = p;
   return MOE_OK;
 }
@@ -444,7 +468,11 @@ moe_status cuda_failed(cudaError_t e, int line) {
 }  // namespace
 
 namespace moe {
+ApiRange::ApiRange(const char* name) { nvtxRangePushA(name); }
+ApiRange::~ApiRange() { nvtxRangePop(); }
+
 ProfScope::ProfScope(cudaStream_t s, const char* name) : stream(s) {
+  nvtxRangePushA(name);
   if (!g_prof_on || g_prof_n >= kProfCap) return;
   if (g_prof_only[0] && std::strcmp(g_prof_only, name) != 0) return;
   ProfRec& r = g_prof[g_prof_n];
@@ -458,6 +486,7 @@ ProfScope::ProfScope(cudaStream_t s, const char* name) : stream(s) {
 }
 ProfScope::~ProfScope() {
   if (slot >= 0) cudaEventRecord(g_prof[slot].b, stream);
+  nvtxRangePop();
 }
 }  // namespace moe
 
@@ -485,6 +514,7 @@ moe_status moe_query_sizes(const moe_dims* dims, const moe_opts* opts, moe_sizes
 
 moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr, const float* bias,
                      const moe_routing* rt, void* ws, size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_route");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -536,6 +566,7 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
 
 moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
                            size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_token_round");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -570,6 +601,7 @@ moe_status moe_token_round(const moe_dims* dims, const moe_opts* opts, const moe
 
 moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1, const void* W2,
                        const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_forward");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -718,6 +750,7 @@ extern "C" {
 moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const void* X, const void* W1,
                              const void* W2, const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes,
                              void* stream) {
+  ApiRange api_range("moe_forward_mxfp8");
   if (!W1 || !W2 || !aligned16(W1) || !aligned16(W2)) {
     Plan p;
     const moe_status s = make_plan(dims, opts, &p);
@@ -738,6 +771,7 @@ moe_status moe_forward_mxfp8(const moe_dims* dims, const moe_opts* opts, const v
 
 moe_status moe_mx_quantize_weights(const moe_dims* dims, const moe_opts* opts, const void* W1, const void* W2,
                                    void* wq, size_t wq_bytes, void* stream) {
+  ApiRange api_range("moe_mx_quantize_weights");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -758,6 +792,7 @@ moe_status moe_mx_quantize_weights(const moe_dims* dims, const moe_opts* opts, c
 
 moe_status moe_forward_mxfp8_q(const moe_dims* dims, const moe_opts* opts, const void* X, const void* wq,
                                const moe_routing* rt, void* O, void* H, void* ws, size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_forward_mxfp8_q");
   if (!wq || !aligned16(wq)) {
     Plan p;
     const moe_status s = make_plan(dims, opts, &p);
@@ -819,6 +854,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
                            const void* W1, const void* W2, const moe_routing* rt, const void* H, void* dX,
                            void* dW1, void* dW2, float* dWr, void* ws, size_t ws_bytes, void* const* grad_ready,
                            void* stream) {
+  ApiRange api_range("moe_backward_ev");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -979,6 +1015,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
 
 moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, void* ws,
                            size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_route_given");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -1006,6 +1043,7 @@ moe_status moe_route_given(const moe_dims* dims, const moe_opts* opts, const moe
 moe_status moe_ep_pack(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const void* src,
                        void* send_rows, float* send_gate, int32_t* pair_pos, void* ws, size_t ws_bytes,
                        void* stream) {
+  ApiRange api_range("moe_ep_pack");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -1028,6 +1066,7 @@ moe_status moe_ep_pack(const moe_dims* dims, const moe_opts* opts, const moe_rou
 
 moe_status moe_ep_combine(const moe_dims* dims, const moe_opts* opts, const moe_routing* rt, const int32_t* pair_pos,
                           const void* rows, void* out, void* stream) {
+  ApiRange api_range("moe_ep_combine");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -1048,6 +1087,7 @@ moe_status moe_ep_combine(const moe_dims* dims, const moe_opts* opts, const moe_
 moe_status moe_router_backward(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
                                const moe_routing* rt, const float* dS, const int32_t* pair_pos, void* dX, float* dWr,
                                void* ws, size_t ws_bytes, void* stream) {
+  ApiRange api_range("moe_router_backward");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;
@@ -1229,6 +1269,7 @@ size_t carve_noalloc_route(const Plan& p, void* base, RouteWs* w) {
 
 extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* opts, const void* X, const float* Wr,
                                         const float* bias, const moe_routing* rt, void* stream) {
+  ApiRange api_range("moe_route_noalloc");
   Plan p;
   moe_status s = make_plan(dims, opts, &p);
   if (s != MOE_OK) return s;

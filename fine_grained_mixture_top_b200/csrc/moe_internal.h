@@ -67,11 +67,19 @@ cudaError_t launch_pair_lists(const int* offsets, int E, int* pairs, int* left, 
 
 // Per-kernel timing (moe_profile_enable): while on, each launch site brackets
 // its kernel with two CUDA events recorded on the launching stream.
+// Every launch site also opens an NVTX range with the same name (a no-op
+// unless a profiler is attached), so a profiler's timeline shows the kernel
+// names the breakdown uses.
 struct ProfScope {
   int slot = -1;
   cudaStream_t stream;
   ProfScope(cudaStream_t s, const char* name);
   ~ProfScope();
+};
+// An NVTX range over one call of the C ABI.
+struct ApiRange {
+  explicit ApiRange(const char* name);
+  ~ApiRange();
 };
 
 // ---- routing (moe_route.cu)

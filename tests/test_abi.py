@@ -173,3 +173,23 @@ def test_saved_activation_is_constant_in_granularity():
         assert base <= h <= base + 254 * E * n + 256 * n
     assert max(saved) / min(saved) < 1.13
     assert y_cache[-1] == 8 * y_cache[0]
+
+
+def test_plan_log_prints_each_shape_once():
+    """MOE_LOG=1 prints the tile plan of a new shape once on stderr (host
+    only: moe_query_sizes plans without a GPU)."""
+    code = (
+        "import ctypes\n"
+        "from fine_grained_mixture_top_b200 import moe\n"
+        "s = moe.MoeSizes()\n"
+        "for T in (4096, 4096, 8192):\n"
+        "    assert moe.lib().moe_query_sizes(ctypes.byref(moe.dims_of(T, 1536, 128, 256, 8)),\n"
+        "                                     ctypes.byref(moe.opts_of()), ctypes.byref(s)) == 0\n"
+    )
+    env = dict(os.environ, MOE_LOG="1")
+    r = subprocess.run([os.sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=120)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stderr.splitlines() if ln.startswith("moe plan")]
+    assert len(lines) == 2, r.stderr
+    assert "T=4096 d=1536 E=128 n=256 K=8" in lines[0] and "router tile 384 columns" in lines[0]
