@@ -162,9 +162,9 @@ __global__ void __maxnreg__((PairShape<KIND, EPI>::kMaxReg)) __cluster_dims__(2,
   const int per_e = mt_count * nt_count;
   const int num_tiles = p.E * per_e;
 
-  // Tile claims (first CTA's producer), as in moe_gemm_kernel: pairs of even
-  // index from the largest experts' end of the order, odd pairs from the
-  // smallest experts' end.
+  // Tile claims (first CTA's producer), as in moe_gemm_kernel with
+  // dual_ended = 1 (any nonzero mode here): pairs of even index from the
+  // largest experts' end of the order, odd pairs from the smallest experts' end.
   const bool front_end = !p.dual_ended || (pair & 1) == 0;
   const int nfront0 = p.dual_ended ? (npairs + 1) / 2 : npairs;
   const int nback0 = npairs - nfront0;
