@@ -83,6 +83,19 @@ def test_layer_parity_pair_tiles(name, monkeypatch):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["0", "1", "2"])
+def test_weight_gradients_under_every_claim_order(mode, monkeypatch):
+    """The weight-gradient tiles come from a dynamic queue: largest experts
+    first (0), from both ends by CTA parity (1), or alternating ends in every
+    CTA (2, the default).  Each order covers every tile exactly once."""
+    monkeypatch.setenv("MOE_DW_DUAL", mode)
+    cfg = next(c for c in SHAPES if c.name == "pairs")
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
 def test_expert_only_gradient_without_router_path():
     cfg = SHAPES[1]
     inp = make_inputs(cfg, "cuda")
