@@ -174,39 +174,11 @@ cudaError_t launch_softmax_topk(const RouteArgs& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------- permutation
-// Stable counting sort of all (token, expert) pairs by expert, in three
+// Stable counting sort of all (token, expert) pairs by expert, in two
 // launches.  Tokens are cut into chunks of 256; inside a chunk the rank of
 // token t among the chunk's tokens routed to e is a popcount over a
 // per-expert bit mask, so the result does not depend on the order in which
 // threads run.
-__global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
-  pdl_wait();
-  extern __shared__ uint32_t bits[];  // [E][8]
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.sync = 0;  // for chunk_scan_kernel's last block
-  const int words = kChunk / 32;
-  for (int i = threadIdx.x; i < a.E * words; i += blockDim.x) bits[i] = 0u;
-  __syncthreads();
-  const int t = blockIdx.x * kChunk + threadIdx.x;
-  const int w = threadIdx.x >> 5, b = threadIdx.x & 31;
-  int p0 = 0, p1 = 0;
-  if (t < a.T) {
-    p0 = a.tok_ptr[t];
-    p1 = a.tok_ptr[t + 1];
-    for (int p = p0; p < p1; ++p) atomicOr(&bits[a.pair_expert[p] * words + w], 1u << b);
-  }
-  __syncthreads();
-  for (int p = p0; p < p1; ++p) {
-    const uint32_t* be = bits + a.pair_expert[p] * words;
-    int r = __popc(be[w] & ((1u << b) - 1u));
-    for (int j = 0; j < w; ++j) r += __popc(be[j]);
-    a.local_rank[p] = r;
-  }
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-    int c = 0;
-    for (int j = 0; j < words; ++j) c += __popc(bits[e * words + j]);
-    a.hist[(size_t)blockIdx.x * a.E + e] = c;
-  }
-}
 
 // Exclusive scan over a block of kScanThreads threads; *total gets the sum.
 constexpr int kScanThreads = 256;
@@ -233,29 +205,37 @@ __device__ int block_exclusive_scan_256(int v, int* sh /*[8]*/, int* total) {
   return prefix + x - v;
 }
 
-// Per expert (one warp each, several blocks): exclusive scan over the chunks
-// of its per-chunk counts (chunk bases relative to the expert's segment) and
-// the expert's total count.  The last block to finish then computes the
-// 128-padded segment offsets (exclusive scan over experts).
-__global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(RouteArgs a) {
+// One block per chunk: each pair's rank inside its chunk and expert, and the
+// chunk's per-expert counts.  The last block to finish then scans, per
+// expert (a thread each), its chunk counts into chunk bases relative to the
+// expert's segment and the expert's total count, and the 128-padded segment
+// offsets over the experts (*a.sync zeroed before the launch).
+static_assert(kChunk == kScanThreads, "the rank kernel's block scans with kScanThreads threads");
+__global__ void __launch_bounds__(kChunk) rank_kernel(RouteArgs a) {
   pdl_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * (kScanThreads / 32) + warp;
-  if (e < a.E) {
-    int carry = 0;
-    for (int c0 = 0; c0 < a.nchunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int h = c < a.nchunks ? a.hist[(size_t)c * a.E + e] : 0;
-      int x = h;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (c < a.nchunks) a.hist[(size_t)c * a.E + e] = carry + x - h;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) a.counts[e] = carry;
+  extern __shared__ uint32_t bits[];  // [E][8]
+  const int words = kChunk / 32;
+  for (int i = threadIdx.x; i < a.E * words; i += blockDim.x) bits[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunk + threadIdx.x;
+  const int w = threadIdx.x >> 5, b = threadIdx.x & 31;
+  int p0 = 0, p1 = 0;
+  if (t < a.T) {
+    p0 = a.tok_ptr[t];
+    p1 = a.tok_ptr[t + 1];
+    for (int p = p0; p < p1; ++p) atomicOr(&bits[a.pair_expert[p] * words + w], 1u << b);
+  }
+  __syncthreads();
+  for (int p = p0; p < p1; ++p) {
+    const uint32_t* be = bits + a.pair_expert[p] * words;
+    int r = __popc(be[w] & ((1u << b) - 1u));
+    for (int j = 0; j < w; ++j) r += __popc(be[j]);
+    a.local_rank[p] = r;
+  }
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    int c = 0;
+    for (int j = 0; j < words; ++j) c += __popc(bits[e * words + j]);
+    a.hist[(size_t)blockIdx.x * a.E + e] = c;
   }
   // The last block to arrive sees every block's counts: each block fences its
   // writes before it counts itself done, and the last one fences before reading.
@@ -267,10 +247,29 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(RouteArgs a) {
   __syncthreads();
   if (!is_last) return;
   __threadfence();
+  // a thread per expert: its chunk counts (coalesced over the experts) in
+  // batches of 16 loads in flight, scanned in chunk order
+  constexpr int kB = 16;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    int carry = 0;
+    for (int c0 = 0; c0 < a.nchunks; c0 += kB) {
+      int h[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) h[j] = c0 + j < a.nchunks ? __ldcg(a.hist + (size_t)(c0 + j) * a.E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+        if (c0 + j < a.nchunks) {
+          a.hist[(size_t)(c0 + j) * a.E + e] = carry;
+          carry += h[j];
+        }
+    }
+    a.counts[e] = carry;
+  }
+  __syncthreads();  // every count written (and visible to the block)
   int carry = 0;
   for (int e0 = 0; e0 < a.E; e0 += kScanThreads) {
     const int ee = e0 + threadIdx.x;
-    const int padded = ee < a.E ? ((__ldcg(a.counts + ee) + kTile - 1) / kTile) * kTile : 0;
+    const int padded = ee < a.E ? ((a.counts[ee] + kTile - 1) / kTile) * kTile : 0;
     int total;
     const int ex = block_exclusive_scan_256(padded, sh, &total);
     if (ee < a.E) a.offsets[ee] = carry + ex;
@@ -310,13 +309,11 @@ __global__ void __launch_bounds__(256) scatter_kernel(RouteArgs a, int token_blo
 }
 
 cudaError_t launch_permute(const RouteArgs& a, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(a.sync, 0, sizeof(int), s);  // the rank kernel's last-block counter
+  if (err != cudaSuccess) return err;
   {
     ProfScope ps(s, "permute_rank");
     launch_pdl(rank_kernel, dim3(a.nchunks), dim3(kChunk), (size_t)a.E * (kChunk / 32) * sizeof(uint32_t), s, a);
-  }
-  {
-    ProfScope ps(s, "permute_scan");
-    launch_pdl(chunk_scan_kernel, dim3((a.E + 7) / 8), dim3(kScanThreads), 0, s, a);
   }
   {
     ProfScope ps(s, "permute_scatter");
