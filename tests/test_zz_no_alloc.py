@@ -50,7 +50,7 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row():
         inp = make_inputs(cfg, "cuda", need_grad_inputs=False)
         ref = moe.MoELayer(cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
         # moe_route runs the same kernels first, so none of them is loaded
-        # (lazily, by the driver) during the measured call below
+        # (lazily, by the CUDA driver) during the measured call below
         ref.route(inp["X"], inp["Wr"], inp["bias"])
         rt = moe.Routing.allocate(ref.dims, ref.sizes, "cuda")
         torch.cuda.synchronize()
