@@ -14,6 +14,7 @@
 
 #include <cfloat>
 #include <climits>
+#include <cstdlib>
 
 #include "moe_internal.h"
 
@@ -1036,7 +1037,10 @@ cudaError_t launch_token_round(const RouteArgs& a, const RoundArgs& r, cudaStrea
     ProfScope ps(s, "round_select");
     // stage the expert's keys and routed-token words when they fit
     const size_t staged = kTrSelFixed + (size_t)W * sizeof(uint32_t);
-    if (staged <= kTrSelMax) {
+    // MOE_TR_UNSTAGED=1 takes the path of rows too long to stage (for tests)
+    const char* fu = std::getenv("MOE_TR_UNSTAGED");
+    const bool force_unstaged = fu && std::atoi(fu) != 0;
+    if (staged <= kTrSelMax && !force_unstaged) {
       err = set_max_dynamic_smem(reinterpret_cast<const void*>(tr_select_kernel<true>), (int)kTrSelMax);
       if (err != cudaSuccess) return err;
       launch_pdl(tr_select_kernel<true>, dim3(r.E), dim3(kTrSelThreads), staged, s, r.T, W, r.mode, r.seed, a.counts,

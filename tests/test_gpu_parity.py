@@ -115,6 +115,22 @@ def test_token_rounding_parity(mode, T, E, K, wr_std):
     are then broken by token index alone."""
     cfg = MoEConfig("tr", T=T, d=128, E=E, n=64, K=K, w_std=0.05, wr_std=wr_std,
                     bias="normal" if wr_std > 0 else "none", seed=21)
+    _check_token_rounding(cfg, mode)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wr_std", [0.02, 0.0])
+def test_token_rounding_parity_unstaged(wr_std, monkeypatch):
+    """The selection's path for expert rows too long to stage in shared
+    memory (reading candidates and keys from global memory), forced on a
+    small layer; with wr_std = 0 it also takes the radix fallback there."""
+    monkeypatch.setenv("MOE_TR_UNSTAGED", "1")
+    cfg = MoEConfig("tr", T=6000, d=128, E=8 if wr_std == 0 else 130, n=64, K=2 if wr_std == 0 else 4, w_std=0.05,
+                    wr_std=wr_std, bias="normal" if wr_std > 0 else "none", seed=22)
+    _check_token_rounding(cfg, 2)
+
+
+def _check_token_rounding(cfg, mode):
     seed = 1234
     inp = make_inputs(cfg, "cuda")
     layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K, round_mode=mode, seed=seed)
