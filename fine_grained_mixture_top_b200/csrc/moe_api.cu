@@ -161,24 +161,36 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   p.bn_dw1 = ((2 * n) % 256 == 0) ? 256 : 128;
   p.bn_dw2 = p.bn_down;
   p.nts = n / p.bn_dh;
-  // Eight epilogue warps where the epilogue bounds a tile: the dH tile's
-  // epilogue (H reload, three outputs) outlasts a main loop of up to 24
-  // k-blocks (d <= 1536); the dX~ epilogue (a 64 KB store per tile plus the
-  // router path) outlasts a main loop of up to 16 k-blocks (2n <= 1024).
-  // Longer main loops keep 4 warps.  (The down-proj kernel measured slower
-  // with 8: its short main loop is bound by the Y stores, not the epilogue.)
-  p.epi_dh = (d / 64 <= 24) ? 8 : 4;
-  p.epi_dxt = (2 * n / 64 <= 16) ? 8 : 4;
-  // The weight-gradient tiles run K over an expert's rows; with few rows per
-  // expert (at most 8 k-blocks on average) a tile is bound by storing its
-  // 128 x BN result, so the epilogue gets 8 warps.
-  p.epi_dw = (T * K / E <= 8 * 64) ? 8 : 4;
+  // Eight epilogue warps only where the epilogue outlasts a short main loop;
+  // otherwise 4 warps, whose smaller staging leaves room for a deeper stage
+  // ring.  Measured: dH with 4 warps 4 % faster at d = 1536 (24 k-blocks) and
+  // at d = 2048; dX~ with 4 warps 7 % faster at 2n = 512 (8 k-blocks), with 8
+  // warps 25 % faster at 2n = 256 (4 k-blocks: a 64 KB store plus the router
+  // path per tile).  The dH threshold (12 k-blocks) is half the shortest main
+  // loop measured to prefer 4.  (The down-proj kernel measured slower with 8:
+  // its short main loop is bound by the Y stores, not the epilogue.)
+  p.epi_dh = (d / 64 <= 12) ? 8 : 4;
+  p.epi_dxt = (2 * n / 64 <= 4) ? 8 : 4;
+  // The weight-gradient kernels keep 4 epilogue warps.  Their short tiles
+  // (an expert's few rows) are bound by storing the 128 x BN result, but with
+  // claims alternating between long and short tiles those stores run under
+  // the long tiles' main loops, and the fourth ring stage that 4 warps' staging
+  // leaves room for pays more: dW1 3-6 % faster than with 8 warps on the
+  // DeepSeek-V3-shaped, E = 256 and small-expert layers (8 warps with one
+  // staging buffer each, also 4 stages, measured level with 4 warps).
+  p.epi_dw = 4;
   p.dw_dual = 2;  // every CTA alternates ends: short tiles' stores run under long tiles' main loops
-  // tuning overrides, for measurements: MOE_EPI_DW (4 or 8), MOE_DW_DUAL (0 or 1)
-  if (const char* v = std::getenv("MOE_EPI_DW")) {
-    const int x = std::atoi(v);
-    if (x == 4 || x == 8) p.epi_dw = x;
-  }
+  // tuning overrides, for measurements: MOE_EPI_DW, MOE_EPI_DH, MOE_EPI_DXT
+  // (4 or 8 epilogue warps), MOE_DW_DUAL (0 to 2)
+  auto epi_override = [](const char* name, int& field) {
+    if (const char* v = std::getenv(name)) {
+      const int x = std::atoi(v);
+      if (x == 4 || x == 8) field = x;
+    }
+  };
+  epi_override("MOE_EPI_DW", p.epi_dw);
+  epi_override("MOE_EPI_DH", p.epi_dh);
+  epi_override("MOE_EPI_DXT", p.epi_dxt);
   if (const char* v = std::getenv("MOE_DW_DUAL")) {
     const int x = std::atoi(v);
     if (x >= 0 && x <= 2) p.dw_dual = x;
@@ -326,7 +338,9 @@ size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   w->dH = c.take<__nv_bfloat16>((size_t)p.R_max * 2 * p.n);
   w->Ahat = c.take<__nv_bfloat16>((size_t)p.R_max * p.n);
   w->dXt = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
-  w->dS_part = c.take<float>((size_t)p.R_max * p.nds);
+  // sized for 8 dH epilogue warps whatever the plan picked, so that the
+  // MOE_EPI_DH override cannot outgrow a workspace sized before it was set
+  w->dS_part = c.take<float>((size_t)p.R_max * p.nts * 2);
   w->dz_split = c.take<__nv_bfloat16>((size_t)p.T * 2 * p.Epad);
   w->dz_row = c.take<float>((size_t)p.R_max);
   w->WrT = c.take<float>((size_t)p.E * p.d);

@@ -96,6 +96,21 @@ def test_weight_gradients_under_every_claim_order(mode, monkeypatch):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("var,warps,name", [("MOE_EPI_DW", "8", "sparse"), ("MOE_EPI_DW", "8", "bn64"),
+                                            ("MOE_EPI_DH", "4", "bn64"), ("MOE_EPI_DH", "4", "bn256"),
+                                            ("MOE_EPI_DXT", "4", "bn256"), ("MOE_EPI_DXT", "8", "pairs_n640")])
+def test_layer_parity_other_epilogue_widths(var, warps, name, monkeypatch):
+    """The plan picks 4 or 8 epilogue warps per kernel from the shape; the
+    other width of the weight-gradient (empty experts included), dH and dX~
+    kernels, forced."""
+    monkeypatch.setenv(var, warps)
+    cfg = next(c for c in SHAPES if c.name == name)
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
 def test_expert_only_gradient_without_router_path():
     cfg = SHAPES[1]
     inp = make_inputs(cfg, "cuda")
