@@ -126,6 +126,7 @@ struct Plan {
                         // 2 every CTA alternating ends
   int dw1_pair, dw2_pair;  // weight-gradient GEMMs on CTA pairs (256 x 256 tiles)
   int gm_pair;             // down-proj and dX~ on CTA pairs (256 x 256 tiles of two M tiles)
+  int wide_down, wide_dxt;  // down-proj / dX~ with 256 x 256 tiles (two M tiles) on one CTA
   int ksplit, ksplit_rows;
 };
 
@@ -205,6 +206,22 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   // 128 x 256 tile on any workload here, and slower on the balanced ones.
   p.gm_pair = 0;
   if (const char* v = std::getenv("MOE_GM_PAIR")) p.gm_pair = (d % 256 == 0) && std::atoi(v) != 0;
+  // Down-proj with 256 x 256 tiles on one CTA (two M tiles sharing B) where N
+  // = d splits into 256-column tiles and the main loop (n / 64 k-blocks) is
+  // long enough for the single-buffered accumulator.  Measured against the
+  // 128 x 256 tiles: 1.5-5 % faster at n = 768..2048 (12-32 k-blocks), 5 %
+  // slower at n = 256 (4).  dX~ on the same tiles measured level or slower on
+  // the balanced layers (+3 % at 2n = 1536) and 1.4 % faster on the
+  // DeepSeek-V3-shaped one, so it stays opt-in: MOE_GM_WIDE=1 turns both on,
+  // MOE_GM_WIDE=0 both off.
+  p.wide_down = (d % 256 == 0) && (n / 64 >= 12);
+  p.wide_dxt = 0;
+  if (const char* v = std::getenv("MOE_GM_WIDE")) {
+    const int x = std::atoi(v);
+    p.wide_down = (d % 256 == 0) && x != 0;
+    p.wide_dxt = (d % 256 == 0) && x != 0;
+  }
+  if (p.gm_pair) p.wide_down = p.wide_dxt = 0;
   p.nds = p.nts * (p.epi_dh / 4);
   // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
   const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
@@ -222,10 +239,12 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
         std::fprintf(stderr,
                      "moe plan T=%lld d=%d E=%d n=%d K=%d round=%d: P_max=%lld R_max=%lld; BN up %d down %d dH %d "
                      "dX~ %d dW1 %d dW2 %d; epilogue warps dH %d dX~ %d dW %d; dW tiles from both ends %d; CTA pairs "
-                     "dW1 %d dW2 %d down/dX~ %d; router tile %d columns; dWr split-K %d x %d rows\n",
+                     "dW1 %d dW2 %d down/dX~ %d; 256-row tiles on one CTA down %d dX~ %d; router tile %d columns; "
+                     "dWr split-K %d x %d rows\n",
                      (long long)T, d, E, n, K, opts->round_mode, (long long)p.P_max, (long long)p.R_max, p.bn_up,
                      p.bn_down, p.bn_dh, p.bn_dxt, p.bn_dw1, p.bn_dw2, p.epi_dh, p.epi_dxt, p.epi_dw, p.dw_dual,
-                     p.dw1_pair, p.dw2_pair, p.gm_pair, p.Epad == 128 ? 384 : 192, p.ksplit, p.ksplit_rows);
+                     p.dw1_pair, p.dw2_pair, p.gm_pair, p.wide_down, p.wide_dxt, p.Epad == 128 ? 384 : 192, p.ksplit,
+                     p.ksplit_rows);
     }
   }
   *pl = p;
@@ -277,6 +296,7 @@ struct FwdWs {
   __nv_bfloat16* A;
   __nv_bfloat16* Y;
   int *mpair, *mleft;  // pair and leftover lists of the M tiles (CTA-pair down-proj)
+  int* mwide;          // 256-row tile list of the M tiles (one-CTA 256 x 256 down-proj)
 };
 // MXFP8 forward: codes and scales of X, W1, W2 and A, and Y
 // MXFP8 expert weights: codes K-major and scales in the MMA's tile layout
@@ -296,6 +316,7 @@ size_t carve_fwd(const Plan& p, void* ws, FwdWs* w) {
   w->Y = c.take<__nv_bfloat16>((size_t)p.R_max * p.d);
   w->mpair = c.take<int>((size_t)(p.R_max / 256 + 2));
   w->mleft = c.take<int>((size_t)p.E + 1);
+  w->mwide = c.take<int>((size_t)(p.R_max / 256 + p.E + 2));
   return c.off;
 }
 
@@ -332,6 +353,7 @@ struct BwdWs {
   float *dS_part, *dz_row, *WrT, *dWr_part;
   int *sched, *expert_order;
   int *mpair, *mleft;  // pair and leftover lists of the M tiles (CTA-pair dX~)
+  int* mwide;          // 256-row tile list of the M tiles (one-CTA 256 x 256 dX~)
 };
 size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   Carve c{static_cast<char*>(ws)};
@@ -349,6 +371,7 @@ size_t carve_bwd(const Plan& p, void* ws, BwdWs* w) {
   w->expert_order = c.take<int>((size_t)p.E);
   w->mpair = c.take<int>((size_t)(p.R_max / 256 + 2));
   w->mleft = c.take<int>((size_t)p.E + 1);
+  w->mwide = c.take<int>((size_t)(p.R_max / 256 + p.E + 2));
   return c.off;
 }
 
@@ -666,6 +689,11 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
       g.mlist = w.mleft;
       MOE_TRY_CUDA(launch_gemm(G_DOWN, 256, 4, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
                                false));
+    } else if (p.wide_down) {
+      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
+      g.num_n_tiles = p.d / 256;
+      g.mlist = w.mwide;
+      MOE_TRY_CUDA(launch_gemm_wide_m(G_DOWN, g, grid_for((mtiles / 2 + p.E) * g.num_n_tiles, sms), st));
     } else {
       MOE_TRY_CUDA(launch_gemm(G_DOWN, p.bn_down, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
     }
@@ -1013,6 +1041,13 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
       MOE_TRY_CUDA(
           launch_gemm(G_DXT, 256, p.epi_dxt, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
                       false));
+    } else if (p.wide_dxt) {
+      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
+      GemmParams gw = g;
+      MOE_TRY_MAP(make_tmap(&gw.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 256));
+      gw.num_n_tiles = p.d / 256;
+      gw.mlist = w.mwide;
+      MOE_TRY_CUDA(launch_gemm_wide_m(G_DXT, gw, grid_for((mtiles / 2 + p.E) * gw.num_n_tiles, sms), st));
     } else {
       MOE_TRY_CUDA(launch_gemm(G_DXT, p.bn_dxt, p.epi_dxt, g, grid_for(mtiles * g.num_n_tiles, sms), st));
     }

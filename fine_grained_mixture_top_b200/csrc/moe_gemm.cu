@@ -11,6 +11,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_pair_m.cuh"
+#include "gemm_wide_m.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -220,6 +221,86 @@ cudaError_t launch_gemm_pair_m(int kind, int epi, const GemmParams& p_in, int ma
   if (kind == G_DXT && epi == 4) return launch_gm_pair_one<G_DXT, 4>(p, max_pairs, s);
   if (kind == G_DXT && epi == 8) return launch_gm_pair_one<G_DXT, 8>(p, max_pairs, s);
   return cudaErrorInvalidValue;
+}
+
+template <int KIND>
+static cudaError_t launch_gm_wide_one(const GemmParams& p, int grid, cudaStream_t stream) {
+  using SH = WideMShape<KIND>;
+  constexpr int smem = SH::kSmemBytes;
+  auto fn = moe_gm_wide_kernel<KIND>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fn), smem);
+  if (e == cudaSuccess && grid > 0) e = launch_pdl(fn, dim3(grid), dim3(SH::kThreads), (size_t)smem, stream, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // the error is returned here; do not leave it for a later call to find
+    cudaFuncAttributes fa = {};
+    cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(fn));
+    std::snprintf(g_launch_diag, sizeof(g_launch_diag),
+                  "wide gemm (M) kind %d: grid %d x %d threads, %d B dynamic smem; kernel: %d regs, max %d threads, "
+                  "max dynamic smem %d B",
+                  KIND, grid, SH::kThreads, smem, fa.numRegs, fa.maxThreadsPerBlock, fa.maxDynamicSharedSizeBytes);
+  }
+  return e;
+}
+
+cudaError_t launch_gemm_wide_m(int kind, const GemmParams& p_in, int grid, cudaStream_t s) {
+  GemmParams p = p_in;
+  {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (kind == g_trace_kind) {
+      p.trace = g_trace_buf;
+      p.trace_cap = g_trace_cap;
+    }
+  }
+  if (kind == G_DOWN) return launch_gm_wide_one<G_DOWN>(p, grid, s);
+  if (kind == G_DXT) return launch_gm_wide_one<G_DXT>(p, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+// List of 256-row tiles of the grouped-M M tiles: for expert e, whose segment
+// holds tiles [offsets[e] / 128, offsets[e + 1] / 128), one entry per pair of
+// consecutive tiles (its first tile, with kWideSecond set) and one for the
+// last tile of an odd count (without the flag); [count, entry...] in expert
+// order.  One block, a thread per expert (E <= 1024).
+__global__ void __launch_bounds__(1024) wide_list_kernel(const int* __restrict__ offsets, int E,
+                                                         int* __restrict__ list) {
+  __shared__ int wsum[32];
+  const int e = threadIdx.x;
+  const int lane = e & 31, w = e >> 5;
+  pdl_wait();
+  int t0 = 0, nt = 0;
+  if (e < E) {
+    const int o0 = __ldg(offsets + e), o1 = __ldg(offsets + e + 1);
+    t0 = o0 / kBM;
+    nt = (o1 - o0) / kBM;
+  }
+  const int nw = (nt + 1) >> 1;
+  int sw = nw;  // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, sw, o);
+    if (lane >= o) sw += a;
+  }
+  if (lane == 31) wsum[w] = sw;
+  __syncthreads();
+  if (w == 0) {  // scan of the warp totals
+    const int nwarps = (int)(blockDim.x >> 5);
+    int a = lane < nwarps ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, a, o);
+      if (lane >= o) a += x;
+    }
+    wsum[lane] = a;
+  }
+  __syncthreads();
+  const int b = (w > 0 ? wsum[w - 1] : 0) + sw - nw;  // exclusive offset
+  for (int j = 0; j < nw; ++j) list[1 + b + j] = (t0 + 2 * j) | (2 * j + 1 < nt ? kWideSecond : 0);
+  if (e == (int)blockDim.x - 1) list[0] = b + nw;
+}
+
+cudaError_t launch_wide_list(const int* offsets, int E, int* list, cudaStream_t s) {
+  if (E < 1 || E > 1024) return cudaErrorInvalidValue;
+  return launch_pdl(wide_list_kernel, dim3(1), dim3(1024), 0, s, offsets, E, list);
 }
 
 // Pair and leftover lists of the grouped-M M tiles: for expert e, whose

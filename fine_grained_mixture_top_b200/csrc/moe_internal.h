@@ -60,6 +60,12 @@ cudaError_t launch_gemm_pair(int kind, int epi, const GemmParams& p, int pairs, 
 // p.num_n_tiles counts 256-column tiles; at most `max_pairs` clusters of 2
 // (fewer if fewer fit the device at once).
 cudaError_t launch_gemm_pair_m(int kind, int epi, const GemmParams& p, int max_pairs, cudaStream_t s);
+// Down-proj and dX~ with 256 x 256 tiles on one CTA (gemm_wide_m.cuh) over
+// the list p.mlist of 256-row tiles; p.num_n_tiles counts 256-column tiles.
+cudaError_t launch_gemm_wide_m(int kind, const GemmParams& p, int grid, cudaStream_t s);
+// List of the grouped-M tiles in 256-row tiles from the segment offsets
+// ([count, entry...]: up to R_max / 256 + E entries after the count).
+cudaError_t launch_wide_list(const int* offsets, int E, int* list, cudaStream_t s);
 // Pair list and leftover list of the grouped-M tiles from the segment offsets
 // (each [count, tile...]; `pairs` holds up to R_max / 256 + 1 entries after the
 // count, `left` up to E).

@@ -83,6 +83,20 @@ def test_layer_parity_pair_tiles(name, monkeypatch):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("name", ["pairs", "pairs_n640", "bn256"])
+def test_layer_parity_wide_tiles(name, monkeypatch):
+    """Down-proj and dX~ with 256 x 256 tiles on one CTA (two M tiles of one
+    expert sharing B; an expert's odd last M tile as a half-filled tile),
+    forced on small layers: even and odd tile counts per expert, experts of
+    one tile only, the router path of dX~."""
+    monkeypatch.setenv("MOE_GM_WIDE", "1")
+    cfg = next(c for c in SHAPES if c.name == name)
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("mode", ["0", "1", "2"])
 def test_weight_gradients_under_every_claim_order(mode, monkeypatch):
     """The weight-gradient tiles come from a dynamic queue: largest experts
