@@ -133,6 +133,13 @@ struct Plan {
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Column width of the router-logit tiles: 384 (two 64-expert groups, all 512
+// TMEM columns) where the padded expert count is a multiple of 128, so that
+// every 128-row tile of X is read once per two groups; else 192 (one group).
+// On the DeepSeek-V3-shaped layer (Epad = 256, 64 row tiles) that is 128 tiles
+// in one wave instead of 256 in 1.73.
+inline int router_bn(int Epad) { return Epad % 128 == 0 ? 384 : 192; }
+
 moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   if (!dims || !opts) return MOE_ERR_INVALID_ARG;
   if (opts->round_mode < 0 || opts->round_mode > 2 || (opts->router_grad != 0 && opts->router_grad != 1))
@@ -223,12 +230,28 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
   }
   if (p.gm_pair) p.wide_down = p.wide_dxt = 0;
   p.nds = p.nts * (p.epi_dh / 4);
-  // split-K of the router-weight gradient: about two tiles per SM of a 148-SM part
-  const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
-  int64_t ks = std::max<int64_t>(1, cdiv(296, mn_tiles));
-  ks = std::min<int64_t>(ks, cdiv(T, 64));
-  p.ksplit_rows = (int)(cdiv(cdiv(T, ks), 64) * 64);
-  p.ksplit = (int)cdiv(T, p.ksplit_rows);
+  // split-K of the router-weight gradient: the split count with the shortest
+  // critical path of the persistent launch on 148 SMs -- tiles round-robin,
+  // so (waves of tiles) x (k-blocks per tile) -- plus the reduction's read of
+  // the fp32 partials (about 450 KB per k-block of one tile's load time).
+  // A fixed "two tiles per SM" left 3.03 waves on the DeepSeek-V3-shaped layer
+  // and 2.1 on the 7B-class one.
+  {
+    const int64_t mn_tiles = cdiv(d, 128) * (p.Epad / 64);
+    double best = 0.0;
+    const int64_t ks_max = std::min<int64_t>(64, cdiv(T, 64));
+    for (int64_t ks = 1; ks <= ks_max; ++ks) {
+      const int64_t rows = cdiv(cdiv(T, ks), 64) * 64;
+      const int64_t splits = cdiv(T, rows);
+      const double cost =
+          (double)cdiv(mn_tiles * splits, 148) * (double)(rows / 64) + (double)splits * d * p.Epad / 450000.0;
+      if (ks == 1 || cost < best) {
+        best = cost;
+        p.ksplit_rows = (int)rows;
+        p.ksplit = (int)splits;
+      }
+    }
+  }
   // MOE_LOG=1: the tile plan of each new shape, once, on stderr
   if (const char* v = std::getenv("MOE_LOG")) {
     if (std::atoi(v) != 0) {
@@ -243,7 +266,7 @@ moe_status make_plan(const moe_dims* dims, const moe_opts* opts, Plan* pl) {
                      "dWr split-K %d x %d rows\n",
                      (long long)T, d, E, n, K, opts->round_mode, (long long)p.P_max, (long long)p.R_max, p.bn_up,
                      p.bn_down, p.bn_dh, p.bn_dxt, p.bn_dw1, p.bn_dw2, p.epi_dh, p.epi_dxt, p.epi_dw, p.dw_dual,
-                     p.dw1_pair, p.dw2_pair, p.gm_pair, p.wide_down, p.wide_dxt, p.Epad == 128 ? 384 : 192, p.ksplit,
+                     p.dw1_pair, p.dw2_pair, p.gm_pair, p.wide_down, p.wide_dxt, router_bn(p.Epad), p.ksplit,
                      p.ksplit_rows);
     }
   }
@@ -579,7 +602,7 @@ moe_status moe_route(const moe_dims* dims, const moe_opts* opts, const void* X, 
   MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
   // one tile covers both groups of 64 experts where E <= 128 (TMEM holds two
   // groups' hi slots and mid/lo accumulators), so X is read once per row tile
-  const int bn_rtr = p.Epad == 128 ? 384 : 192;
+  const int bn_rtr = router_bn(p.Epad);
   g.num_m_tiles = (int)cdiv(p.T, 128);
   g.num_n_tiles = 3 * p.Epad / bn_rtr;
   g.outf = const_cast<float*>(a.logits);
@@ -1342,7 +1365,7 @@ extern "C" moe_status moe_route_noalloc(const moe_dims* dims, const moe_opts* op
   GemmParams g = base_params(p, rt, status);
   MOE_TRY_MAP(make_tmap(&g.tmA, X, (uint64_t)p.T, (uint64_t)p.d, 64, 128));
   MOE_TRY_MAP(make_tmap(&g.tmB, w.Wr_split, (uint64_t)p.d, (uint64_t)3 * p.Epad, 64, 64));
-  const int bn_rtr = p.Epad == 128 ? 384 : 192;  // as in moe_route
+  const int bn_rtr = router_bn(p.Epad);
   g.num_m_tiles = (int)cdiv(p.T, 128);
   g.num_n_tiles = 3 * p.Epad / bn_rtr;
   g.outf = rt->logits;
