@@ -702,6 +702,10 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
+    if (p.wide_down) {  // the 256-row tile list, in its own profiler scope (one kernel per scope)
+      ProfScope pl(st, "down_proj_tile_list");
+      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
+    }
     ProfScope ps(st, "down_proj_gemm");
     if (p.gm_pair) {
       // pairs of M tiles on CTA pairs, then each expert's odd last M tile on one CTA
@@ -713,7 +717,6 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
       MOE_TRY_CUDA(launch_gemm(G_DOWN, 256, 4, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
                                false));
     } else if (p.wide_down) {
-      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
       g.num_n_tiles = p.d / 256;
       g.mlist = w.mwide;
       MOE_TRY_CUDA(launch_gemm_wide_m(G_DOWN, g, grid_for((mtiles / 2 + p.E) * g.num_n_tiles, sms), st));
@@ -1048,6 +1051,10 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
       g.rscale = w.dz_row;
     }
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.dXt, (uint64_t)p.R_max, (uint64_t)p.d));
+    if (p.wide_dxt) {
+      ProfScope pl(st, "dxt_tile_list");
+      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
+    }
     ProfScope ps(st, "dxt_gemm");
     if (p.gm_pair) {
       // pairs of M tiles on CTA pairs (each CTA loading 128 of a tile's 256 W1
@@ -1065,7 +1072,6 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
           launch_gemm(G_DXT, 256, p.epi_dxt, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
                       false));
     } else if (p.wide_dxt) {
-      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
       GemmParams gw = g;
       MOE_TRY_MAP(make_tmap(&gw.tmB, W1, (uint64_t)p.E * p.d, (uint64_t)2 * p.n, 64, 256));
       gw.num_n_tiles = p.d / 256;
