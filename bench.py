@@ -479,8 +479,8 @@ def main():
             entry["gbs"] = round(by / (avg * 1e-3) / 1e9, 1)
         breakdown[name] = entry
     # forward / backward split of the breakdown pass (routing counted apart)
-    fwd_k = {"up_proj_gemm", "down_proj_gemm", "down_proj_tile_list", "aggregate_fwd", "up_proj_gemm_mx",
-             "down_proj_gemm_mx", "mx_quant_x", "mx_quant_w"}
+    fwd_k = {"up_proj_gemm", "down_proj_gemm", "aggregate_fwd", "up_proj_gemm_mx", "down_proj_gemm_mx",
+             "mx_quant_x", "mx_quant_w"}
     route_us = fwd_us = bwd_us = 0.0
     for name, ts in per.items():
         us = 1e3 * sum(ts) / n_breakdown

@@ -71,6 +71,9 @@ struct GemmParams {
   // grouped-M kinds: the 128-row M tiles to run, [count, tile...], or null
   // for all of them (the pair kernel's list: the first of each pair of tiles)
   const int* mlist;
+  // up-proj only: where the first CTA writes the 256-row tile list of the
+  // grouped-M tiles for the down-proj launch that follows (or null)
+  int* wlist;
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
   // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
@@ -160,6 +163,37 @@ struct EpiCfg {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
+constexpr int kWideSecond = 1 << 30;  // 256-row tile list entry flag: the pair's second M tile exists
+
+// The 256-row tile list of the grouped-M tiles, by one warp: for expert e,
+// whose padded segment holds M tiles [offsets[e] / 128, offsets[e + 1] / 128),
+// one entry per pair of consecutive tiles (its first tile, with kWideSecond)
+// and one for the last tile of an odd count (without the flag);
+// list = [count, entry...] in expert order.
+__device__ __forceinline__ void write_wide_list(const int* __restrict__ offsets, int E, int* __restrict__ list,
+                                                int lane) {
+  int base = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int t0 = 0, nt = 0;
+    if (e < E) {
+      const int o0 = __ldg(offsets + e), o1 = __ldg(offsets + e + 1);
+      t0 = o0 / kBM;
+      nt = (o1 - o0) / kBM;
+    }
+    const int nw = (nt + 1) >> 1;
+    int sw = nw;  // inclusive scan over the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, sw, o);
+      if (lane >= o) sw += a;
+    }
+    const int b = base + sw - nw;
+    for (int j = 0; j < nw; ++j) list[1 + b + j] = (t0 + 2 * j) | (2 * j + 1 < nt ? kWideSecond : 0);
+    base += __shfl_sync(0xffffffffu, sw, 31);
+  }
+  if (lane == 0) list[0] = base;
+}
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
 constexpr int kStageBudget = 200 * 1024;
@@ -920,6 +954,11 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     int tcount = 0, ntr = 0;
     const bool tracer = (warp == 2 && lane == 0);
     bool ok = true;
+    if constexpr (KIND == G_UP) {
+      // the first CTA's first epilogue warp writes the down-proj's tile list
+      // while the first tile's main loop runs
+      if (p.wlist && blockIdx.x == 0 && warp == 2) write_wide_list(p.offsets, p.E, p.wlist, lane);
+    }
     for (int ti = 0; ok; ++ti) {
       TileInfo t;
       const int tile = consume_tile(ti, ok, t);

@@ -39,8 +39,6 @@
 
 namespace moe {
 
-constexpr int kWideSecond = 1 << 30;  // list entry flag: the pair's second M tile exists
-
 template <int KIND>
 struct WideMShape {
   static_assert(KIND == G_DOWN || KIND == G_DXT, "256-row tiles: down-proj and dX~");

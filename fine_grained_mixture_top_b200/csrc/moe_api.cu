@@ -691,6 +691,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.out1 = w.A;
     MOE_TRY_MAP(make_store_map(&g.tmC0, H, (uint64_t)p.R_max, (uint64_t)2 * p.n));
     MOE_TRY_MAP(make_store_map(&g.tmC1, w.A, (uint64_t)p.R_max, (uint64_t)p.n));
+    if (p.wide_down) g.wlist = w.mwide;  // the down-proj's 256-row tile list, written by the first CTA
     ProfScope ps(st, "up_proj_gemm");
     MOE_TRY_CUDA(launch_gemm(G_UP, p.bn_up, 4, g, grid_for(mtiles * g.num_n_tiles, sms), st));
   }
@@ -702,10 +703,6 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
     g.num_n_tiles = p.d / p.bn_down;
     g.out0 = w.Y;
     MOE_TRY_MAP(make_store_map_wide(&g.tmC0, w.Y, (uint64_t)p.R_max, (uint64_t)p.d));
-    if (p.wide_down) {  // the 256-row tile list, in its own profiler scope (one kernel per scope)
-      ProfScope pl(st, "down_proj_tile_list");
-      MOE_TRY_CUDA(launch_wide_list(rt->offsets, p.E, w.mwide, st));
-    }
     ProfScope ps(st, "down_proj_gemm");
     if (p.gm_pair) {
       // pairs of M tiles on CTA pairs, then each expert's odd last M tile on one CTA
@@ -716,7 +713,7 @@ moe_status moe_forward(const moe_dims* dims, const moe_opts* opts, const void* X
       g.mlist = w.mleft;
       MOE_TRY_CUDA(launch_gemm(G_DOWN, 256, 4, g, grid_for(std::min<int64_t>(p.E, mtiles) * g.num_n_tiles, sms), st,
                                false));
-    } else if (p.wide_down) {
+    } else if (p.wide_down) {  // over the tile list the up-proj kernel wrote
       g.num_n_tiles = p.d / 256;
       g.mlist = w.mwide;
       MOE_TRY_CUDA(launch_gemm_wide_m(G_DOWN, g, grid_for((mtiles / 2 + p.E) * g.num_n_tiles, sms), st));

@@ -256,51 +256,16 @@ cudaError_t launch_gemm_wide_m(int kind, const GemmParams& p_in, int grid, cudaS
   return cudaErrorInvalidValue;
 }
 
-// List of 256-row tiles of the grouped-M M tiles: for expert e, whose segment
-// holds tiles [offsets[e] / 128, offsets[e + 1] / 128), one entry per pair of
-// consecutive tiles (its first tile, with kWideSecond set) and one for the
-// last tile of an odd count (without the flag); [count, entry...] in expert
-// order.  One block, a thread per expert (E <= 1024).
-__global__ void __launch_bounds__(1024) wide_list_kernel(const int* __restrict__ offsets, int E,
-                                                         int* __restrict__ list) {
-  __shared__ int wsum[32];
-  const int e = threadIdx.x;
-  const int lane = e & 31, w = e >> 5;
+// The 256-row tile list (write_wide_list) as a launch of its own, for the dX~
+// kernel on 256-row tiles (the down-proj's list comes from the up-proj kernel).
+__global__ void __launch_bounds__(32) wide_list_kernel(const int* __restrict__ offsets, int E, int* __restrict__ list) {
   pdl_wait();
-  int t0 = 0, nt = 0;
-  if (e < E) {
-    const int o0 = __ldg(offsets + e), o1 = __ldg(offsets + e + 1);
-    t0 = o0 / kBM;
-    nt = (o1 - o0) / kBM;
-  }
-  const int nw = (nt + 1) >> 1;
-  int sw = nw;  // inclusive scan within the warp
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int a = __shfl_up_sync(0xffffffffu, sw, o);
-    if (lane >= o) sw += a;
-  }
-  if (lane == 31) wsum[w] = sw;
-  __syncthreads();
-  if (w == 0) {  // scan of the warp totals
-    const int nwarps = (int)(blockDim.x >> 5);
-    int a = lane < nwarps ? wsum[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int x = __shfl_up_sync(0xffffffffu, a, o);
-      if (lane >= o) a += x;
-    }
-    wsum[lane] = a;
-  }
-  __syncthreads();
-  const int b = (w > 0 ? wsum[w - 1] : 0) + sw - nw;  // exclusive offset
-  for (int j = 0; j < nw; ++j) list[1 + b + j] = (t0 + 2 * j) | (2 * j + 1 < nt ? kWideSecond : 0);
-  if (e == (int)blockDim.x - 1) list[0] = b + nw;
+  write_wide_list(offsets, E, list, (int)threadIdx.x);
 }
 
 cudaError_t launch_wide_list(const int* offsets, int E, int* list, cudaStream_t s) {
-  if (E < 1 || E > 1024) return cudaErrorInvalidValue;
-  return launch_pdl(wide_list_kernel, dim3(1), dim3(1024), 0, s, offsets, E, list);
+  if (E < 1) return cudaErrorInvalidValue;
+  return launch_pdl(wide_list_kernel, dim3(1), dim3(32), 0, s, offsets, E, list);
 }
 
 // Pair and leftover lists of the grouped-M M tiles: for expert e, whose
