@@ -524,18 +524,20 @@ def main():
     roof["traffic"] = measured_traffic(dom, args.config)
 
     # ---- end-to-end through the public API with host buffers: every step
-    # copies its X and dO from pinned host memory and its O back to pinned host
-    # memory (HostFedRunner overlaps those copies with the kernels)
+    # copies its X and dO from pinned host memory and its per-token outputs O
+    # and dX back to pinned host memory (HostFedRunner overlaps those copies
+    # with the kernels)
     e2e = None
     if not args.no_e2e:
         Xh = X.cpu().pin_memory()
         dOh = dO.cpu().pin_memory()
         Oh = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+        dXh = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
         if ep is None:
             runner = moe.HostFedRunner(layer)
 
             def e2e_step():
-                runner.step(Xh, dOh, Oh, Wr, b, W1, W2)
+                runner.step(Xh, dOh, Oh, Wr, b, W1, W2, dXh=dXh)
                 if world > 1:
                     for g in (layer.dW1, layer.dW2, layer.dWr):
                         dist.all_reduce(g)
@@ -549,7 +551,7 @@ def main():
                 X.copy_(Xh, non_blocking=True)
                 dO.copy_(dOh, non_blocking=True)
                 Oh.copy_(ep.forward(X, Wr, b, W1, W2), non_blocking=True)
-                ep.backward(dO, X, Wr, W1, W2)
+                dXh.copy_(ep.backward(dO, X, Wr, W1, W2)[0], non_blocking=True)
 
         for _ in range(3):
             e2e_step()
@@ -571,8 +573,8 @@ def main():
         e_ms_step = float(ems.item()) / args.steps
         e2e = {"value": round(flops_step * world / (e_ms_step * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(Xh.numel() * 2 + dOh.numel() * 2),
-               "d2h_bytes_per_step": int(Oh.numel() * 2), "ms_per_step": round(e_ms_step, 4),
-               "api": "HostFedRunner.step (pinned host X, dO in; O out)"}
+               "d2h_bytes_per_step": int(Oh.numel() * 2 + dXh.numel() * 2), "ms_per_step": round(e_ms_step, 4),
+               "api": "HostFedRunner.step (pinned host X, dO in; O, dX out)"}
 
     # ---- CPU baseline: the oracle on a bounded sample of the same batch
     # (the device's own input bytes), rank 0 at N=1 only

@@ -445,10 +445,12 @@ class MoELayer:
         moe_forward_mxfp8_q(self.dims, self.opts, X, wq, self.routing, O, self.H, self.ws_fwd_mx, stream)
         return O
 
-    def backward(self, dO, X, Wr, W1, W2, stream=None, grad_events=None):
-        moe_backward(self.dims, self.opts, dO, X, Wr, W1, W2, self.routing, self.H, self.dX, self.dW1, self.dW2,
+    def backward(self, dO, X, Wr, W1, W2, stream=None, grad_events=None, dX=None):
+        """dX: output buffer [T, d] bf16 (default: self.dX)."""
+        dX = self.dX if dX is None else dX
+        moe_backward(self.dims, self.opts, dO, X, Wr, W1, W2, self.routing, self.H, dX, self.dW1, self.dW2,
                      self.dWr if self.opts.router_grad else None, self.ws_bwd, stream, grad_events)
-        return self.dX, self.dW1, self.dW2, self.dWr
+        return dX, self.dW1, self.dW2, self.dWr
 
     def step(self, X, Wr, bias, W1, W2, dO, stream=None, grad_events=None):
         """One pass of the whole path: route (+ rounding), forward, backward."""
@@ -516,11 +518,12 @@ class OverlappedGradReduce:
 class HostFedRunner:
     """Whole steps (route, forward, backward) on batches held in pinned host
     memory.  Each step's inputs X and dO are copied to the device on a copy
-    stream and its output O is copied back on a second copy stream as soon as
-    the forward is done, so the copies of consecutive steps overlap with the
-    kernels.  Device input and output buffers alternate between two sets;
-    events keep a buffer from being overwritten while a step still uses it.
-    Weight gradients stay on the device (layer.dW1, layer.dW2, layer.dWr)."""
+    stream; its per-token outputs O and dX are copied back on a second copy
+    stream, O as soon as the forward is done and dX after the backward, so the
+    copies of consecutive steps overlap with the kernels.  Device input and
+    output buffers alternate between two sets; events keep a buffer from being
+    overwritten while a step or a copy still uses it.  Weight gradients stay
+    on the device (layer.dW1, layer.dW2, layer.dWr)."""
 
     def __init__(self, layer: MoELayer):
         import torch
@@ -531,18 +534,22 @@ class HostFedRunner:
         self.X = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
         self.dO = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
         self.O = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
+        self.dX = [torch.empty(T, d, dtype=bf, device=dev) for _ in range(2)]
         self.h2d = torch.cuda.Stream(device=dev)
         self.d2h = torch.cuda.Stream(device=dev)
         ev = torch.cuda.Event
         self.inputs_ready = [ev(), ev()]
         self.inputs_free = [ev(), ev()]
         self.fwd_done = [ev(), ev()]
+        self.bwd_done = [ev(), ev()]
         self.out_free = [ev(), ev()]
         self.i = 0
 
-    def step(self, Xh, dOh, Oh, Wr, bias, W1, W2):
-        """Enqueue one step; Xh, dOh, Oh are pinned host tensors [T, d] bf16.
-        Returns immediately; call finish() before reading Oh."""
+    def step(self, Xh, dOh, Oh, Wr, bias, W1, W2, dXh=None):
+        """Enqueue one step; Xh, dOh, Oh (and dXh, if given) are pinned host
+        tensors [T, d] bf16.  Returns immediately; call finish() before
+        reading Oh or dXh.  Without dXh the step's dX stays on the device
+        (the buffer of this step's set, self.dX[step % 2])."""
         import torch
         j = self.i & 1
         compute = torch.cuda.current_stream()
@@ -560,9 +567,14 @@ class HostFedRunner:
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.fwd_done[j])
             Oh.copy_(self.O[j], non_blocking=True)
-            self.out_free[j].record(self.d2h)
-        L.backward(self.dO[j], self.X[j], Wr, W1, W2)
+        L.backward(self.dO[j], self.X[j], Wr, W1, W2, dX=self.dX[j])
         self.inputs_free[j].record(compute)
+        self.bwd_done[j].record(compute)
+        with torch.cuda.stream(self.d2h):
+            if dXh is not None:
+                self.d2h.wait_event(self.bwd_done[j])
+                dXh.copy_(self.dX[j], non_blocking=True)
+            self.out_free[j].record(self.d2h)
         self.i += 1
 
     def finish(self):

@@ -227,14 +227,16 @@ def test_host_fed_runner_matches_device_steps():
     Xh = inp["X"].cpu().pin_memory()
     dOh = inp["dO"].cpu().pin_memory()
     outs = [torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-    for Oh in outs:        # three steps in a row, both buffer sets used
-        runner.step(Xh, dOh, Oh, inp["Wr"], inp["bias"], inp["W1"], inp["W2"])
+    grads = [torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    for Oh, dXh in zip(outs, grads):   # three steps in a row, both buffer sets used
+        runner.step(Xh, dOh, Oh, inp["Wr"], inp["bias"], inp["W1"], inp["W2"], dXh=dXh)
     runner.finish()
     torch.cuda.synchronize()
     assert moe.moe_get_status() == (0, 0)
-    for Oh in outs:
+    for Oh, dXh in zip(outs, grads):
         assert torch.equal(Oh, ref.O.cpu())
-    for k in ("dX", "dW1", "dW2", "dWr"):
+        assert torch.equal(dXh, ref.dX.cpu())
+    for k in ("dW1", "dW2", "dWr"):
         assert torch.equal(getattr(layer, k), getattr(ref, k)), k
 
 
