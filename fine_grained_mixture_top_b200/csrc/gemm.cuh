@@ -72,8 +72,14 @@ struct GemmParams {
   // for all of them (the pair kernel's list: the first of each pair of tiles)
   const int* mlist;
   // up-proj only: where the first CTA writes the 256-row tile list of the
-  // grouped-M tiles for the down-proj launch that follows (or null)
+  // grouped-M tiles for the down-proj launch that follows (or null), and the
+  // list's first entry of each expert [E + 1]
   int* wlist;
+  int* wbase;
+  // grouped-M tile order: 0 M-tile-major (the N tiles of one M tile run side
+  // by side), 1 weight-stationary (within an expert, the M tiles of one N
+  // tile run side by side, so each weight tile is read from DRAM once)
+  int wstat;
   const float* rvec;         // DXT router path: Wr transposed [E, d], or null
   const float* rscale;       // DXT router path: dz of each row [R_max] (padding rows unset)
   // MXFP8 kinds.  Scale tiles are 512 bytes: 128 tile rows x 4 scales (one
@@ -169,9 +175,10 @@ constexpr int kWideSecond = 1 << 30;  // 256-row tile list entry flag: the pair'
 // whose padded segment holds M tiles [offsets[e] / 128, offsets[e + 1] / 128),
 // one entry per pair of consecutive tiles (its first tile, with kWideSecond)
 // and one for the last tile of an odd count (without the flag);
-// list = [count, entry...] in expert order.
+// list = [count, entry...] in expert order, and base[e] = the index (after the
+// count) of expert e's first entry, base[E] = the count.
 __device__ __forceinline__ void write_wide_list(const int* __restrict__ offsets, int E, int* __restrict__ list,
-                                                int lane) {
+                                                int* __restrict__ base_out, int lane) {
   int base = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
     const int e = e0 + lane;
@@ -190,9 +197,13 @@ __device__ __forceinline__ void write_wide_list(const int* __restrict__ offsets,
     }
     const int b = base + sw - nw;
     for (int j = 0; j < nw; ++j) list[1 + b + j] = (t0 + 2 * j) | (2 * j + 1 < nt ? kWideSecond : 0);
+    if (e < E) base_out[e] = b;
     base += __shfl_sync(0xffffffffu, sw, 31);
   }
-  if (lane == 0) list[0] = base;
+  if (lane == 0) {
+    list[0] = base;
+    base_out[E] = base;
+  }
 }
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBoxBytes = 64 * 64 * 2;  // one 64x64 bf16 box (MN-major operand)
@@ -278,6 +289,15 @@ __device__ __forceinline__ TileInfo gemm_tile(const GemmParams& p, int tile) {
     t.nt = tile - t.mt * p.num_n_tiles;
     if (p.mlist) t.mt = __ldg(p.mlist + 1 + t.mt);
     t.e = __ldg(p.tile_expert + t.mt);
+    if (p.wstat && !p.mlist) {
+      // the expert's tiles are [t0, t0 + m) x N tiles in either order; walk
+      // its M tiles first within each N tile
+      const int t0 = __ldg(p.offsets + t.e) / kBM;
+      const int m = __ldg(p.offsets + t.e + 1) / kBM - t0;
+      const int l = tile - t0 * p.num_n_tiles;
+      t.nt = l / m;
+      t.mt = t0 + (l - t.nt * m);
+    }
     t.m0 = t.mt * kBM;
     if constexpr (KIND == G_UP || KIND == G_UPQ) t.n0 = t.nt * (BN / 2);
     else t.n0 = t.nt * BN;
@@ -957,7 +977,7 @@ __global__ void __maxnreg__((EpiCfg<KIND, EPI>::kMaxReg))
     if constexpr (KIND == G_UP) {
       // the first CTA's first epilogue warp writes the down-proj's tile list
       // while the first tile's main loop runs
-      if (p.wlist && blockIdx.x == 0 && warp == 2) write_wide_list(p.offsets, p.E, p.wlist, lane);
+      if (p.wlist && blockIdx.x == 0 && warp == 2) write_wide_list(p.offsets, p.E, p.wlist, p.wbase, lane);
     }
     for (int ti = 0; ok; ++ti) {
       TileInfo t;

@@ -125,11 +125,21 @@ __global__ void __maxnreg__((WideMShape<KIND>::kMaxReg)) moe_gm_wide_kernel(cons
   const int ntn = p.num_n_tiles;  // 256-column tiles
   const int num_tiles = __ldg(p.mlist) * ntn;
   const int nkb = (KIND == G_DOWN) ? p.n / kBK : 2 * p.n / kBK;
-  // tile -> (first M tile, whether the second exists, expert, N tile)
+  // tile -> (first M tile, whether the second exists, expert, N tile).  With
+  // p.wstat an expert's tiles, [b, b + w) entries x N tiles, walk its entries
+  // first within each N tile (each weight tile read from DRAM once).
   auto decode = [&](int tile, bool& two) -> TileInfo {
     TileInfo t;
-    const int j = tile / ntn;
+    int j = tile / ntn;
     t.nt = tile - j * ntn;
+    if (p.wstat) {
+      const int e = __ldg(p.tile_expert + (__ldg(p.mlist + 1 + j) & (kWideSecond - 1)));
+      const int b = __ldg(p.wbase + e);
+      const int w = __ldg(p.wbase + e + 1) - b;
+      const int l = tile - b * ntn;
+      t.nt = l / w;
+      j = b + (l - t.nt * w);
+    }
     const int ent = __ldg(p.mlist + 1 + j);
     two = (ent & kWideSecond) != 0;
     t.mt = ent & (kWideSecond - 1);

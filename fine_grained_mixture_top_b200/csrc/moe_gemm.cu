@@ -258,14 +258,15 @@ cudaError_t launch_gemm_wide_m(int kind, const GemmParams& p_in, int grid, cudaS
 
 // The 256-row tile list (write_wide_list) as a launch of its own, for the dX~
 // kernel on 256-row tiles (the down-proj's list comes from the up-proj kernel).
-__global__ void __launch_bounds__(32) wide_list_kernel(const int* __restrict__ offsets, int E, int* __restrict__ list) {
+__global__ void __launch_bounds__(32) wide_list_kernel(const int* __restrict__ offsets, int E, int* __restrict__ list,
+                                                       int* __restrict__ base) {
   pdl_wait();
-  write_wide_list(offsets, E, list, (int)threadIdx.x);
+  write_wide_list(offsets, E, list, base, (int)threadIdx.x);
 }
 
-cudaError_t launch_wide_list(const int* offsets, int E, int* list, cudaStream_t s) {
+cudaError_t launch_wide_list(const int* offsets, int E, int* list, int* base, cudaStream_t s) {
   if (E < 1) return cudaErrorInvalidValue;
-  return launch_pdl(wide_list_kernel, dim3(1), dim3(32), 0, s, offsets, E, list);
+  return launch_pdl(wide_list_kernel, dim3(1), dim3(32), 0, s, offsets, E, list, base);
 }
 
 // Pair and leftover lists of the grouped-M M tiles: for expert e, whose

@@ -64,8 +64,9 @@ cudaError_t launch_gemm_pair_m(int kind, int epi, const GemmParams& p, int max_p
 // the list p.mlist of 256-row tiles; p.num_n_tiles counts 256-column tiles.
 cudaError_t launch_gemm_wide_m(int kind, const GemmParams& p, int grid, cudaStream_t s);
 // List of the grouped-M tiles in 256-row tiles from the segment offsets
-// ([count, entry...]: up to R_max / 256 + E entries after the count).
-cudaError_t launch_wide_list(const int* offsets, int E, int* list, cudaStream_t s);
+// ([count, entry...]: up to R_max / 256 + E entries after the count) and each
+// expert's first entry (base [E + 1]).
+cudaError_t launch_wide_list(const int* offsets, int E, int* list, int* base, cudaStream_t s);
 // Pair list and leftover list of the grouped-M tiles from the segment offsets
 // (each [count, tile...]; `pairs` holds up to R_max / 256 + 1 entries after the
 // count, `left` up to E).

@@ -97,6 +97,22 @@ def test_layer_parity_wide_tiles(name, monkeypatch):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("name,wide,order", [("pairs", "0", "0"), ("bn64", "0", "1"), ("pairs", "1", "1"),
+                                             ("pairs_n640", "1", "0"), ("pairs_n640", "1", "1")])
+def test_layer_parity_both_tile_orders(name, wide, order, monkeypatch):
+    """The grouped-M GEMMs walk an expert's tiles M-tile-major or
+    weight-stationary (its M tiles side by side within each N tile), as the
+    plan picks from the shape; both orders, forced, on the 128-row and the
+    256-row tiles."""
+    monkeypatch.setenv("MOE_TILE_ORDER", order)
+    monkeypatch.setenv("MOE_GM_WIDE", wide)
+    cfg = next(c for c in SHAPES if c.name == name)
+    inp = make_inputs(cfg, "cuda")
+    layer = P.run_layer(inp, cfg.T, cfg.d, cfg.E, cfg.n, cfg.K)
+    _compare_layer(layer, cfg, inp)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("mode", ["0", "1", "2"])
 def test_weight_gradients_under_every_claim_order(mode, monkeypatch):
     """The weight-gradient tiles come from a dynamic queue: largest experts
