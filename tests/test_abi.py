@@ -193,3 +193,43 @@ def test_plan_log_prints_each_shape_once():
     lines = [ln for ln in r.stderr.splitlines() if ln.startswith("moe plan")]
     assert len(lines) == 2, r.stderr
     assert "T=4096 d=1536 E=128 n=256 K=8" in lines[0] and "router tile 384 columns" in lines[0]
+
+
+def test_plan_choices_for_the_benchmark_layers():
+    """The tile plan the measurements chose, per benchmark layer (host only:
+    moe_query_sizes plans without a GPU; MOE_LOG=1 prints the plan): epilogue
+    warps of dH / dX~ / the weight gradients, the 256-row down-proj tiles,
+    the router tile width and the dWr split-K."""
+    import re
+    layers = {  # (T, d, E, n, K): (dH, dX~, dW warps, wide down, router columns, dWr splits)
+        (8192, 7168, 256, 2048, 8): (4, 4, 4, 1, 384, 3),
+        (16384, 1536, 128, 256, 8): (4, 4, 4, 0, 384, 6),
+        (32768, 2048, 128, 768, 8): (4, 4, 4, 1, 384, None),
+        (32768, 2048, 64, 1024, 8): (4, 4, 4, 1, 192, None),
+        (16384, 1536, 256, 128, 8): (4, 8, 4, 0, 384, None),
+        (16384, 1536, 512, 64, 8): (4, 8, 4, 0, 384, None),
+        (512, 128, 16, 64, 2): (8, 8, 4, 0, 192, None),
+    }
+    code = (
+        "import ctypes\n"
+        "from fine_grained_mixture_top_b200 import moe\n"
+        "s = moe.MoeSizes()\n"
+        f"for T, d, E, n, K in {list(layers)!r}:\n"
+        "    assert moe.lib().moe_query_sizes(ctypes.byref(moe.dims_of(T, d, E, n, K)),\n"
+        "                                     ctypes.byref(moe.opts_of()), ctypes.byref(s)) == 0\n"
+    )
+    env = {k: v for k, v in os.environ.items() if not k.startswith("MOE_")}
+    env["MOE_LOG"] = "1"
+    r = subprocess.run([os.sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=120)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stderr.splitlines() if ln.startswith("moe plan")]
+    assert len(lines) == len(layers), r.stderr
+    for ln, ((T, d, E, n, K), want) in zip(lines, layers.items()):
+        assert f"T={T} d={d} E={E} n={n} K={K}" in ln, ln
+        warps = tuple(int(x) for x in re.search(r"epilogue warps dH (\d+) dX~ (\d+) dW (\d+)", ln).groups())
+        wide = int(re.search(r"256-row tiles on one CTA down (\d+)", ln).group(1))
+        rtr = int(re.search(r"router tile (\d+) columns", ln).group(1))
+        splits = int(re.search(r"dWr split-K (\d+) x", ln).group(1))
+        got = warps + (wide, rtr, splits if want[5] is not None else None)
+        assert got == want, (ln, got, want)
