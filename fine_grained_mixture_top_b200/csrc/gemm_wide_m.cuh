@@ -21,8 +21,10 @@
 // Tiles: the list p.mlist holds one entry per pair of consecutive M tiles of
 // an expert, its first tile index with bit 30 set when the second tile
 // exists (an expert with an odd number of M tiles ends with a single tile).
-// Tile j = (entry j / N tiles, N tile), walked round-robin by the CTAs, so
-// neighbouring CTAs share one pair's A rows through L2.
+// The CTAs walk the tiles round-robin, an expert's tiles either entry-major
+// (tile = entry x N tiles + N tile: neighbouring CTAs share one pair's A rows
+// through L2) or, with p.wstat, N-tile-major (neighbouring CTAs share one
+// weight tile, read from DRAM once).
 //
 // Roles:
 //   warp 0 lane 0   TMA loads: A (one or two 128-row boxes) and B

@@ -72,8 +72,11 @@ cudaError_t launch_aggregate_fwd(int T, int d, const int* tok_ptr, const int* pa
 // and the token's dense dz row split into bf16 hi + lo parts for the
 // tensor-core dWr = X^T dz GEMM (layout: group g of 64 experts at columns
 // [128 g, 128 g + 128): hi parts then lo parts).
-__device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, int lane) {
-  const int T = a.T, Epad = a.Epad, nts = a.nds;
+__device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, int sub) {
+  // a segment of a.lanes lanes (a power of two, aligned in the warp) per
+  // token, so that one warp overlaps the dependent loads of several tokens;
+  // every lane runs the shuffles, tokens past T do no memory work
+  const int T = a.T, Epad = a.Epad, nts = a.nds, L = a.lanes;
   const int* __restrict__ tok_ptr = a.tok_ptr;
   const int* __restrict__ pair_row = a.pair_row;
   const int* __restrict__ pair_expert = a.pair_expert;
@@ -81,10 +84,10 @@ __device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, in
   const float* __restrict__ dS_part = a.dS_part;
   float* __restrict__ dz_row = a.dz_row;
   __nv_bfloat16* __restrict__ dz_split = a.dz_split;
-  if (t >= T) return;
-  const int p0 = tok_ptr[t], p1 = tok_ptr[t + 1];
+  const bool live = t < T;
+  const int p0 = live ? tok_ptr[t] : 0, p1 = live ? tok_ptr[t + 1] : 0;
   float inner = 0.f;
-  for (int p = p0 + lane; p < p1; p += 32) {
+  for (int p = p0 + sub; p < p1; p += L) {
     const float* part = dS_part + (size_t)pair_row[p] * nts;
     float ds = 0.f;
     for (int j = 0; j < nts; ++j) ds += part[j];
@@ -94,14 +97,14 @@ __device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, in
     inner += pair_gate[p] * ds;
   }
   if (!a.router) return;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) inner += __shfl_xor_sync(0xffffffffu, inner, o);
+  for (int o = L >> 1; o > 0; o >>= 1) inner += __shfl_xor_sync(0xffffffffu, inner, o);
+  if (live) {  // the dense dz row: zeros, then each pair's hi and lo parts
+    uint4* row4 = reinterpret_cast<uint4*>(dz_split + (size_t)t * 2 * Epad);
+    for (int c = sub; c < Epad / 4; c += L) row4[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
   __syncwarp();
   __nv_bfloat16* row = dz_split + (size_t)t * 2 * Epad;
-  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-  for (int c = lane; c < 2 * Epad; c += 32) row[c] = zero;
-  __syncwarp();
-  for (int p = p0 + lane; p < p1; p += 32) {
+  for (int p = p0 + sub; p < p1; p += L) {
     const int r = pair_row[p];
     const float dz = pair_gate[p] * (dz_row[r] - inner);
     dz_row[r] = dz;
@@ -113,6 +116,7 @@ __device__ __forceinline__ void router_bwd_token(const BwdPrepArgs& a, int t, in
     row[col + 64] = lo;
   }
 }
+
 
 
 // WrT[e, i] = Wr[i, e]
@@ -294,7 +298,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
   pdl_wait();
   const int b = blockIdx.x;
   if (b < a.tok_blocks) {
-    router_bwd_token(a, b * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+    const int per_warp = 32 / a.lanes;
+    const int lane = threadIdx.x & 31;
+    router_bwd_token(a, (b * 8 + (threadIdx.x >> 5)) * per_warp + lane / a.lanes, lane & (a.lanes - 1));
     return;
   }
   if (b < a.tok_blocks + a.tr_blocks) {
@@ -309,7 +315,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
 
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a0, cudaStream_t s) {
   BwdPrepArgs a = a0;
-  a.tok_blocks = (a.router || a.pair_dS) ? (a.T + 7) / 8 : 0;
+  // lanes per token: the power of two at or above K, at most 32 (tokens that
+  // gained pairs in token rounding loop over them)
+  a.lanes = 1;
+  while (a.lanes < a.K && a.lanes < 32) a.lanes <<= 1;
+  const int tok_per_block = 8 * (32 / a.lanes);
+  a.tok_blocks = (a.router || a.pair_dS) ? (a.T + tok_per_block - 1) / tok_per_block : 0;
   a.tr_blocks = a.router ? ((a.E + 31) / 32) * ((a.d + 31) / 32) : 0;
   launch_pdl(bwd_prep_kernel, dim3(a.tok_blocks + a.tr_blocks + 1), dim3(256), 0, s, a);
   return cudaGetLastError();

@@ -987,6 +987,7 @@ moe_status moe_backward_ev(const moe_dims* dims, const moe_opts* opts, const voi
     a.E = p.E;
     a.Epad = p.Epad;
     a.nds = p.nds;
+    a.K = p.K;
     a.router = rg ? 1 : 0;
     a.tok_ptr = rt->tok_ptr;
     a.pair_row = rt->pair_row;

@@ -151,7 +151,8 @@ struct BwdPrepArgs {
   int* expert_order;           // [E]
   int* sched;                  // [16] weight-gradient tile counters, zeroed here
   float* pair_dS;              // [P] dS of each pair, or null
-  int tok_blocks, tr_blocks;   // set by the launcher
+  int K;                       // experts per token (pairs per token before rounding)
+  int lanes, tok_blocks, tr_blocks;  // set by the launcher: lanes per token, block counts
 };
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t s);
 cudaError_t launch_dwr_reduce(int d, int E, int Epad, int splits, const float* part, float* dWr, cudaStream_t s);
